@@ -1,0 +1,20 @@
+"""CPU oracle for the SA compression step (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+and reference legs may import this package.  It shares no code with the CUDA
+library and never calls it.
+"""
+
+from .sa_oracle import (  # noqa: F401
+    DEFAULT_STEPS,
+    affinity,
+    aggregate,
+    mass_normalised,
+    project_keys,
+    project_prototypes,
+    prototype_mass,
+    prototype_softmax,
+    sa_batch,
+    sa_user,
+)
+from .brute import sa_user_bruteforce  # noqa: F401
