@@ -1,0 +1,184 @@
+/*
+ * sa.h -- C ABI of the Sketch Attention (SA) compression library (libsa.so).
+ *
+ * What it computes.  One SA layer of SequenceO1, as section 2.1 ("Sketch
+ * Attention") of the reading notes "SequenceO1：用可缓存的低秩草图实现端到端十万级用户历史建模"
+ * defines it.  For each user b with history X_b (n_b x d, one row per
+ * behaviour), shared prototypes P (k x d) and projections W_Q, W_K (d x d):
+ *
+ *     S   = (P W_Q)(X_b W_K)^T * scale                 k x n_b affinities
+ *     A   = softmax of S over the PROTOTYPE axis j      every column sums to 1
+ *     X~_b = A X_b                                      k x d sketch, no value projection
+ *     m_b  = A 1                                        k per-prototype masses
+ *
+ * (sum_j m_bj = n_b; X~_bj / m_bj is the mass-normalised sketch.)  The
+ * library evaluates S through Q' = P W_Q W_K^T * scale, the rearrangement
+ * section 1 of the same notes describes for single-query cross-attention,
+ * so the key projection X W_K is never formed; and it fuses affinity,
+ * stable softmax and aggregation in one pass over X without writing the
+ * k x n matrices to memory, as section 2.4 describes for FlashSA, over
+ * ragged batches.
+ *
+ * Conventions.
+ *  - Device pointers are CUDA device memory of the current device (the one
+ *    current when the query was prepared).  Host pointers are host memory.
+ *  - All arrays are dense and row-major.  bf16 data is IEEE bfloat16 bit
+ *    patterns (uint16); fp32 data is IEEE binary32.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Device-side work is enqueued on it and runs asynchronously unless an
+ *    entry point says otherwise.
+ *  - The caller owns every buffer it passes; the library owns only what is
+ *    inside an sa_query (freed by sa_sketch_free).
+ *  - Host-side argument errors are reported immediately and nothing is
+ *    enqueued.  Offsets live on the device, so their validity is checked on
+ *    the device: a bad offsets array never causes an out-of-bounds access,
+ *    but it makes the outputs unspecified and raises a device flag that
+ *    sa_read_device_status reports.
+ */
+#ifndef SA_H_
+#define SA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sa_status {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned buffer, wrong device */
+  SA_ERR_UNSUPPORTED = 2,  /* shape/dtype/GPU without a kernel in this build */
+  SA_ERR_WORKSPACE = 3,    /* workspace smaller than sa_workspace_bytes() */
+  SA_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+  SA_ERR_DEVICE_FLAG = 5   /* a kernel flagged bad offsets or a timed-out wait */
+} sa_status;
+
+typedef enum sa_dtype {
+  SA_BF16 = 0, /* bf16 inputs, tensor-core pass, fp32 accumulation */
+  SA_FP32 = 1  /* fp32 inputs, CUDA-core pass, fp64 accumulation */
+} sa_dtype;
+
+/* Device flag bits reported through sa_read_device_status. */
+#define SA_DEVFLAG_OFFSET0_NONZERO 1u  /* offsets[0] != 0 */
+#define SA_DEVFLAG_OFFSETS_DECREASE 2u /* offsets[b] > offsets[b+1] for some b */
+#define SA_DEVFLAG_OFFSET_LAST 4u      /* offsets[batch] != total_rows */
+#define SA_DEVFLAG_TIMEOUT 8u          /* a kernel's bounded wait gave up */
+
+/* Opaque handle: the precomputed query Q' for one weight set. */
+typedef struct sa_query_s* sa_query;
+
+/*
+ * sa_prepare_query -- precompute Q' = P W_Q W_K^T * scale (times log2 e) for
+ * one set of SA parameters (section 2.1: P^(0) in R^{k x d}, W_Q, W_K in
+ * R^{d x d}; section 1: the query/key rearrangement).
+ *
+ *   P     device, k x d, dtype          shared prototypes P^(0)
+ *   W_Q   device, d x d, dtype          query projection
+ *   W_K   device, d x d, dtype          key projection
+ *   k     1 <= k <= 256                 number of prototypes
+ *   d     64, 128 or 256                embedding width
+ *   scale finite                        affinity scale (1/sqrt(d) in the paper's setting)
+ *   dtype SA_BF16 or SA_FP32            element type of P, W_Q, W_K and of X later
+ *   stream                              the precompute kernel runs on it
+ *   out   host; receives the handle
+ *
+ * Allocates device memory (cudaMalloc) for Q'.  P, W_Q and W_K are read by
+ * a kernel enqueued on `stream`; they must stay alive until it completes.
+ * Returns SA_ERR_UNSUPPORTED for bf16 shapes without a tensor-core kernel
+ * (currently bf16 needs k <= 128 for d = 64/128 and k <= 64 for d = 256) or
+ * for a GPU other than sm_100.
+ */
+sa_status sa_prepare_query(const void* P, const void* W_Q, const void* W_K, int k, int d,
+                           float scale, sa_dtype dtype, void* stream, sa_query* out);
+
+/* Releases a query and its device memory (synchronises with the device).
+ * NULL is a no-op. */
+void sa_sketch_free(sa_query q);
+
+/* Bytes of device workspace sa_sketch_forward needs for a batch of `batch`
+ * users and `total_rows` rows.  Independent of the batch size beyond a fixed
+ * bound (it scales with the number of SMs, not with the number of users). */
+size_t sa_workspace_bytes(sa_query q, int64_t batch, int64_t total_rows);
+
+/*
+ * sa_sketch_forward -- one SA layer over a ragged batch (section 2.1; ragged
+ * batches and fused tiling: section 2.4).
+ *
+ *   q           prepared query
+ *   X           device, total_rows x d, q's dtype; user b owns rows
+ *               [offsets[b], offsets[b+1]).  16-byte aligned.
+ *   offsets     device, int64, batch + 1 entries: offsets[0] == 0,
+ *               non-decreasing, offsets[batch] == total_rows.  No padding:
+ *               rows outside a user's range never contribute to it
+ *               (section 3.1: padding must not receive mass).
+ *   batch       number of users B >= 0
+ *   total_rows  N >= 0, < 2^31 - 256
+ *   X_tilde     device out, B x k x d fp32 (16-byte aligned): the sketches
+ *   mass        device out, B x k fp32: m_bj = sum_i A_ji
+ *   workspace   device, >= sa_workspace_bytes(q, B, N) bytes, 256-byte
+ *               aligned; no initial contents needed; one call at a time
+ *   stream      work is enqueued here; outputs are ready when it is done
+ *
+ * A user with no rows gets X~ = 0 and m = 0.  Results are bitwise
+ * reproducible for the same inputs on the same GPU model.
+ */
+sa_status sa_sketch_forward(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
+                            int64_t total_rows, float* X_tilde, float* mass, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
+ * The two kernels sa_sketch_forward enqueues, for callers that schedule (or
+ * time) them separately.  sa_sketch_partials runs the fused pass over X,
+ * writing users that lie inside one CTA's row range to the outputs and the
+ * others to partial slots in the workspace; sa_sketch_finalize then sums the
+ * partial slots in a fixed order, zero-fills empty users and validates the
+ * offsets.  Calling both, in this order, on one stream with the same
+ * arguments equals sa_sketch_forward.
+ */
+sa_status sa_sketch_partials(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
+                             int64_t total_rows, float* X_tilde, float* mass, void* workspace,
+                             size_t workspace_bytes, void* stream);
+sa_status sa_sketch_finalize(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
+                             int64_t total_rows, float* X_tilde, float* mass, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
+ * sa_sketch_forward_host -- the same layer on HOST buffers (end-to-end use).
+ *
+ *   X_host        host, total_rows x d, q's dtype (pinned memory copies fastest)
+ *   offsets_host  host, batch + 1 int64 (validated on the host before any copy)
+ *   X_tilde_host  host out, B x k x d fp32
+ *   mass_host     host out, B x k fp32
+ *   device_buffer device, >= sa_host_path_device_bytes(q, B, N), 256-byte aligned
+ *
+ * Copies X and the offsets to device_buffer, runs sa_sketch_forward there,
+ * copies the results back and synchronises `stream` before returning.
+ */
+size_t sa_host_path_device_bytes(sa_query q, int64_t batch, int64_t total_rows);
+sa_status sa_sketch_forward_host(sa_query q, const void* X_host, const int64_t* offsets_host,
+                                 int64_t batch, int64_t total_rows, float* X_tilde_host,
+                                 float* mass_host, void* device_buffer,
+                                 size_t device_buffer_bytes, void* stream);
+
+/*
+ * sa_read_device_status -- synchronises `stream`, reads the device flags of
+ * the last call that used `workspace` and clears them.  Returns SA_OK if no
+ * flag was set, SA_ERR_DEVICE_FLAG otherwise (with the SA_DEVFLAG_* bits in
+ * *flags_out if it is not NULL), SA_ERR_CUDA if the copy failed.
+ */
+sa_status sa_read_device_status(void* workspace, size_t workspace_bytes, void* stream,
+                                uint32_t* flags_out);
+
+/* Static description of a status code. */
+const char* sa_status_string(sa_status s);
+
+/* Shape of a prepared query: k, d, dtype, and the padded prototype count
+ * the tensor-core pass uses (0 for fp32). */
+sa_status sa_query_info(sa_query q, int* k, int* d, int* dtype, int* k_pad);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA_H_ */

@@ -1,0 +1,16 @@
+"""B200-native Sketch Attention (SA) compression.
+
+The compute path is libsa.so (CUDA, sm_100a), declared in include/sa.h; this
+package holds its sources (csrc/), its build script (build.py) and a ctypes
+binding (binding.py).  Importing the package does not load the library;
+``SketchQuery`` does, and fails loudly if it is missing.
+"""
+
+from .binding import (  # noqa: F401
+    SA_BF16,
+    SA_FP32,
+    SAError,
+    SketchQuery,
+    load_library,
+    read_device_status,
+)

@@ -1,0 +1,251 @@
+"""ctypes binding of libsa.so (argument marshalling only).
+
+Every step of the SA layer runs in the CUDA library; this module turns torch
+tensors and streams into the plain pointers and sizes of the C ABI declared
+in include/sa.h.  PyTorch provides device memory and streams.  There is no
+fallback: if libsa.so is missing or a call fails, an exception is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import numpy as np
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libsa.so")
+
+SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA, \
+    SA_ERR_DEVICE_FLAG = range(6)
+SA_BF16, SA_FP32 = 0, 1
+DEVFLAG_OFFSET0_NONZERO, DEVFLAG_OFFSETS_DECREASE, DEVFLAG_OFFSET_LAST, DEVFLAG_TIMEOUT = \
+    1, 2, 4, 8
+
+# name -> (restype, argtypes); mirrors include/sa.h
+_vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, \
+    ctypes.c_float
+_FWD_ARGS = [_vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _sz, _vp]
+SIGNATURES = {
+    "sa_prepare_query": (_i32, [_vp, _vp, _vp, _i32, _i32, _f32, _i32, _vp,
+                                ctypes.POINTER(_vp)]),
+    "sa_sketch_free": (None, [_vp]),
+    "sa_workspace_bytes": (_sz, [_vp, _i64, _i64]),
+    "sa_sketch_forward": (_i32, _FWD_ARGS),
+    "sa_sketch_partials": (_i32, _FWD_ARGS),
+    "sa_sketch_finalize": (_i32, _FWD_ARGS),
+    "sa_host_path_device_bytes": (_sz, [_vp, _i64, _i64]),
+    "sa_sketch_forward_host": (_i32, _FWD_ARGS),
+    "sa_read_device_status": (_i32, [_vp, _sz, _vp, ctypes.POINTER(ctypes.c_uint32)]),
+    "sa_status_string": (ctypes.c_char_p, [_i32]),
+    "sa_query_info": (_i32, [_vp, ctypes.POINTER(_i32), ctypes.POINTER(_i32),
+                             ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+class SAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libsa.so (built in-tree) and declares its signatures."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m sketch_attention_compression_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return load_library().sa_status_string(status).decode()
+    except Exception:  # pragma: no cover - only for messages
+        return "unknown"
+
+
+def _check(status: int, what: str) -> None:
+    if status != SA_OK:
+        raise SAError(status, what)
+
+
+def _torch():
+    import torch  # deferred: the binding is importable without torch for the ABI checks
+    return torch
+
+
+def _stream_handle(stream) -> int:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t == torch.bfloat16:
+        return SA_BF16
+    if t == torch.float32:
+        return SA_FP32
+    raise TypeError(f"unsupported dtype {t}; use torch.bfloat16 or torch.float32")
+
+
+def _dev_ptr(t, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class SketchQuery:
+    """A prepared SA query: Q' = P W_Q W_K^T * scale for one weight set.
+
+    P (k, d), W_Q and W_K (d, d) are CUDA tensors of one dtype (bf16 or fp32).
+    """
+
+    def __init__(self, P, W_Q, W_K, scale: float, stream=None):
+        lib = load_library()
+        if P.dtype != W_Q.dtype or P.dtype != W_K.dtype:
+            raise TypeError("P, W_Q and W_K must share a dtype")
+        self.k, self.d = int(P.shape[0]), int(P.shape[1])
+        if tuple(W_Q.shape) != (self.d, self.d) or tuple(W_K.shape) != (self.d, self.d):
+            raise ValueError("W_Q and W_K must be d x d")
+        self.dtype = P.dtype
+        self.device = P.device
+        handle = ctypes.c_void_p()
+        st = lib.sa_prepare_query(_dev_ptr(P, "P"), _dev_ptr(W_Q, "W_Q"), _dev_ptr(W_K, "W_K"),
+                                  self.k, self.d, float(scale), _dtype_code(P.dtype),
+                                  ctypes.c_void_p(_stream_handle(stream)), ctypes.byref(handle))
+        _check(st, "sa_prepare_query")
+        self._h = handle
+        self._lib = lib
+        k, d, dt, kp = (ctypes.c_int() for _ in range(4))
+        _check(lib.sa_query_info(self._h, ctypes.byref(k), ctypes.byref(d), ctypes.byref(dt),
+                                 ctypes.byref(kp)), "sa_query_info")
+        self.k_pad = kp.value
+
+    # -- sizes -------------------------------------------------------------
+    def workspace_bytes(self, batch: int, total_rows: int) -> int:
+        return int(self._lib.sa_workspace_bytes(self._h, batch, total_rows))
+
+    def host_path_device_bytes(self, batch: int, total_rows: int) -> int:
+        return int(self._lib.sa_host_path_device_bytes(self._h, batch, total_rows))
+
+    def new_workspace(self, batch: int, total_rows: int):
+        torch = _torch()
+        return torch.empty(self.workspace_bytes(batch, total_rows), dtype=torch.uint8,
+                           device=self.device)
+
+    # -- device path -------------------------------------------------------
+    def _args(self, X, offsets, X_tilde, mass, workspace):
+        torch = _torch()
+        if X.dtype != self.dtype:
+            raise TypeError(f"X dtype {X.dtype} != query dtype {self.dtype}")
+        if X.dim() != 2 or X.shape[1] != self.d:
+            raise ValueError("X must be (N, d)")
+        if offsets.dtype != torch.int64 or offsets.dim() != 1:
+            raise TypeError("offsets must be a 1-D int64 tensor")
+        B = int(offsets.shape[0]) - 1
+        N = int(X.shape[0])
+        if X_tilde is None:
+            X_tilde = torch.empty((B, self.k, self.d), dtype=torch.float32, device=X.device)
+        if mass is None:
+            mass = torch.empty((B, self.k), dtype=torch.float32, device=X.device)
+        if workspace is None:
+            workspace = self.new_workspace(B, N)
+        xp = ctypes.c_void_p(X.data_ptr()) if N > 0 else ctypes.c_void_p(0)
+        if N > 0:
+            _dev_ptr(X, "X")
+        args = (xp, _dev_ptr(offsets, "offsets"), B, N, _dev_ptr(X_tilde, "X_tilde"),
+                _dev_ptr(mass, "mass"), _dev_ptr(workspace, "workspace"),
+                int(workspace.numel() * workspace.element_size()))
+        return args, X_tilde, mass, workspace
+
+    def forward(self, X, offsets, X_tilde=None, mass=None, workspace=None, stream=None,
+                check: bool = False) -> Tuple[object, object]:
+        """X~ (B, k, d) and m (B, k) for the ragged batch (X (N, d), offsets (B+1,))."""
+        args, X_tilde, mass, workspace = self._args(X, offsets, X_tilde, mass, workspace)
+        sh = ctypes.c_void_p(_stream_handle(stream))
+        _check(self._lib.sa_sketch_forward(self._h, *args, sh), "sa_sketch_forward")
+        if check:
+            read_device_status(workspace, stream)
+        return X_tilde, mass
+
+    def partials(self, X, offsets, X_tilde, mass, workspace, stream=None) -> None:
+        args, *_ = self._args(X, offsets, X_tilde, mass, workspace)
+        _check(self._lib.sa_sketch_partials(self._h, *args, ctypes.c_void_p(_stream_handle(stream))),
+               "sa_sketch_partials")
+
+    def finalize(self, X, offsets, X_tilde, mass, workspace, stream=None) -> None:
+        args, *_ = self._args(X, offsets, X_tilde, mass, workspace)
+        _check(self._lib.sa_sketch_finalize(self._h, *args, ctypes.c_void_p(_stream_handle(stream))),
+               "sa_sketch_finalize")
+
+    # -- host path ---------------------------------------------------------
+    def forward_host(self, X_host, offsets_host: np.ndarray, device_buffer=None, stream=None,
+                     out_x: Optional[np.ndarray] = None, out_m: Optional[np.ndarray] = None):
+        """Same layer on host arrays.  X_host: a CPU torch tensor (bf16/fp32,
+        ideally pinned) or a float32 numpy array for fp32 queries; offsets a
+        numpy int64 array.  Returns numpy X~ (B, k, d) and m (B, k)."""
+        torch = _torch()
+        offsets_host = np.ascontiguousarray(offsets_host, dtype=np.int64)
+        B = len(offsets_host) - 1
+        if isinstance(X_host, np.ndarray):
+            if self.dtype != torch.float32:
+                raise TypeError("numpy X is only accepted for fp32 queries")
+            X_host = torch.from_numpy(np.ascontiguousarray(X_host, dtype=np.float32))
+        if X_host.is_cuda or X_host.dtype != self.dtype or not X_host.is_contiguous():
+            raise ValueError("X_host must be a contiguous CPU tensor of the query dtype")
+        N = int(X_host.shape[0])
+        if device_buffer is None:
+            device_buffer = torch.empty(self.host_path_device_bytes(B, N), dtype=torch.uint8,
+                                        device=self.device)
+        if out_x is None:
+            out_x = np.empty((B, self.k, self.d), dtype=np.float32)
+        if out_m is None:
+            out_m = np.empty((B, self.k), dtype=np.float32)
+        st = self._lib.sa_sketch_forward_host(
+            self._h, ctypes.c_void_p(X_host.data_ptr() if N > 0 else 0),
+            offsets_host.ctypes.data_as(ctypes.c_void_p), B, N,
+            out_x.ctypes.data_as(ctypes.c_void_p), out_m.ctypes.data_as(ctypes.c_void_p),
+            _dev_ptr(device_buffer, "device_buffer"),
+            int(device_buffer.numel()), ctypes.c_void_p(_stream_handle(stream)))
+        _check(st, "sa_sketch_forward_host")
+        return out_x, out_m
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self._lib.sa_sketch_free(self._h)
+            self._h = None
+
+    def __del__(self):  # pragma: no cover
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def read_device_status(workspace, stream=None) -> int:
+    """Synchronises the stream, returns the device flag bits of the last call
+    on `workspace` (0 when clean) and clears them."""
+    lib = load_library()
+    flags = ctypes.c_uint32(0)
+    st = lib.sa_read_device_status(ctypes.c_void_p(workspace.data_ptr()),
+                                   int(workspace.numel() * workspace.element_size()),
+                                   ctypes.c_void_p(_stream_handle(stream)), ctypes.byref(flags))
+    if st not in (SA_OK, SA_ERR_DEVICE_FLAG):
+        _check(st, "sa_read_device_status")
+    return int(flags.value)

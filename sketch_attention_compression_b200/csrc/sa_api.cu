@@ -1,0 +1,339 @@
+// C-ABI layer of libsa.so: argument checks, workspace layout, tensor maps
+// and kernel launches.  See include/sa.h for the contract of each entry.
+#include <math.h>
+#include <string.h>
+
+#include <new>
+
+#include "../../include/sa.h"
+#include "sa_internal.h"
+
+struct sa_query_s {
+  int device;
+  int sms;
+  int k;
+  int d;
+  int k_pad;  // prototype rows of the bf16 Q' copy (multiple of 64), 0 for fp32
+  sa_dtype dtype;
+  float* q_f32;      // [k][d]
+  uint16_t* q_bf16;  // [k_pad][d], rows >= k zero
+  CUtensorMap tmap_q;
+};
+
+namespace {
+
+using sa::PassArgs;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows][cols] array, boxes of
+// 64 columns (128 bytes) x box_rows rows, 128-byte swizzle, zero fill.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+constexpr int64_t kMaxRows = (int64_t{1} << 31) - 256;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int64_t grid_for(const sa_query_s* q, int64_t total_rows) {
+  const int64_t T = sa::tiles_of(total_rows);
+  int64_t G = T < q->sms ? T : q->sms;
+  return G < 1 ? 1 : G;
+}
+
+struct WsLayout {
+  size_t part_x_off, part_m_off, total;
+};
+
+WsLayout ws_layout(const sa_query_s* q, int64_t total_rows) {
+  const size_t G = static_cast<size_t>(grid_for(q, total_rows));
+  WsLayout l;
+  l.part_x_off = sa::kWsHeaderBytes;
+  l.part_m_off = round_up(l.part_x_off + 2 * G * q->k * q->d * sizeof(float), 256);
+  l.total = round_up(l.part_m_off + 2 * G * q->k * sizeof(float), 256);
+  return l;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool same_device(const sa_query_s* q) {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess && dev == q->device;
+}
+
+enum class Phase { kBoth, kPartials, kFinalize };
+
+sa_status run(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
+              int64_t total_rows, float* X_tilde, float* mass, void* workspace,
+              size_t workspace_bytes, void* stream, Phase phase) {
+  if (q == nullptr) return SA_ERR_INVALID_ARG;
+  if (batch < 0 || total_rows < 0 || total_rows > kMaxRows) return SA_ERR_INVALID_ARG;
+  if (batch == 0) return total_rows == 0 ? SA_OK : SA_ERR_INVALID_ARG;
+  if (offsets == nullptr || X_tilde == nullptr || mass == nullptr || workspace == nullptr)
+    return SA_ERR_INVALID_ARG;
+  if (total_rows > 0 && X == nullptr) return SA_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(X_tilde, 16) || !aligned(mass, 4) || !aligned(offsets, 8) ||
+      !aligned(workspace, 256))
+    return SA_ERR_INVALID_ARG;
+  if (!same_device(q)) return SA_ERR_INVALID_ARG;
+  const WsLayout l = ws_layout(q, total_rows);
+  if (workspace_bytes < l.total) return SA_ERR_WORKSPACE;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  PassArgs a;
+  a.offsets = offsets;
+  a.batch = batch;
+  a.total_rows = total_rows;
+  a.tiles = sa::tiles_of(total_rows);
+  a.k = q->k;
+  a.d = q->d;
+  a.out_x = X_tilde;
+  a.out_m = mass;
+  a.part_x = reinterpret_cast<float*>(ws + l.part_x_off);
+  a.part_m = reinterpret_cast<float*>(ws + l.part_m_off);
+  a.header = reinterpret_cast<sa::WsHeader*>(ws);
+  const int G = static_cast<int>(grid_for(q, total_rows));
+
+  if (phase != Phase::kFinalize) {
+    cudaError_t err;
+    if (q->dtype == SA_BF16) {
+      CUtensorMap tmx;
+      // A zero-row tensor map is not encodable; with N == 0 the kernel
+      // issues no loads, so Q' stands in as a valid dummy.
+      const bool ok = total_rows > 0
+                          ? make_tmap_bf16(&tmx, X, static_cast<uint64_t>(total_rows),
+                                           static_cast<uint64_t>(q->d), sa::kTileRows)
+                          : make_tmap_bf16(&tmx, q->q_bf16, static_cast<uint64_t>(q->k_pad),
+                                           static_cast<uint64_t>(q->d), 64);
+      if (!ok) return SA_ERR_CUDA;
+      err = sa::launch_fused_bf16(tmx, q->tmap_q, q->k_pad, a, G, st);
+    } else {
+      err = sa::launch_simt_fp32(q->q_f32, static_cast<const float*>(X), a, G, st);
+    }
+    if (err != cudaSuccess) return SA_ERR_CUDA;
+  }
+  if (phase != Phase::kPartials) {
+    if (sa::launch_finalize(a, G, st) != cudaSuccess) return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sa_status_string(sa_status s) {
+  switch (s) {
+    case SA_OK: return "ok";
+    case SA_ERR_INVALID_ARG: return "invalid argument";
+    case SA_ERR_UNSUPPORTED: return "unsupported shape, dtype or GPU";
+    case SA_ERR_WORKSPACE: return "workspace too small";
+    case SA_ERR_CUDA: return "CUDA error";
+    case SA_ERR_DEVICE_FLAG: return "device flagged bad offsets or a timed-out wait";
+  }
+  return "unknown status";
+}
+
+sa_status sa_prepare_query(const void* P, const void* W_Q, const void* W_K, int k, int d,
+                           float scale, sa_dtype dtype, void* stream, sa_query* out) {
+  if (out == nullptr) return SA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (P == nullptr || W_Q == nullptr || W_K == nullptr) return SA_ERR_INVALID_ARG;
+  if (k < 1 || k > 256 || !(d == 64 || d == 128 || d == 256) || !isfinite(scale))
+    return SA_ERR_INVALID_ARG;
+  if (dtype != SA_BF16 && dtype != SA_FP32) return SA_ERR_INVALID_ARG;
+  const size_t elem = dtype == SA_BF16 ? 2 : 4;
+  if (!aligned(P, elem) || !aligned(W_Q, elem) || !aligned(W_K, elem)) return SA_ERR_INVALID_ARG;
+
+  int dev = 0, major = 0, minor = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return SA_ERR_CUDA;
+  if (major != 10 || minor != 0) return SA_ERR_UNSUPPORTED;  // built for sm_100a only
+
+  int k_pad = 0;
+  if (dtype == SA_BF16) {
+    k_pad = k <= 64 ? 64 : (k <= 128 ? 128 : 256);
+    if (!sa::fused_bf16_supported(d, k_pad)) return SA_ERR_UNSUPPORTED;
+  }
+
+  sa_query_s* q = new (std::nothrow) sa_query_s;
+  if (q == nullptr) return SA_ERR_CUDA;
+  memset(q, 0, sizeof(*q));
+  q->device = dev;
+  q->sms = sms;
+  q->k = k;
+  q->d = d;
+  q->k_pad = k_pad;
+  q->dtype = dtype;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  bool ok = cudaMalloc(&q->q_f32, static_cast<size_t>(k) * d * sizeof(float)) == cudaSuccess;
+  if (ok && dtype == SA_BF16) {
+    const size_t qb = static_cast<size_t>(k_pad) * d * sizeof(uint16_t);
+    ok = cudaMalloc(&q->q_bf16, qb) == cudaSuccess && cudaMemsetAsync(q->q_bf16, 0, qb, st) == cudaSuccess;
+    ok = ok && make_tmap_bf16(&q->tmap_q, q->q_bf16, static_cast<uint64_t>(k_pad),
+                              static_cast<uint64_t>(d), static_cast<uint32_t>(k_pad));
+  }
+  ok = ok && sa::launch_prepare_query(P, W_Q, W_K, k, d, static_cast<double>(scale),
+                                      dtype == SA_BF16, q->q_f32, q->q_bf16, st) == cudaSuccess;
+  if (!ok) {
+    cudaFree(q->q_f32);
+    cudaFree(q->q_bf16);
+    delete q;
+    return SA_ERR_CUDA;
+  }
+  *out = q;
+  return SA_OK;
+}
+
+void sa_sketch_free(sa_query q) {
+  if (q == nullptr) return;
+  cudaFree(q->q_f32);
+  cudaFree(q->q_bf16);
+  delete q;
+}
+
+sa_status sa_query_info(sa_query q, int* k, int* d, int* dtype, int* k_pad) {
+  if (q == nullptr) return SA_ERR_INVALID_ARG;
+  if (k) *k = q->k;
+  if (d) *d = q->d;
+  if (dtype) *dtype = static_cast<int>(q->dtype);
+  if (k_pad) *k_pad = q->k_pad;
+  return SA_OK;
+}
+
+size_t sa_workspace_bytes(sa_query q, int64_t batch, int64_t total_rows) {
+  (void)batch;
+  if (q == nullptr || total_rows < 0) return 0;
+  return ws_layout(q, total_rows).total;
+}
+
+sa_status sa_sketch_forward(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
+                            int64_t total_rows, float* X_tilde, float* mass, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  return run(q, X, offsets, batch, total_rows, X_tilde, mass, workspace, workspace_bytes, stream,
+             Phase::kBoth);
+}
+
+sa_status sa_sketch_partials(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
+                             int64_t total_rows, float* X_tilde, float* mass, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  return run(q, X, offsets, batch, total_rows, X_tilde, mass, workspace, workspace_bytes, stream,
+             Phase::kPartials);
+}
+
+sa_status sa_sketch_finalize(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
+                             int64_t total_rows, float* X_tilde, float* mass, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  return run(q, X, offsets, batch, total_rows, X_tilde, mass, workspace, workspace_bytes, stream,
+             Phase::kFinalize);
+}
+
+size_t sa_host_path_device_bytes(sa_query q, int64_t batch, int64_t total_rows) {
+  if (q == nullptr || batch < 0 || total_rows < 0) return 0;
+  const size_t elem = q->dtype == SA_BF16 ? 2 : 4;
+  size_t s = round_up(static_cast<size_t>(total_rows) * q->d * elem, 256);
+  s += round_up(static_cast<size_t>(batch + 1) * sizeof(int64_t), 256);
+  s += round_up(static_cast<size_t>(batch) * q->k * q->d * sizeof(float), 256);
+  s += round_up(static_cast<size_t>(batch) * q->k * sizeof(float), 256);
+  s += ws_layout(q, total_rows).total;
+  return s;
+}
+
+sa_status sa_sketch_forward_host(sa_query q, const void* X_host, const int64_t* offsets_host,
+                                 int64_t batch, int64_t total_rows, float* X_tilde_host,
+                                 float* mass_host, void* device_buffer,
+                                 size_t device_buffer_bytes, void* stream) {
+  if (q == nullptr || offsets_host == nullptr || batch < 0 || total_rows < 0 ||
+      total_rows > kMaxRows)
+    return SA_ERR_INVALID_ARG;
+  if (batch == 0) return total_rows == 0 ? SA_OK : SA_ERR_INVALID_ARG;
+  if (X_tilde_host == nullptr || mass_host == nullptr || device_buffer == nullptr ||
+      (total_rows > 0 && X_host == nullptr) || !aligned(device_buffer, 256))
+    return SA_ERR_INVALID_ARG;
+  if (offsets_host[0] != 0 || offsets_host[batch] != total_rows) return SA_ERR_INVALID_ARG;
+  for (int64_t b = 0; b < batch; ++b)
+    if (offsets_host[b] > offsets_host[b + 1]) return SA_ERR_INVALID_ARG;
+  if (device_buffer_bytes < sa_host_path_device_bytes(q, batch, total_rows))
+    return SA_ERR_WORKSPACE;
+
+  const size_t elem = q->dtype == SA_BF16 ? 2 : 4;
+  const size_t x_bytes = static_cast<size_t>(total_rows) * q->d * elem;
+  const size_t o_bytes = static_cast<size_t>(batch + 1) * sizeof(int64_t);
+  const size_t xt_bytes = static_cast<size_t>(batch) * q->k * q->d * sizeof(float);
+  const size_t m_bytes = static_cast<size_t>(batch) * q->k * sizeof(float);
+  uint8_t* p = static_cast<uint8_t*>(device_buffer);
+  void* x_dev = p;
+  p += round_up(x_bytes, 256);
+  int64_t* o_dev = reinterpret_cast<int64_t*>(p);
+  p += round_up(o_bytes, 256);
+  float* xt_dev = reinterpret_cast<float*>(p);
+  p += round_up(xt_bytes, 256);
+  float* m_dev = reinterpret_cast<float*>(p);
+  p += round_up(m_bytes, 256);
+  void* ws = p;
+  const size_t ws_bytes = ws_layout(q, total_rows).total;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (x_bytes > 0 && cudaMemcpyAsync(x_dev, X_host, x_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return SA_ERR_CUDA;
+  if (cudaMemcpyAsync(o_dev, offsets_host, o_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return SA_ERR_CUDA;
+  sa_status s = run(q, x_dev, o_dev, batch, total_rows, xt_dev, m_dev, ws, ws_bytes, stream,
+                    Phase::kBoth);
+  if (s != SA_OK) return s;
+  if (cudaMemcpyAsync(X_tilde_host, xt_dev, xt_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(mass_host, m_dev, m_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return SA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SA_ERR_CUDA;
+  return SA_OK;
+}
+
+sa_status sa_read_device_status(void* workspace, size_t workspace_bytes, void* stream,
+                                uint32_t* flags_out) {
+  if (workspace == nullptr || workspace_bytes < sa::kWsHeaderBytes) return SA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t h[2] = {0, 0};
+  if (cudaMemcpyAsync(h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return SA_ERR_CUDA;
+  const uint32_t bits = h[0] | h[1];
+  if (flags_out) *flags_out = bits;
+  if (bits == 0) return SA_OK;
+  if (cudaMemsetAsync(workspace, 0, sizeof(h), st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return SA_ERR_CUDA;
+  return SA_ERR_DEVICE_FLAG;
+}
+
+}  // extern "C"

@@ -1,0 +1,123 @@
+// Host-side check of the row-range schedule in sa_internal.h (the code the
+// kernels run), on random ragged batches: every row of every user is
+// covered by exactly one segment; users inside one CTA range go straight to
+// the outputs; split users use distinct partial slots below 2G; the
+// finalize pass reduces every split user exactly once, over exactly the
+// slots that the partial pass wrote for it, in ascending CTA order.
+#include <cstdio>
+#include <cstdlib>
+#include <map>
+#include <random>
+#include <set>
+#include <vector>
+
+#include "sa_internal.h"
+
+using namespace sa;
+
+static int fail(const char* what, long long a, long long b) {
+  std::printf("FAIL %s (%lld, %lld)\n", what, a, b);
+  return 1;
+}
+
+static int check(const std::vector<int64_t>& off, int64_t sms) {
+  const int64_t B = static_cast<int64_t>(off.size()) - 1, N = off.back();
+  const int64_t T = tiles_of(N);
+  int64_t G = T < sms ? T : sms;
+  if (G < 1) G = 1;
+  std::vector<int> covered(N, 0);
+  std::map<int64_t, std::set<int64_t>> written;  // user -> slots
+  std::map<int64_t, int64_t> slot_owner;          // slot -> user
+  std::vector<int> direct(B, 0);
+  for (int64_t c = 0; c < G; ++c) {
+    const int64_t R0 = cta_row_begin(c, G, T, N), R1 = cta_row_begin(c + 1, G, T, N);
+    if (N > 0 && R0 >= R1) return fail("empty CTA range", c, R0);
+    if (R0 % kTileRows) return fail("unaligned range", c, R0);
+    if (R0 < R1 && cta_of_row(R0, G, T) != c) return fail("cta_of_row(R0)", c, R0);
+    if (R0 < R1 && cta_of_row(R1 - 1, G, T) != c) return fail("cta_of_row(R1-1)", c, R1);
+    const int64_t b0 = (B > 0 && R0 < R1) ? user_at_or_before(off.data(), B, R0) : B;
+    SegmentWalker w{off.data(), B, R0, R1, b0};
+    int64_t u, s, e, lo, hi;
+    while (w.next(u, s, e, lo, hi)) {
+      if (s < R0 || e > R1 || s < lo || e > hi) return fail("segment bounds", s, e);
+      for (int64_t r = s; r < e; ++r) covered[r]++;
+      const int64_t slot = segment_slot(c, lo, hi, R0, R1);
+      if (slot < 0) {
+        direct[u]++;
+        continue;
+      }
+      if (slot >= 2 * G) return fail("slot range", slot, 2 * G);
+      if (slot_owner.count(slot)) return fail("slot reused", slot, u);
+      slot_owner[slot] = u;
+      written[u].insert(slot);
+    }
+  }
+  for (int64_t r = 0; r < N; ++r)
+    if (covered[r] != 1) return fail("row coverage", r, covered[r]);
+  // finalize ownership, same arithmetic as finalize_kernel
+  std::map<int64_t, std::vector<int64_t>> reduced;
+  for (int64_t cb = 1; cb < G; ++cb) {
+    const int64_t Rc = cta_row_begin(cb, G, T, N), Rp = cta_row_begin(cb - 1, G, T, N);
+    const int64_t b = user_at_or_before(off.data(), B, Rc);
+    const int64_t lo = off[b], hi = off[b + 1];
+    if (!(lo < Rc && lo >= Rp && hi > Rc)) continue;
+    if (reduced.count(b)) return fail("user reduced twice", b, cb);
+    int64_t c_hi = cta_of_row(hi - 1 < N - 1 ? hi - 1 : N - 1, G, T);
+    if (c_hi > G - 1) c_hi = G - 1;
+    std::vector<int64_t> slots{2 * (cb - 1) + (lo <= Rp ? 0 : 1)};
+    for (int64_t cc = cb; cc <= c_hi; ++cc) slots.push_back(2 * cc);
+    reduced[b] = slots;
+  }
+  for (int64_t b = 0; b < B; ++b) {
+    const bool split = written.count(b) > 0;
+    const bool empty = off[b] == off[b + 1];
+    if (empty && (split || direct[b])) return fail("empty user written", b, 0);
+    if (!empty && split == (direct[b] == 1)) return fail("user both/neither direct+split", b, direct[b]);
+    if (direct[b] > 1) return fail("direct twice", b, direct[b]);
+    if (split) {
+      if (!reduced.count(b)) return fail("split user never reduced", b, 0);
+      std::set<int64_t> want(reduced[b].begin(), reduced[b].end());
+      if (want != written[b]) return fail("reduced slots != written slots", b, (long long)want.size());
+      for (size_t i = 1; i < reduced[b].size(); ++i)
+        if (reduced[b][i] <= reduced[b][i - 1]) return fail("slot order", b, i);
+    } else if (reduced.count(b)) {
+      return fail("unsplit user reduced", b, 0);
+    }
+  }
+  return 0;
+}
+
+int main() {
+  std::mt19937_64 rng(12345);
+  long long cases = 0;
+  const int64_t sms_list[] = {1, 2, 3, 7, 148};
+  for (int iter = 0; iter < 3000; ++iter) {
+    const int64_t sms = sms_list[iter % 5];
+    const int B = 1 + static_cast<int>(rng() % 40);
+    std::vector<int64_t> off{0};
+    const int mode = iter % 4;
+    for (int b = 0; b < B; ++b) {
+      int64_t n;
+      switch (mode) {
+        case 0: n = rng() % 300; break;                          // small, many empties possible
+        case 1: n = (rng() % 4 == 0) ? 0 : 1 + rng() % 5000; break;
+        case 2: n = 127 + rng() % 3; break;                      // around one tile
+        default: n = 1 + rng() % 40000; break;
+      }
+      off.push_back(off.back() + n);
+    }
+    if (check(off, sms)) {
+      std::printf("case iter=%d B=%d N=%lld sms=%lld\n", iter, B, (long long)off.back(), (long long)sms);
+      return 1;
+    }
+    ++cases;
+  }
+  // the benchmark shapes
+  std::vector<int64_t> u16{0};
+  for (int b = 0; b < 16; ++b) u16.push_back(u16.back() + 100000);
+  if (check(u16, 148)) return 1;
+  std::vector<int64_t> zero{0, 0, 0};
+  if (check(zero, 148)) return 1;
+  std::printf("OK %lld cases\n", cases + 2);
+  return 0;
+}

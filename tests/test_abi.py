@@ -1,0 +1,84 @@
+"""The C-ABI library: it loads, exports every function include/sa.h
+declares, and rejects bad host-side arguments before touching the GPU.
+No compute call is made here (this runs without a GPU)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from sketch_attention_compression_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sa.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sa_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(binding.LIB_PATH):
+        from sketch_attention_compression_b200 import build
+        build.build()
+    return binding.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("sa_prepare_query", "sa_sketch_forward", "sa_sketch_free"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (sa_\w+)", out))
+    for name in declared_functions():
+        assert name in exported, f"{name} declared in sa.h but not exported"
+        assert getattr(lib, name) is not None
+
+
+def test_binding_covers_header():
+    assert sorted(binding.SIGNATURES) == declared_functions()
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert lib.sa_status_string(code)
+    assert b"workspace" in lib.sa_status_string(binding.SA_ERR_WORKSPACE)
+
+
+def test_null_and_range_arguments_rejected_on_host(lib):
+    out = ctypes.c_void_p(123)
+    st = lib.sa_prepare_query(None, None, None, 16, 64, 0.125, binding.SA_FP32, None,
+                              ctypes.byref(out))
+    assert st == binding.SA_ERR_INVALID_ARG and out.value is None
+    dummy = ctypes.c_void_p(256)
+    for k, d in [(0, 64), (257, 64), (16, 96), (16, 512)]:
+        st = lib.sa_prepare_query(dummy, dummy, dummy, k, d, 0.1, binding.SA_BF16, None,
+                                  ctypes.byref(out))
+        assert st == binding.SA_ERR_INVALID_ARG
+    st = lib.sa_prepare_query(dummy, dummy, dummy, 16, 64, float("nan"), binding.SA_BF16, None,
+                              ctypes.byref(out))
+    assert st == binding.SA_ERR_INVALID_ARG
+    st = lib.sa_prepare_query(dummy, dummy, dummy, 16, 64, 0.1, 7, None, ctypes.byref(out))
+    assert st == binding.SA_ERR_INVALID_ARG
+    assert lib.sa_sketch_forward(None, None, None, 1, 1, None, None, None, 0, None) == \
+        binding.SA_ERR_INVALID_ARG
+    assert lib.sa_workspace_bytes(None, 1, 1) == 0
+    lib.sa_sketch_free(None)  # NULL-safe
+    assert lib.sa_read_device_status(None, 0, None, None) == binding.SA_ERR_INVALID_ARG
+
+
+def test_host_path_rejects_bad_offsets_before_any_copy(lib):
+    # q == NULL is checked first; the offsets checks need a real query and
+    # run in the GPU suite.
+    offs = (ctypes.c_int64 * 3)(0, 5, 3)
+    assert lib.sa_sketch_forward_host(None, None, offs, 2, 3, None, None, None, 0, None) == \
+        binding.SA_ERR_INVALID_ARG

@@ -1,0 +1,25 @@
+"""Host-side logic of the CUDA path, checked without a GPU."""
+
+import os
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
+def test_row_range_schedule(tmp_path):
+    """Compiles the kernels' schedule code (sa_internal.h) for the host and
+    checks coverage, slot uniqueness and finalize ownership on thousands of
+    random ragged batches."""
+    exe = tmp_path / "schedule_check"
+    cuda_inc = "/usr/local/cuda/include"
+    subprocess.run(["g++", "-O1", "-std=c++17",
+                    "-I", os.path.join(ROOT, "sketch_attention_compression_b200", "csrc"),
+                    "-I", cuda_inc, os.path.join(ROOT, "tests", "host", "schedule_check.cpp"),
+                    "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stdout + out.stderr
+    assert out.stdout.startswith("OK")
