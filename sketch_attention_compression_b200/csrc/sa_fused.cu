@@ -89,8 +89,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_empty = s_full + 2;
   uint64_t* p_full = s_empty + 2;
   uint64_t* p_empty = p_full + 2;
+  // Two acc_full barriers, used by segment parity.  A softmax group that
+  // waits for segment s cannot see a stale parity: segment s-2's
+  // aggregation was issued before the MMA1 whose completion let the group
+  // reach this tile, so that earlier phase of acc_full[s & 1] has completed.
   uint64_t* acc_full = p_empty + 2;
-  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* acc_empty = acc_full + 2;
   uint64_t* q_full = acc_empty + 1;
   uint64_t* drain = q_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -104,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t N = a.total_rows;
   const int64_t R0 = cta_row_begin(c, G, a.tiles, N);
   const int64_t R1 = cta_row_begin(c + 1, G, a.tiles, N);
-  uint32_t* sticky = &a.header->sticky_flags;
+  uint32_t* sticky = &a.header->timeout_flags;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
@@ -114,13 +118,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[i], 128);
       mbar_init(&p_empty[i], 1);
     }
-    mbar_init(acc_full, 1);
+    mbar_init(&acc_full[0], 1);
+    mbar_init(&acc_full[1], 1);
     mbar_init(acc_empty, 128);
     mbar_init(q_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0u;
     *b0_slot = (a.batch > 0 && R0 < R1) ? user_at_or_before(a.offsets, a.batch, R0) : a.batch;
-    if (c == 0) a.header->flags = 0u;
+    if (c == 0) { a.header->flags = 0u; a.header->timeout_flags = 0u; }
     fence_mbar_init();
   }
   if (threadIdx.x < 128) {  // 512 B of bf16 ones: B operand of the mass MMA
@@ -205,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&x_empty[st]);
         mma_commit(&p_empty[pb]);
-        if (last) mma_commit(acc_full);
+        if (last) mma_commit(&acc_full[seg & 1u]);
         return true;
       };
 
@@ -331,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         if (last) {
           // ---------------------------------------------- drain X~ and m
-          if (!warp_wait(acc_full, seg & 1u, abort_flag, sticky)) { ok = false; break; }
+          if (!warp_wait(&acc_full[seg & 1u], (seg >> 1) & 1u, abort_flag, sticky)) { ok = false; break; }
           tc_fence_after();
           const int64_t slot = segment_slot(c, lo, hi, R0, R1);
           float* dx = slot < 0 ? a.out_x + user * k * D : a.part_x + slot * k * D;

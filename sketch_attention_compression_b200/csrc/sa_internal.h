@@ -32,8 +32,11 @@ constexpr int kTileRows = 128;
 
 // Workspace: [header 256 B][part_x: 2G * k * d fp32][part_m: 2G * k fp32]
 struct WsHeader {
-  uint32_t flags;         // offset validation bits, rewritten by every call
-  uint32_t sticky_flags;  // timeout bits, cleared only by sa_read_device_status
+  uint32_t flags;          // offset validation bits (set by the finalize pass)
+  uint32_t timeout_flags;  // bounded-wait timeouts (set by the partial pass)
+  // Both words are zeroed by CTA 0 of the partial pass at the start of every
+  // call; all CTAs of that pass are resident together, so this precedes any
+  // timeout report (which takes seconds to arise).
   uint32_t pad[62];
 };
 constexpr size_t kWsHeaderBytes = 256;
