@@ -1,0 +1,429 @@
+"""Benchmark of the SA compression step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step is one SA layer over the whole batch: the fused tensor-core pass
+over X plus the finalize pass, through the C ABI (libsa.so).  The default
+workload is 16 users x 100K behaviours, d = 128, k = 128, bf16 (X drawn from
+a 512-component Gaussian mixture) -- the configuration whose roofline is the
+target.  X is 409.6 MB, larger than the 126 MB L2, so every step streams it
+from HBM.
+
+Prints one JSON line (rank 0).  ``value`` is rows/s over all ranks with X
+resident in HBM; ``e2e`` is the same metric through the host-buffer entry
+point, host->device copy of X and device->host copy of the sketches inside
+the timed region; ``roofline`` is the fused kernel against the measured HBM
+peak; ``cpu_baseline`` is the CPU oracle timed on a bounded sample.
+
+With --gpus N > 1 (launched by torchrun) every rank runs its own batch
+(users are independent; no collective on the data path) and the timing is
+the max over ranks (weak scaling).  ``--impl reference`` times the CPU
+oracle instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synthetic import WORKLOADS, generate  # noqa: E402
+
+METRIC = "SA history rows/sec and % of roofline (max(HBM, bf16 TC)) on 1 B200"
+DEFAULT_WORKLOAD = "batch16_n100k_d128_k128_mixture_bf16"
+L2_BYTES = 126e6
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+KERNEL_SOURCES = ["sketch_attention_compression_b200/csrc/sa_fused.cu",
+                  "sketch_attention_compression_b200/csrc/sa_ptx.cuh",
+                  "sketch_attention_compression_b200/csrc/sa_internal.h"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fused_sa_batch16_n100k_d128_k128.md")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def load_traffic():
+    """DRAM bytes per launch of the fused kernel from the committed ncu
+    summary, if it was taken on the current kernel source (else None)."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    text = open(TRAFFIC_FILE).read()
+    m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_tr or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_tr.group(1))
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9 or (self.uuid and parts[0] != self.uuid):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline / reference arm)
+# ---------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return int(max(i.get("num_threads", 1) for i in info))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_rows_per_s(inp: dict, budget_s: float, users=None):
+    """Runs the oracle user by user until `budget_s` has elapsed (at least one
+    user); returns (rows/s, rows, seconds, users)."""
+    from oracle import sa_user
+    offs = inp["offsets"]
+    order = list(range(len(offs) - 1)) if users is None else users
+    rows = 0
+    done = []
+    t0 = time.perf_counter()
+    for b in order:
+        lo, hi = int(offs[b]), int(offs[b + 1])
+        sa_user(inp["X"][lo:hi], inp["P"], inp["W_Q"], inp["W_K"], inp["scale"])
+        rows += hi - lo
+        done.append(b)
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return rows / dt, rows, dt, done
+
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return
+    inp = generate(args.workload)
+    w = WORKLOADS[args.workload]
+    offs = inp["offsets"]
+    # one step = the oracle over one user's history (a bounded sample)
+    user = 0
+    step_rows = int(offs[user + 1] - offs[user])
+    for _ in range(args.warmup):
+        oracle_rows_per_s(inp, 0.0, users=[user])
+    times = []
+    for _ in range(args.steps):
+        _, rows, dt, _ = oracle_rows_per_s(inp, 0.0, users=[user])
+        times.append(dt)
+    total = sum(times)
+    value = step_rows * args.steps / total
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "users": w.batch, "d": w.d, "k": w.k,
+                   "step_sample": f"user {user} ({step_rows} rows) per step"},
+        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": cores, "kind": "oracle",
+                         "sample": f"user {user} of the workload, {step_rows} rows per step"},
+        "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    from sketch_attention_compression_b200 import SketchQuery, load_library, read_device_status
+
+    load_library()  # fails loudly if the CUDA library is missing
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOADS[args.workload]
+    inp = generate(args.workload, seed=w.seed + rank)  # each rank: its own batch
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    X = torch.from_numpy(inp["X"]).to(dev).to(tdt)
+    P, W_Q, W_K = (torch.from_numpy(inp[k]).to(dev).to(tdt) for k in ("P", "W_Q", "W_K"))
+    offsets = torch.from_numpy(inp["offsets"]).to(dev)
+    B = len(inp["offsets"]) - 1
+    N = int(inp["offsets"][-1])
+    elem = 2 if w.dtype == "bf16" else 4
+
+    stream = torch.cuda.current_stream(dev)
+    q = SketchQuery(P, W_Q, W_K, inp["scale"], stream=stream)
+    ws = q.new_workspace(B, N)
+    Xt = torch.empty((B, w.k, w.d), dtype=torch.float32, device=dev)
+    m = torch.empty((B, w.k), dtype=torch.float32, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up (also checks the device flags once)
+    for _ in range(max(args.warmup, 1)):
+        q.forward(X, offsets, Xt, m, ws, stream=stream)
+    if read_device_status(ws, stream) != 0:
+        raise RuntimeError("device flags raised during warm-up")
+
+    clocks = None
+    sampler = None
+    if rank == 0:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        sampler.start()
+        time.sleep(0.3)
+
+    # -- timed region A: the product call, back to back -------------------
+    launches = 0
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        q.forward(X, offsets, Xt, m, ws, stream=stream)
+        launches += 2
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    step_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+
+    # -- timed region B: the two passes split by events (kernel durations) --
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(3 * args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    for s in range(args.steps):
+        evs[3 * s].record(stream)
+        q.partials(X, offsets, Xt, m, ws, stream=stream)
+        evs[3 * s + 1].record(stream)
+        q.finalize(X, offsets, Xt, m, ws, stream=stream)
+        evs[3 * s + 2].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    fused_ms = statistics.mean(evs[3 * s].elapsed_time(evs[3 * s + 1]) for s in range(args.steps))
+    fin_ms = statistics.mean(evs[3 * s + 1].elapsed_time(evs[3 * s + 2]) for s in range(args.steps))
+    fused_ms = max_over_ranks(fused_ms)
+    fin_ms = max_over_ranks(fin_ms)
+    if read_device_status(ws, stream) != 0:
+        raise RuntimeError("device flags raised during the timed region")
+
+    # -- timed region C: end to end on host buffers ----------------------
+    X_host = X.cpu().pin_memory()
+    offs_host = np.ascontiguousarray(inp["offsets"])
+    dev_buf = torch.empty(q.host_path_device_bytes(B, N), dtype=torch.uint8, device=dev)
+    out_x = torch.empty((B, w.k, w.d), dtype=torch.float32).pin_memory().numpy()
+    out_m = torch.empty((B, w.k), dtype=torch.float32).pin_memory().numpy()
+    e2e_steps = max(3, min(args.steps, 20))
+    q.forward_host(X_host, offs_host, dev_buf, stream=stream, out_x=out_x, out_m=out_m)
+    barrier()
+    torch.cuda.synchronize(dev)
+    h0 = torch.cuda.Event(enable_timing=True)
+    h1 = torch.cuda.Event(enable_timing=True)
+    h0.record(stream)
+    for _ in range(e2e_steps):
+        q.forward_host(X_host, offs_host, dev_buf, stream=stream, out_x=out_x, out_m=out_m)
+    h1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(h0.elapsed_time(h1) / e2e_steps)
+
+    if sampler is not None:
+        clocks = sampler.stop()
+
+    # sanity on the last outputs: every behaviour spreads unit mass
+    msum = m.sum(dim=1).double().cpu().numpy()
+    n_b = np.diff(inp["offsets"]).astype(np.float64)
+    if np.max(np.abs(msum - n_b) / np.maximum(n_b, 1)) > 1e-3:
+        raise RuntimeError("mass check failed")
+
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    bytes_x = float(N) * w.d * elem
+    flops = 4.0 * w.k * w.d * N
+    t_hbm = bytes_x / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    fused_s = fused_ms * 1e-3
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    if bound == "hbm":
+        achieved, peak, unit = bytes_x / fused_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved, peak, unit = flops / fused_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    traffic = load_traffic()
+    rows_total = N * world
+    value = rows_total / (step_ms * 1e-3)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rps, rows, dt, users = oracle_rows_per_s(inp, args.cpu_budget)
+        cpu = {"value": rps, "unit": "rows/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"users {users[0]}..{users[-1]} ({rows} rows, {dt:.1f} s, numpy fp64)"}
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "rows/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": args.workload, "users_per_gpu": w.batch, "rows_per_gpu": N,
+            "d": w.d, "k": w.k, "x_bytes_per_gpu": bytes_x,
+            "l2": f"inputs larger than L2 (X {bytes_x / 1e6:.1f} MB > {L2_BYTES / 1e6:.0f} MB)",
+            "parallelism": f"independent batch per GPU x{world}",
+        },
+        "roofline": {
+            "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": traffic,
+            "kernel": "fused_sa_kernel<128,128>" if (w.d, w.k) == (128, 128) else "fused_sa_kernel",
+            "kernel_ms": fused_ms, "finalize_ms": fin_ms,
+            "roofline_ms": 1e3 * max(t_hbm, t_tc),
+            "tensor_frac": (flops / fused_s / 1e12) / peaks["bf16_tflops"],
+            "hbm_frac": (bytes_x / fused_s / 1e9) / peaks["hbm_gbs"],
+            "peak_source": f"MEASURED_PEAKS.json ({peak_kind}, burst)",
+            "algorithmic": f"{2 * w.d} B and {4 * w.k * w.d} flop per row x {N} rows",
+        },
+        "e2e": {"value": rows_total / (e2e_ms * 1e-3), "unit": "rows/s",
+                "h2d_bytes_per_step": int(bytes_x + 8 * (B + 1)),
+                "d2h_bytes_per_step": int(4 * B * w.k * (w.d + 1)),
+                "ms_per_step": e2e_ms},
+        "gpu_launches": launches * 2 + 2 * e2e_steps + 2,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-budget", type=float, default=10.0,
+                    help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

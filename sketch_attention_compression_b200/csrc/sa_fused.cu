@@ -33,6 +33,7 @@ namespace sa {
 namespace {
 
 constexpr int kThreads = 384;
+constexpr int kRing = 16;  // issuer's ring of in-flight tile descriptors
 constexpr int kMaxDynSmem = 232448;  // 227 KB per block on sm_100
 
 template <int D, int KM>
@@ -68,7 +69,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
-template <int D, int KM>
+// FULL: k == KM, so no prototype column needs masking.
+template <int D, int KM, bool FULL>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_sa_kernel(const __grid_constant__ CUtensorMap tm_x,
                     const __grid_constant__ CUtensorMap tm_q, const PassArgs a) {
@@ -100,6 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   int64_t* b0_slot = reinterpret_cast<int64_t*>(tmem_slot + 2);
+  uint32_t* tile_ring = reinterpret_cast<uint32_t*>(b0_slot + 1);  // issuer's tile descriptors
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -188,72 +191,99 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(q_full, 0, abort_flag, sticky);
       tc_fence_after();
 
-      // MMA2 + mass of tile u (deferred by one tile).
-      auto issue_aggregate = [&](uint32_t u, int st, bool first, bool last,
-                                 uint32_t seg) -> bool {
-        const int pb = u & 1;
-        if (!mbar_wait(&p_full[pb], (u >> 1) & 1u, abort_flag, sticky)) return false;
-        if (first && !mbar_wait(acc_empty, (seg & 1u) ^ 1u, abort_flag, sticky)) return false;
-        tc_fence_after();
-        const uint32_t pa = p_a + pb * C::kPBytes;
-        const uint32_t xa = x_a + st * C::kXBytes;
-#pragma unroll
-        for (int ks = 0; ks < kTileRows / 16; ++ks) {
-          const uint64_t ad = smem_desc(pa + ks * 2048, 16384, 1024, 2);
-          const uint64_t bd = smem_desc(xa + ks * 2048, 16384, 1024, 2);
-          mma_bf16_ss(tmem + C::kColAcc, ad, bd, idesc_x, (!first || ks > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int ks = 0; ks < kTileRows / 16; ++ks) {
-          const uint64_t ad = smem_desc(pa + ks * 2048, 16384, 1024, 2);
-          mma_bf16_ss(tmem + C::kColMass, ad, ones_desc, idesc_m, (!first || ks > 0) ? 1u : 0u);
-        }
-        mma_commit(&x_empty[st]);
-        mma_commit(&p_empty[pb]);
-        if (last) mma_commit(&acc_full[seg & 1u]);
-        return true;
-      };
-
+      // Non-blocking scheduler with two cursors over the CTA's tiles:
+      //   t1: next tile whose affinity MMA (MMA1) is issued, as soon as its X
+      //       stage has landed and its S^T buffer has been read out;
+      //   t2: next tile whose aggregation (MMA2 + mass) is issued, as soon as
+      //       its probabilities are in shared memory (and, for the first
+      //       tile of a user segment, the accumulator has been drained).
+      // MMA1 thus runs ahead of the softmax instead of waiting for the
+      // previous tile's aggregation.  The tensor pipe executes the issued
+      // MMAs in order.
+      // Tile descriptors of issued-but-not-aggregated tiles, in shared memory:
+      // bits 0-7 stage, bit 8 first of segment, bit 9 last, bits 10+ segment.
+      static_assert(kRing >= S + 2, "tile ring");
       SegmentWalker w{a.offsets, a.batch, R0, R1, b0};
-      int64_t user, s, e, lo, hi;
-      uint32_t t = 0, seg = 0;
-      bool have_prev = false, prev_first = false, prev_last = false;
-      uint32_t prev_t = 0, prev_seg = 0;
-      int prev_st = 0;
-      while (ok && w.next(user, s, e, lo, hi)) {
-        for (int64_t r = s; r < e; r += kTileRows) {
-          const int st = t % S;
-          const int sb = t & 1;
-          if (!mbar_wait(&x_full[st], (t / S) & 1u, abort_flag, sticky) ||
-              !mbar_wait(&s_empty[sb], ((t >> 1) & 1u) ^ 1u, abort_flag, sticky)) {
-            ok = false;
-            break;
+      int64_t user = 0, s = 0, e = 0, lo = 0, hi = 0, r = 0;
+      bool have_seg = false, walker_done = false;
+      uint32_t t1 = 0, t2 = 0, seg = 0;
+      unsigned long long idle_since = globaltimer_ns();
+      while (ok) {
+        bool progressed = false;
+        // ---- MMA1 for tile t1
+        if (!walker_done) {
+          if (!have_seg) {
+            have_seg = w.next(user, s, e, lo, hi);
+            if (have_seg) r = s; else walker_done = true;
           }
-          tc_fence_after();
-          const uint32_t xa = x_a + st * C::kXBytes;
+          if (have_seg) {
+            const int st = t1 % S;
+            const int sb = t1 & 1;
+            if (mbar_try_wait(&x_full[st], (t1 / S) & 1u) &&
+                mbar_try_wait(&s_empty[sb], ((t1 >> 1) & 1u) ^ 1u)) {
+              tc_fence_after();
+              const uint32_t xa = x_a + st * C::kXBytes;
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-            const uint64_t ad = smem_desc(xa + koff, 16, 1024, 2);
-            const uint64_t bd = smem_desc(q_a + (ks >> 2) * (KM * 128) + (ks & 3) * 32, 16, 1024, 2);
-            mma_bf16_ss(tmem + C::kColS + sb * KM, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+              for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                const uint64_t ad = smem_desc(xa + koff, 16, 1024, 2);
+                const uint64_t bd =
+                    smem_desc(q_a + (ks >> 2) * (KM * 128) + (ks & 3) * 32, 16, 1024, 2);
+                mma_bf16_ss(tmem + C::kColS + sb * KM, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+              }
+              mma_commit(&s_full[sb]);
+              tile_ring[t1 % kRing] = static_cast<uint32_t>(st) | (r == s ? 0x100u : 0u) |
+                                      (r + kTileRows >= e ? 0x200u : 0u) | (seg << 10);
+              ++t1;
+              r += kTileRows;
+              if (r >= e) { have_seg = false; ++seg; }
+              progressed = true;
+            }
           }
-          mma_commit(&s_full[sb]);
-          if (have_prev && !issue_aggregate(prev_t, prev_st, prev_first, prev_last, prev_seg)) {
-            ok = false;
-            break;
-          }
-          have_prev = true;
-          prev_t = t;
-          prev_st = st;
-          prev_first = (r == s);
-          prev_last = (r + kTileRows >= e);
-          prev_seg = seg;
-          ++t;
         }
-        ++seg;
+        // ---- MMA2 + mass for tile t2
+        if (t2 < t1) {
+          const uint32_t desc = tile_ring[t2 % kRing];
+          const bool first = desc & 0x100u;
+          const bool last = desc & 0x200u;
+          const uint32_t sg = desc >> 10;
+          const int pb = t2 & 1;
+          if (mbar_try_wait(&p_full[pb], (t2 >> 1) & 1u) &&
+              (!first || mbar_try_wait(acc_empty, (sg & 1u) ^ 1u))) {
+            tc_fence_after();
+            const int st = static_cast<int>(desc & 0xFFu);
+            const uint32_t pa = p_a + pb * C::kPBytes;
+            const uint32_t xa = x_a + st * C::kXBytes;
+#pragma unroll
+            for (int ks = 0; ks < kTileRows / 16; ++ks) {
+              const uint64_t ad = smem_desc(pa + ks * 2048, 16384, 1024, 2);
+              const uint64_t bd = smem_desc(xa + ks * 2048, 16384, 1024, 2);
+              mma_bf16_ss(tmem + C::kColAcc, ad, bd, idesc_x, (!first || ks > 0) ? 1u : 0u);
+            }
+#pragma unroll
+            for (int ks = 0; ks < kTileRows / 16; ++ks) {
+              const uint64_t ad = smem_desc(pa + ks * 2048, 16384, 1024, 2);
+              mma_bf16_ss(tmem + C::kColMass, ad, ones_desc, idesc_m,
+                          (!first || ks > 0) ? 1u : 0u);
+            }
+            mma_commit(&x_empty[st]);
+            mma_commit(&p_empty[pb]);
+            if (last) mma_commit(&acc_full[sg & 1u]);
+            ++t2;
+            progressed = true;
+          }
+        }
+        if (walker_done && t2 == t1) break;
+        if (progressed) {
+          idle_since = globaltimer_ns();
+        } else if (*abort_flag) {
+          ok = false;
+        } else if (globaltimer_ns() - idle_since > kWaitTimeoutNs) {
+          *abort_flag = 1u;
+          atomicOr(sticky, DEVFLAG_TIMEOUT);
+          ok = false;
+        }
       }
-      if (ok && have_prev) ok = issue_aggregate(prev_t, prev_st, prev_first, prev_last, prev_seg);
       if (!ok) {  // make sure no MMA is still running when TMEM is released
         mma_commit(drain);
         mbar_wait_bounded(drain, 0);
@@ -289,19 +319,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(&s_empty[grp]);
 
-        // stable softmax over the prototype axis (thread-local)
-        float mx = -INFINITY;
+        // stable softmax over the prototype axis (thread-local); eight
+        // independent max / sum chains keep the FP pipes busy
+        float mx8[8], sm8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
         for (int j = 0; j < KM; ++j)
-          if (j < k) mx = fmaxf(mx, __uint_as_float(sr[j >> 5][j & 31]));
-        float sum = 0.f;
+          if (FULL || j < k) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(sr[j >> 5][j & 31]));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sm8[i] = 0.f;
         float pv[KM];
 #pragma unroll
         for (int j = 0; j < KM; ++j) {
-          const float ev = (j < k) ? ex2_approx(__uint_as_float(sr[j >> 5][j & 31]) - mx) : 0.f;
+          const float ev = (FULL || j < k) ? ex2_approx(__uint_as_float(sr[j >> 5][j & 31]) - mx) : 0.f;
           pv[j] = ev;
-          sum += ev;
+          sm8[j & 7] += ev;
         }
+        const float sum = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
         const float inv = 1.0f / sum;
 
         if (!warp_wait(&p_empty[grp], ((t >> 1) & 1u) ^ 1u, abort_flag, sticky)) { ok = false; break; }
@@ -383,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, int KM>
 cudaError_t launch_one(const CUtensorMap& tx, const CUtensorMap& tq, const PassArgs& a,
                        int grid, cudaStream_t stream) {
-  auto kern = fused_sa_kernel<D, KM>;
+  auto kern = a.k == KM ? fused_sa_kernel<D, KM, true> : fused_sa_kernel<D, KM, false>;
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, KM>::kSmem);
   if (err != cudaSuccess) return err;

@@ -78,16 +78,22 @@ WORKLOADS: Dict[str, Workload] = {
 def bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float32 values to bf16, nearest-even; return the uint16 patterns.
 
-    NaN maps to the quiet NaN 0x7FC0 (sign kept); +-inf stays +-inf.
+    NaN maps to the quiet NaN 0x7FC0 (sign kept); +-inf stays +-inf.  For
+    every non-NaN pattern u <= 0xFF800000 the sum below stays under 2**32,
+    so 32-bit arithmetic suffices.
     """
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    u = x.view(np.uint32).copy()
     nan = np.isnan(x)
+    lsb = (u >> 16) & np.uint32(1)
+    u += np.uint32(0x7FFF)
+    u += lsb
+    del lsb
+    u >>= 16
+    r = u.astype(np.uint16)
     if nan.any():
-        sign = ((u >> 16) & 0x8000).astype(np.uint16)
-        r = np.where(nan, sign | np.uint16(0x7FC0), r)
+        sign = (x.view(np.uint32)[nan] >> 16).astype(np.uint16) & np.uint16(0x8000)
+        r[nan] = sign | np.uint16(0x7FC0)
     return r.reshape(x.shape)
 
 
