@@ -5,7 +5,7 @@
 
 #include <new>
 
-#include "../../include/sa.h"
+#include "sa.h"
 #include "sa_internal.h"
 
 struct sa_query_s {

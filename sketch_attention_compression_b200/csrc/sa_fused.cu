@@ -188,6 +188,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t x_a = smem_u32(x_s);
       const uint32_t p_a = smem_u32(p_s);
       const uint64_t ones_desc = smem_desc(smem_u32(ones_s), 128, 256, 0);
+      // Base descriptors, built once.  A byte offset b within shared memory
+      // is applied by adding b >> 4 to the start-address field (bits 0-13);
+      // every address stays below 2^18 bytes, so the field never carries.
+      // This keeps the issuing thread to one add per MMA: its own scalar
+      // latency would otherwise pace the tensor pipe.
+      const uint64_t xk_desc = smem_desc(x_a, 16, 1024, 2);      // X as K-major A
+      const uint64_t q_desc = smem_desc(q_a, 16, 1024, 2);       // Q' as K-major B
+      const uint64_t p_desc = smem_desc(p_a, 16384, 1024, 2);    // P as MN-major A
+      const uint64_t xmn_desc = smem_desc(x_a, 16384, 1024, 2);  // X as MN-major B
       bool ok = mbar_wait(q_full, 0, abort_flag, sticky);
       tc_fence_after();
 
@@ -207,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t user = 0, s = 0, e = 0, lo = 0, hi = 0, r = 0;
       bool have_seg = false, walker_done = false;
       uint32_t t1 = 0, t2 = 0, seg = 0;
-      unsigned long long idle_since = globaltimer_ns();
+      long long idle_since = cycles_now();
       while (ok) {
         bool progressed = false;
         // ---- MMA1 for tile t1
@@ -219,17 +228,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (have_seg) {
             const int st = t1 % S;
             const int sb = t1 & 1;
-            if (mbar_try_wait(&x_full[st], (t1 / S) & 1u) &&
-                mbar_try_wait(&s_empty[sb], ((t1 >> 1) & 1u) ^ 1u)) {
+            if (mbar_test_wait(&x_full[st], (t1 / S) & 1u) &&
+                mbar_test_wait(&s_empty[sb], ((t1 >> 1) & 1u) ^ 1u)) {
               tc_fence_after();
-              const uint32_t xa = x_a + st * C::kXBytes;
+              const uint64_t xd = xk_desc + ((st * C::kXBytes) >> 4);
+              const uint32_t dcol = tmem + C::kColS + sb * KM;
 #pragma unroll
               for (int ks = 0; ks < D / 16; ++ks) {
-                const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                const uint64_t ad = smem_desc(xa + koff, 16, 1024, 2);
-                const uint64_t bd =
-                    smem_desc(q_a + (ks >> 2) * (KM * 128) + (ks & 3) * 32, 16, 1024, 2);
-                mma_bf16_ss(tmem + C::kColS + sb * KM, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                mma_bf16_ss(dcol, xd + (((ks >> 2) * 16384 + (ks & 3) * 32) >> 4),
+                            q_desc + (((ks >> 2) * (KM * 128) + (ks & 3) * 32) >> 4), idesc_s,
+                            ks > 0 ? 1u : 0u);
               }
               mma_commit(&s_full[sb]);
               tile_ring[t1 % kRing] = static_cast<uint32_t>(st) | (r == s ? 0x100u : 0u) |
@@ -248,24 +256,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool last = desc & 0x200u;
           const uint32_t sg = desc >> 10;
           const int pb = t2 & 1;
-          if (mbar_try_wait(&p_full[pb], (t2 >> 1) & 1u) &&
-              (!first || mbar_try_wait(acc_empty, (sg & 1u) ^ 1u))) {
+          if (mbar_test_wait(&p_full[pb], (t2 >> 1) & 1u) &&
+              (!first || mbar_test_wait(acc_empty, (sg & 1u) ^ 1u))) {
             tc_fence_after();
             const int st = static_cast<int>(desc & 0xFFu);
-            const uint32_t pa = p_a + pb * C::kPBytes;
-            const uint32_t xa = x_a + st * C::kXBytes;
+            const uint64_t pd = p_desc + ((pb * C::kPBytes) >> 4);
+            const uint64_t xd = xmn_desc + ((st * C::kXBytes) >> 4);
+            const uint32_t acc0 = (!first) ? 1u : 0u;
 #pragma unroll
-            for (int ks = 0; ks < kTileRows / 16; ++ks) {
-              const uint64_t ad = smem_desc(pa + ks * 2048, 16384, 1024, 2);
-              const uint64_t bd = smem_desc(xa + ks * 2048, 16384, 1024, 2);
-              mma_bf16_ss(tmem + C::kColAcc, ad, bd, idesc_x, (!first || ks > 0) ? 1u : 0u);
-            }
+            for (int ks = 0; ks < kTileRows / 16; ++ks)
+              mma_bf16_ss(tmem + C::kColAcc, pd + ((ks * 2048) >> 4), xd + ((ks * 2048) >> 4),
+                          idesc_x, ks > 0 ? 1u : acc0);
 #pragma unroll
-            for (int ks = 0; ks < kTileRows / 16; ++ks) {
-              const uint64_t ad = smem_desc(pa + ks * 2048, 16384, 1024, 2);
-              mma_bf16_ss(tmem + C::kColMass, ad, ones_desc, idesc_m,
-                          (!first || ks > 0) ? 1u : 0u);
-            }
+            for (int ks = 0; ks < kTileRows / 16; ++ks)
+              mma_bf16_ss(tmem + C::kColMass, pd + ((ks * 2048) >> 4), ones_desc, idesc_m,
+                          ks > 0 ? 1u : acc0);
             mma_commit(&x_empty[st]);
             mma_commit(&p_empty[pb]);
             if (last) mma_commit(&acc_full[sg & 1u]);
@@ -275,10 +280,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (walker_done && t2 == t1) break;
         if (progressed) {
-          idle_since = globaltimer_ns();
+          idle_since = cycles_now();
+        } else if (!*abort_flag && cycles_now() - idle_since <= kWaitTimeoutCycles) {
+          // Nothing ready: back off briefly so that this polling thread does
+          // not take issue slots from the softmax warps on its SM sub-partition.
+          __nanosleep(64);
         } else if (*abort_flag) {
           ok = false;
-        } else if (globaltimer_ns() - idle_since > kWaitTimeoutNs) {
+        } else if (cycles_now() - idle_since > kWaitTimeoutCycles) {
           *abort_flag = 1u;
           atomicOr(sticky, DEVFLAG_TIMEOUT);
           ok = false;

@@ -18,19 +18,19 @@ enum : uint32_t {
   DEVFLAG_TIMEOUT = 8u,            // a bounded wait inside a kernel gave up
 };
 
-// A wait that has not completed after this many nanoseconds is treated as a
-// hang: the kernel records DEVFLAG_TIMEOUT, stops issuing work and exits.
-constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
+// A wait that has not completed after this many SM clock cycles (about 2 s
+// at the B200's 1.965 GHz boost clock, longer at lower clocks) is treated as
+// a hang: the kernel records DEVFLAG_TIMEOUT, stops issuing work and exits.
+// Elapsed time is read from the per-SM cycle counter: %globaltimer is a slow
+// special register, and reading it inside polling loops costs hundreds of
+// cycles per iteration.
+constexpr long long kWaitTimeoutCycles = 4000000000ll;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ unsigned long long globaltimer_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
+__device__ __forceinline__ long long cycles_now() { return clock64(); }
 
 // ---------------------------------------------------------------- mbarrier
 
@@ -71,19 +71,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of the phase with the given parity (never suspends the
+// thread, unlike try_wait); for schedulers that poll several barriers.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `bar` with the given parity.  Gives up (returns
 // false) when another role of the CTA has raised `abort_flag`, or after
-// kWaitTimeoutNs, in which case it raises `abort_flag` itself and records
+// kWaitTimeoutCycles, in which case it raises `abort_flag` itself and records
 // DEVFLAG_TIMEOUT in `sticky_flag` (global memory).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           volatile uint32_t* abort_flag,
                                           uint32_t* sticky_flag) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
+  const long long t0 = cycles_now();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+    if (cycles_now() - t0 > kWaitTimeoutCycles) {
       *abort_flag = 1u;
       atomicOr(sticky_flag, DEVFLAG_TIMEOUT);
       return false;
@@ -93,9 +107,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 
 // Bounded wait used only on the abort path (no flag bookkeeping).
 __device__ __forceinline__ void mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-  const unsigned long long t0 = globaltimer_ns();
+  const long long t0 = cycles_now();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) return;
+    if (cycles_now() - t0 > kWaitTimeoutCycles) return;
   }
 }
 
@@ -122,6 +136,15 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
       ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+
+// Bulk-tensor prefetch of one box into L2 (no shared memory, no completion
+// signal).  Same coordinate rules as tma_load_2d.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
 }
 
 __device__ __forceinline__ uint64_t policy_evict_first() {
