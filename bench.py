@@ -177,10 +177,21 @@ def oracle_rows_per_s(inp: dict, budget_s: float, users=None):
     return rows / dt, rows, dt, done
 
 
+def workload_inputs(args, seed=None) -> dict:
+    """The named workload; with --users U, only its first U users (a smaller
+    case of the same shapes, e.g. for a profiler capture)."""
+    inp = generate(args.workload, seed=seed)
+    if args.users and args.users < len(inp["offsets"]) - 1:
+        offs = inp["offsets"][: args.users + 1].copy()
+        inp["offsets"] = offs
+        inp["X"] = inp["X"][: int(offs[-1])]
+    return inp
+
+
 def run_reference(args, rank: int):
     if rank != 0:
         return
-    inp = generate(args.workload)
+    inp = workload_inputs(args)
     w = WORKLOADS[args.workload]
     offs = inp["offsets"]
     # one step = the oracle over one user's history (a bounded sample)
@@ -200,7 +211,7 @@ def run_reference(args, rank: int):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "users": w.batch, "d": w.d, "k": w.k,
+        "config": {"workload": args.workload, "users": len(offs) - 1, "d": w.d, "k": w.k,
                    "step_sample": f"user {user} ({step_rows} rows) per step"},
         "cpu_baseline": {"value": value, "unit": "rows/s", "cores": cores, "kind": "oracle",
                          "sample": f"user {user} of the workload, {step_rows} rows per step"},
@@ -224,7 +235,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = WORKLOADS[args.workload]
-    inp = generate(args.workload, seed=w.seed + rank)  # each rank: its own batch
+    inp = workload_inputs(args, seed=w.seed + rank)  # each rank: its own batch
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     X = torch.from_numpy(inp["X"]).to(dev).to(tdt)
     P, W_Q, W_K = (torch.from_numpy(inp[k]).to(dev).to(tdt) for k in ("P", "W_Q", "W_K"))
@@ -362,7 +373,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
         "config": {
-            "workload": args.workload, "users_per_gpu": w.batch, "rows_per_gpu": N,
+            "workload": args.workload, "users_per_gpu": B, "rows_per_gpu": N,
             "d": w.d, "k": w.k, "x_bytes_per_gpu": bytes_x,
             "l2": f"inputs larger than L2 (X {bytes_x / 1e6:.1f} MB > {L2_BYTES / 1e6:.0f} MB)",
             "parallelism": f"independent batch per GPU x{world}",
@@ -399,6 +410,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0,
                     help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--users", type=int, default=0,
+                    help="use only the first U users of the workload (smaller case)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
