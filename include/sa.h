@@ -170,6 +170,44 @@ sa_status sa_sketch_forward_host(sa_query q, const void* X_host, const int64_t* 
 sa_status sa_read_device_status(void* workspace, size_t workspace_bytes, void* stream,
                                 uint32_t* flags_out);
 
+/*
+ * sa_sketch_forward_noalloc -- sa_sketch_forward for callers that cannot
+ * allocate device memory.  (The SequenceO1 paper has no counterpart to this
+ * entry point; it exists for callers of this library.)
+ *
+ * Some callers cannot call cudaMalloc or any other allocator where they run
+ * the SA layer: code inside an allocator's own hooks, code under a memory
+ * pool that must not grow, or hosts that hand the library only fixed,
+ * pre-registered buffers.  This call takes the same inputs and outputs as
+ * sa_sketch_forward, but in place of a caller-provided workspace it uses a
+ * fixed 32 MiB scratch array inside the library's device image.  Every GPU
+ * that loads the library holds that array until the process exits.  The
+ * call itself allocates nothing.
+ *
+ *   q, X, offsets, batch, total_rows, X_tilde, mass, stream
+ *                     as for sa_sketch_forward
+ *   device_flags_out  device, 2 uint32 words (4-byte aligned), or NULL:
+ *                     receives, in stream order, this call's device flags
+ *                     (word 0: the SA_DEVFLAG_OFFSET* bits, word 1:
+ *                     SA_DEVFLAG_TIMEOUT), which sa_read_device_status
+ *                     reports for the workspace path
+ *
+ * Returns SA_ERR_WORKSPACE when the call needs more scratch than the array
+ * holds (sa_workspace_bytes(q, batch, total_rows) > 32 MiB; this covers
+ * every query with k * d <= 128 * 128 on a 148-SM GPU), SA_ERR_CUDA if the
+ * array's address cannot be looked up, and otherwise what sa_sketch_forward
+ * returns.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture on the device.  All calls share the
+ * one array, so calls whose work overlaps on the GPU (other streams, other
+ * host threads) race on it and give wrong results: serialise them.
+ */
+sa_status sa_sketch_forward_noalloc(sa_query q, const void* X, const int64_t* offsets,
+                                    int64_t batch, int64_t total_rows, float* X_tilde,
+                                    float* mass, uint32_t* device_flags_out, void* stream);
+
 /* Static description of a status code. */
 const char* sa_status_string(sa_status s);
 

@@ -36,6 +36,7 @@ SIGNATURES = {
     "sa_sketch_finalize": (_i32, _FWD_ARGS),
     "sa_host_path_device_bytes": (_sz, [_vp, _i64, _i64]),
     "sa_sketch_forward_host": (_i32, _FWD_ARGS),
+    "sa_sketch_forward_noalloc": (_i32, [_vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp]),
     "sa_read_device_status": (_i32, [_vp, _sz, _vp, ctypes.POINTER(ctypes.c_uint32)]),
     "sa_status_string": (ctypes.c_char_p, [_i32]),
     "sa_query_info": (_i32, [_vp, ctypes.POINTER(_i32), ctypes.POINTER(_i32),
@@ -193,6 +194,38 @@ class SketchQuery:
         args, *_ = self._args(X, offsets, X_tilde, mass, workspace)
         _check(self._lib.sa_sketch_finalize(self._h, *args, ctypes.c_void_p(_stream_handle(stream))),
                "sa_sketch_finalize")
+
+    def forward_noalloc(self, X, offsets, X_tilde=None, mass=None, device_flags=None,
+                        stream=None) -> Tuple[object, object]:
+        """Same layer through sa_sketch_forward_noalloc: no workspace, the
+        library's fixed scratch array instead (see include/sa.h).  Outputs
+        are allocated here when not given; the C call allocates nothing.
+        ``device_flags`` (int32 CUDA tensor of 2 words) receives the call's
+        device flags."""
+        torch = _torch()
+        if X.dtype != self.dtype:
+            raise TypeError(f"X dtype {X.dtype} != query dtype {self.dtype}")
+        if X.dim() != 2 or X.shape[1] != self.d:
+            raise ValueError("X must be (N, d)")
+        if offsets.dtype != torch.int64 or offsets.dim() != 1:
+            raise TypeError("offsets must be a 1-D int64 tensor")
+        B = int(offsets.shape[0]) - 1
+        N = int(X.shape[0])
+        if X_tilde is None:
+            X_tilde = torch.empty((B, self.k, self.d), dtype=torch.float32, device=X.device)
+        if mass is None:
+            mass = torch.empty((B, self.k), dtype=torch.float32, device=X.device)
+        xp = _dev_ptr(X, "X") if N > 0 else ctypes.c_void_p(0)
+        fp = ctypes.c_void_p(0)
+        if device_flags is not None:
+            if device_flags.numel() * device_flags.element_size() < 8:
+                raise ValueError("device_flags must hold 2 uint32 words")
+            fp = _dev_ptr(device_flags, "device_flags")
+        st = self._lib.sa_sketch_forward_noalloc(
+            self._h, xp, _dev_ptr(offsets, "offsets"), B, N, _dev_ptr(X_tilde, "X_tilde"),
+            _dev_ptr(mass, "mass"), fp, ctypes.c_void_p(_stream_handle(stream)))
+        _check(st, "sa_sketch_forward_noalloc")
+        return X_tilde, mass
 
     # -- host path ---------------------------------------------------------
     def forward_host(self, X_host, offsets_host: np.ndarray, device_buffer=None, stream=None,
