@@ -64,6 +64,7 @@ typedef enum sa_dtype {
 #define SA_DEVFLAG_OFFSETS_DECREASE 2u /* offsets[b] > offsets[b+1] for some b */
 #define SA_DEVFLAG_OFFSET_LAST 4u      /* offsets[batch] != total_rows */
 #define SA_DEVFLAG_TIMEOUT 8u          /* a kernel's bounded wait gave up */
+#define SA_DEVFLAG_SMEM_ALIGN 16u      /* a kernel found its shared memory misaligned (no work done) */
 
 /* Opaque handle: the precomputed query Q' for one weight set. */
 typedef struct sa_query_s* sa_query;
@@ -189,7 +190,7 @@ sa_status sa_read_device_status(void* workspace, size_t workspace_bytes, void* s
  *   device_flags_out  device, 2 uint32 words (4-byte aligned), or NULL:
  *                     receives, in stream order, this call's device flags
  *                     (word 0: the SA_DEVFLAG_OFFSET* bits, word 1:
- *                     SA_DEVFLAG_TIMEOUT), which sa_read_device_status
+ *                     SA_DEVFLAG_TIMEOUT and SA_DEVFLAG_SMEM_ALIGN), which sa_read_device_status
  *                     reports for the workspace path
  *
  * Returns SA_ERR_WORKSPACE when the call needs more scratch than the array

@@ -19,8 +19,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "lib
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA, \
     SA_ERR_DEVICE_FLAG = range(6)
 SA_BF16, SA_FP32 = 0, 1
-DEVFLAG_OFFSET0_NONZERO, DEVFLAG_OFFSETS_DECREASE, DEVFLAG_OFFSET_LAST, DEVFLAG_TIMEOUT = \
-    1, 2, 4, 8
+DEVFLAG_OFFSET0_NONZERO, DEVFLAG_OFFSETS_DECREASE, DEVFLAG_OFFSET_LAST, DEVFLAG_TIMEOUT, \
+    DEVFLAG_SMEM_ALIGN = 1, 2, 4, 8, 16
 
 # name -> (restype, argtypes); mirrors include/sa.h
 _vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, \

@@ -7,25 +7,42 @@
 // matrices never reach HBM, over batches of unequal lengths.
 //
 // Per 128-row tile X_t of one user (rows i, prototypes j):
-//   MMA1  S^T_t = X_t Q'^T          M=128 rows, N=k_pad, K=d   (TMEM, fp32)
-//   softmax over j, one thread per row i (the prototype axis lies along
-//         the thread's own TMEM lane, so no cross-thread reduction):
-//         a_ji = exp2(s_ji - max_j s_ji) / sum_j exp2(...)     (log2 e is in Q')
+//   MMA1  S^T_t = X_t Q'^T            M=128 rows, N=k_pad, K=d     (TMEM, fp32)
+//   softmax over j for every row i (log2 e is folded into Q'):
+//         a_ji = exp2(s_ji - max_j s_ji) / sum_j exp2(...)
 //         rounded to bf16 and stored to shared memory as the A operand of
-//   MMA2  X~ += A_t X_t             M=k_pad, N=d, K=128        (TMEM, fp32)
-//   MASS  m  += A_t 1               M=k_pad, N=16, K=128       (TMEM, fp32)
+//   MMA2  [X~ | m] += A_t [X_t | 1]   M=k_pad, N=d+16, K=128       (TMEM, fp32)
 // The X tile in shared memory serves as the K-major A operand of MMA1 and
 // as the MN-major B operand of MMA2; X is read from HBM once.
 //
+// The masses m_j = sum_i a_ji come out of MMA2 itself: its B operand has 16
+// columns more than X, read from a block of bf16 ones, so accumulator
+// column d holds the masses, computed from the same rounded weights as X~.
+// An MN-major operand with 128-byte swizzle is read in 64-column chunks at
+// a fixed stride (the descriptor's leading byte offset), so every X stage
+// is placed such that its last two boxes and the one shared block of ones
+// lie at that stride (see Plan).  This costs MMA2 one eighth more tensor
+// time and nothing else; summing the weights over rows with the CUDA cores
+// instead (shuffles, or row-sums kept in TMEM) loads the same shared-memory
+// and tensor-memory path that the probability stores and the MMA issue
+// already saturate.
+//
 // Warp roles (384 threads):
-//   warp 0      TMA producer (X ring of kStages tiles; Q' once)
-//   warp 1      MMA issuer (one thread); MMA2 of tile t is issued after MMA1
-//               of tile t+1 so that the softmax of t overlaps MMA1 of t+1
+//   warp 0      TMA producer (X ring of Plan::S tiles; Q' once)
+//   warp 1      MMA1 issuer (one thread): as soon as an X stage has landed
+//               and its group's S^T buffer has been read out
 //   warp 2      TMEM allocation / release
-//   warps 4-7   softmax group 0 (even tiles)
+//   warp 3      MMA2 issuer (one thread): as soon as the probabilities are
+//               stored (and, for a segment's first tile, X~ was drained)
+//   warps 4-7   softmax group 0 (even tiles), one thread per row
 //   warps 8-11  softmax group 1 (odd tiles)
-// The group that finishes a segment's last tile also drains the TMEM
-// accumulator to the outputs (or to a partial slot for split users).
+// Issuing one tcgen05.mma takes a thread tens of cycles, about as long as
+// an N = 128 MMA runs, so the two kinds of MMA get a thread each, and each
+// thread waits on its own barriers only.  The two softmax groups overlap
+// one tile's exponentials with the other tile's stores; they share the one
+// probability buffer.  The group that finishes a segment's last tile drains
+// X~ and m to the outputs (or to a partial slot for a user that crosses CTA
+// ranges).
 #include "sa_internal.h"
 #include "sa_ptx.cuh"
 
@@ -33,33 +50,63 @@ namespace sa {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kRing = 16;  // issuer's ring of in-flight tile descriptors
 constexpr int kMaxDynSmem = 232448;  // 227 KB per block on sm_100
+constexpr int kBlock = 16384;        // shared memory is planned in 16 KB blocks
 
+// Shared-memory plan, in 16 KB blocks (a box is 128 rows x 64 bf16 columns,
+// 128-byte swizzled; Q' is KM x D, the probability tile KM x 128).
+//   D = 128: 4 stages.  Stage s keeps box 0 at O - 2 L_s and box 1 at
+//            O - L_s with L = {1, 3, 4, 5} and the ones at O = 12, so MMA2
+//            reads its chunks at stride L_s.  Q' at 0-1, the probability
+//            tile at 3 (and 5, stride 2, for 128 prototypes).
+//   D = 64:  8 stages at 3..10, ones at 11 (stride 11 - block), Q' at 0,
+//            the probability tile at 1 (and 2).
+//   D = 256: 2 stages; boxes 0-1 at (3, 4) and (6, 7) read as one N = 128
+//            MMA, boxes 2-3 at O - 2 L_s, O - L_s with L = {1, 3} and the
+//            ones at O = 11 read as one N = 144 MMA.  Q' at 0-1, the
+//            probability tile at 2.
+// (tests/test_host_logic.py checks that the regions are disjoint and that
+// every MMA2 operand's chunks lie at its stride.)
 template <int D, int KM>
-struct Cfg {
-  static constexpr int kQBytes = KM * D * 2;                // Q' (bf16), D/64 swizzled boxes
-  static constexpr int kXBytes = kTileRows * D * 2;         // one X tile
-  static constexpr int kPBytes = KM * kTileRows * 2;        // one probability tile
-  static constexpr int kFixed = kQBytes + 2 * kPBytes + 1024 + 1024;  // + ones/barriers + align
-  static constexpr int kStagesFit = (kMaxDynSmem - kFixed) / kXBytes;
-  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
-  static constexpr int kSmem = kFixed + kStages * kXBytes;
-  // TMEM columns (128 lanes x 512 columns of 32 bit are allocated)
-  static constexpr uint32_t kColS = 0;              // two S^T buffers: [0,KM), [KM,2KM)
-  static constexpr uint32_t kColAcc = 2 * KM;       // X~ accumulator, D columns
-  static constexpr uint32_t kColMass = 2 * KM + D;  // mass accumulator, 16 columns
-  static_assert(kColMass + 16 <= 512, "TMEM budget");
-  static_assert(kStages >= 2, "shared memory budget");
+struct Plan {
+  static_assert(D == 64 || D == 128 || D == 256, "width");
+  static_assert(KM == 64 || KM == 128, "prototype padding");
+  static_assert(D != 256 || KM == 64, "d = 256 supports up to 64 prototypes");
+  static constexpr int S = D == 64 ? 8 : (D == 128 ? 4 : 2);
+  static constexpr int kOnes = D == 128 ? 12 : 11;
+  static constexpr int kP0 = D == 64 ? 1 : (D == 128 ? 3 : 2);
+  static constexpr int kPStride = D == 128 ? 2 : 1;  // blocks between the 64-prototype chunks
+  static constexpr int kBlocks = D == 128 ? 13 : 12;
+  static constexpr int kBars = kBlocks * kBlock;     // barriers and scheduler state after the blocks
+  static constexpr int kSmem = kBars + 512;
   static_assert(kSmem <= kMaxDynSmem, "shared memory budget");
-  static_assert(D % 64 == 0 && (KM == 64 || KM == 128), "shape");
-};
+  // TMEM columns: two S^T buffers (one per softmax group), then the
+  // accumulator [X~ | m] with D + 16 columns; the masses are column D.
+  static constexpr uint32_t kColS = 0;
+  static constexpr uint32_t kColAcc = 2 * KM;
+  static_assert(kColAcc + D + 16 <= 512, "TMEM budget");
 
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
+  __host__ __device__ static constexpr int lstride(int s) {
+    return D == 128 ? (s == 0 ? 1 : s + 2) : (s == 0 ? 1 : 3);  // {1,3,4,5} / {1,3}
+  }
+  // Block of box b of stage s.
+  __host__ __device__ static constexpr int box(int s, int b) {
+    return D == 64 ? 3 + s
+         : D == 128 ? (b == 0 ? kOnes - 2 * lstride(s) : kOnes - lstride(s))
+         : (b < 2 ? (s == 0 ? 3 : 6) + b
+                  : (b == 2 ? kOnes - 2 * lstride(s) : kOnes - lstride(s)));
+  }
+  // MMA2 B operand part p (D = 256 has two): first block, chunk stride in
+  // blocks, N.
+  __host__ __device__ static constexpr int b_start(int s, int p) {
+    return D == 256 && p == 0 ? box(s, 0) : box(s, D == 256 ? 2 : 0);
+  }
+  __host__ __device__ static constexpr int b_stride(int s, int p) {
+    return D == 64 ? kOnes - box(s, 0) : (D == 256 && p == 0 ? 1 : lstride(s));
+  }
+  static constexpr int kParts = D == 256 ? 2 : 1;
+  static constexpr int kPartN0 = D == 256 ? 128 : D + 16;  // N of part 0 (part 1: 144)
+};
 
 // Warp-wide wait: every lane polls, and the warp leaves converged with one
 // common verdict (tcgen05.ld that follows is .sync.aligned).
@@ -69,40 +116,43 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
+// One arrival per warp, after every lane's prior work (callers fence first).
+__device__ __forceinline__ void warp_arrive(uint64_t* bar, int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
+
 // FULL: k == KM, so no prototype column needs masking.
 template <int D, int KM, bool FULL>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_sa_kernel(const __grid_constant__ CUtensorMap tm_x,
                     const __grid_constant__ CUtensorMap tm_q, const PassArgs a) {
-  using C = Cfg<D, KM>;
-  constexpr int S = C::kStages;
+  using Pl = Plan<D, KM>;
+  constexpr int S = Pl::S;
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* q_s = smem;
-  uint8_t* x_s = q_s + C::kQBytes;
-  uint8_t* p_s = x_s + S * C::kXBytes;
-  uint8_t* ones_s = p_s + 2 * C::kPBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ones_s + 512);
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0u) {  // the 128-byte swizzle needs 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(&a.header->timeout_flags, DEVFLAG_SMEM_ALIGN);
+    return;
+  }
+  const uint32_t sbase = smem_u32(smem);
+  uint8_t* q_s = smem;                               // Q', block 0
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Pl::kBars);
   uint64_t* x_full = bars;
   uint64_t* x_empty = bars + S;
-  uint64_t* s_full = bars + 2 * S;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;
-  uint64_t* p_empty = p_full + 2;
-  // Two acc_full barriers, used by segment parity.  A softmax group that
-  // waits for segment s cannot see a stale parity: segment s-2's
-  // aggregation was issued before the MMA1 whose completion let the group
-  // reach this tile, so that earlier phase of acc_full[s & 1] has completed.
+  uint64_t* s_full = bars + 2 * S;  // [group]
+  uint64_t* s_empty = s_full + 2;   // [group]
+  uint64_t* p_full = s_empty + 2;   // [group]: the group's probabilities are stored
+  uint64_t* p_empty = p_full + 2;   // [parity of the tile whose MMA2 freed the buffer]
+  // Two acc_full barriers, used by segment parity, so that no wait can
+  // confuse the phase of segment s with that of segment s - 2.
   uint64_t* acc_full = p_empty + 2;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* q_full = acc_empty + 1;
-  uint64_t* drain = q_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = q_full + 1;     // [issuer]: abort path, all of its MMAs done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   int64_t* b0_slot = reinterpret_cast<int64_t*>(tmem_slot + 2);
-  uint32_t* tile_ring = reinterpret_cast<uint32_t*>(b0_slot + 1);  // issuer's tile descriptors
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -117,22 +167,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < S; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 128);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&s_empty[i], 4);
+      mbar_init(&p_full[i], 4);
       mbar_init(&p_empty[i], 1);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&drain[i], 1);
     }
-    mbar_init(&acc_full[0], 1);
-    mbar_init(&acc_full[1], 1);
-    mbar_init(acc_empty, 128);
+    mbar_init(acc_empty, 4);
     mbar_init(q_full, 1);
-    mbar_init(drain, 1);
     *abort_flag = 0u;
     *b0_slot = (a.batch > 0 && R0 < R1) ? user_at_or_before(a.offsets, a.batch, R0) : a.batch;
     if (c == 0) { a.header->flags = 0u; a.header->timeout_flags = 0u; }
     fence_mbar_init();
   }
-  if (threadIdx.x < 128) {  // 512 B of bf16 ones: B operand of the mass MMA
-    reinterpret_cast<uint32_t*>(ones_s)[threadIdx.x] = 0x3F803F80u;
+  {  // the block of bf16 ones read as MMA2's extra 16 columns
+    const uint32_t ones = sbase + Pl::kOnes * kBlock;
+    for (int i = threadIdx.x; i < kBlock / 16; i += kThreads)
+      st_shared_v4(ones + i * 16, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
     fence_proxy_async_smem();
   }
   if (warp == 2) {
@@ -149,28 +200,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      mbar_arrive_expect_tx(q_full, C::kQBytes);
+      mbar_arrive_expect_tx(q_full, KM * D * 2);
 #pragma unroll
       for (int cb = 0; cb < D / 64; ++cb)
         tma_load_2d(q_s + cb * KM * 128, &tm_q, q_full, cb * 64, 0);
-      SegmentWalker w{a.offsets, a.batch, R0, R1, b0};
-      int64_t user, s, e, lo, hi;
+      TileCursor cur{SegmentWalker{a.offsets, a.batch, R0, R1, b0}};
+      int64_t r;
       uint32_t t = 0;
       bool ok = true;
-      while (ok && w.next(user, s, e, lo, hi)) {
-        for (int64_t r = s; r < e; r += kTileRows) {
-          const int st = t % S;
-          if (!mbar_wait(&x_empty[st], ((t / S) & 1u) ^ 1u, abort_flag, sticky)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&x_full[st], C::kXBytes);
-#pragma unroll
-          for (int cb = 0; cb < D / 64; ++cb)
-            tma_load_2d_hint(x_s + st * C::kXBytes + cb * 16384, &tm_x, &x_full[st], cb * 64,
-                             static_cast<int32_t>(r), pol);
-          ++t;
+      while (cur.next(r)) {
+        const int st = t % S;
+        if (!mbar_wait(&x_empty[st], ((t / S) & 1u) ^ 1u, abort_flag, sticky)) {
+          ok = false;
+          break;
         }
+        mbar_arrive_expect_tx(&x_full[st], kTileRows * D * 2);
+#pragma unroll
+        for (int cb = 0; cb < D / 64; ++cb)
+          tma_load_2d_hint(smem + Pl::box(st, cb) * kBlock, &tm_x, &x_full[st], cb * 64,
+                           static_cast<int32_t>(r), pol);
+        ++t;
       }
       if (!ok) {  // let the copies in flight land before the CTA exits
         for (uint32_t u = (t > static_cast<uint32_t>(S) ? t - S : 0u); u < t; ++u)
@@ -178,124 +227,81 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_bounded(q_full, 0);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------------ MMA issuers
+    // A commit covers the MMAs of its own thread only: MMA1's commits
+    // release S^T buffers; MMA2's release X stages (MMA2 of a tile starts
+    // after that tile's MMA1 has completed, because its probabilities were
+    // computed from the MMA1 result), the probability buffer and the
+    // accumulator.
     if (lane == 0) {
+      const int role = warp == 1 ? 0 : 1;
+      // Descriptors.  A byte offset b within shared memory is applied by
+      // adding b >> 4 to the start-address field (bits 0-13); every address
+      // stays below 2^18 bytes, so the field never carries.
+      const uint64_t xk_desc = smem_desc(sbase, 16, 1024, 2);                // X as K-major A
+      const uint64_t q_desc = smem_desc(sbase, 16, 1024, 2);                 // Q' as K-major B
+      const uint64_t p_desc =
+          smem_desc(sbase + Pl::kP0 * kBlock, Pl::kPStride * kBlock, 1024, 2);  // P, MN-major A
       constexpr uint32_t idesc_s = idesc_bf16_f32(kTileRows, KM, 0, 0);
-      constexpr uint32_t idesc_x = idesc_bf16_f32(KM, D, 1, 1);
-      constexpr uint32_t idesc_m = idesc_bf16_f32(KM, 16, 1, 0);
-      const uint32_t q_a = smem_u32(q_s);
-      const uint32_t x_a = smem_u32(x_s);
-      const uint32_t p_a = smem_u32(p_s);
-      const uint64_t ones_desc = smem_desc(smem_u32(ones_s), 128, 256, 0);
-      // Base descriptors, built once.  A byte offset b within shared memory
-      // is applied by adding b >> 4 to the start-address field (bits 0-13);
-      // every address stays below 2^18 bytes, so the field never carries.
-      // This keeps the issuing thread to one add per MMA: its own scalar
-      // latency would otherwise pace the tensor pipe.
-      const uint64_t xk_desc = smem_desc(x_a, 16, 1024, 2);      // X as K-major A
-      const uint64_t q_desc = smem_desc(q_a, 16, 1024, 2);       // Q' as K-major B
-      const uint64_t p_desc = smem_desc(p_a, 16384, 1024, 2);    // P as MN-major A
-      const uint64_t xmn_desc = smem_desc(x_a, 16384, 1024, 2);  // X as MN-major B
-      bool ok = mbar_wait(q_full, 0, abort_flag, sticky);
-      tc_fence_after();
-
-      // Non-blocking scheduler with two cursors over the CTA's tiles:
-      //   t1: next tile whose affinity MMA (MMA1) is issued, as soon as its X
-      //       stage has landed and its S^T buffer has been read out;
-      //   t2: next tile whose aggregation (MMA2 + mass) is issued, as soon as
-      //       its probabilities are in shared memory (and, for the first
-      //       tile of a user segment, the accumulator has been drained).
-      // MMA1 thus runs ahead of the softmax instead of waiting for the
-      // previous tile's aggregation.  The tensor pipe executes the issued
-      // MMAs in order.
-      // Tile descriptors of issued-but-not-aggregated tiles, in shared memory:
-      // bits 0-7 stage, bit 8 first of segment, bit 9 last, bits 10+ segment.
-      static_assert(kRing >= S + 2, "tile ring");
+      constexpr uint32_t idesc_x0 = idesc_bf16_f32(KM, Pl::kPartN0, 1, 1);
+      constexpr uint32_t idesc_x1 = idesc_bf16_f32(KM, 144, 1, 1);
+      bool ok = role == 1 || mbar_wait(q_full, 0, abort_flag, sticky);
       SegmentWalker w{a.offsets, a.batch, R0, R1, b0};
-      int64_t user = 0, s = 0, e = 0, lo = 0, hi = 0, r = 0;
-      bool have_seg = false, walker_done = false;
-      uint32_t t1 = 0, t2 = 0, seg = 0;
-      long long idle_since = cycles_now();
-      while (ok) {
-        bool progressed = false;
-        // ---- MMA1 for tile t1
-        if (!walker_done) {
-          if (!have_seg) {
-            have_seg = w.next(user, s, e, lo, hi);
-            if (have_seg) r = s; else walker_done = true;
-          }
-          if (have_seg) {
-            const int st = t1 % S;
-            const int sb = t1 & 1;
-            if (mbar_test_wait(&x_full[st], (t1 / S) & 1u) &&
-                mbar_test_wait(&s_empty[sb], ((t1 >> 1) & 1u) ^ 1u)) {
-              tc_fence_after();
-              const uint64_t xd = xk_desc + ((st * C::kXBytes) >> 4);
-              const uint32_t dcol = tmem + C::kColS + sb * KM;
-#pragma unroll
-              for (int ks = 0; ks < D / 16; ++ks) {
-                mma_bf16_ss(dcol, xd + (((ks >> 2) * 16384 + (ks & 3) * 32) >> 4),
-                            q_desc + (((ks >> 2) * (KM * 128) + (ks & 3) * 32) >> 4), idesc_s,
-                            ks > 0 ? 1u : 0u);
-              }
-              mma_commit(&s_full[sb]);
-              tile_ring[t1 % kRing] = static_cast<uint32_t>(st) | (r == s ? 0x100u : 0u) |
-                                      (r + kTileRows >= e ? 0x200u : 0u) | (seg << 10);
-              ++t1;
-              r += kTileRows;
-              if (r >= e) { have_seg = false; ++seg; }
-              progressed = true;
+      int64_t user, s, e, lo, hi;
+      uint32_t t = 0, seg = 0;
+      while (ok && w.next(user, s, e, lo, hi)) {
+        for (int64_t r = s; r < e; r += kTileRows, ++t) {
+          const int st = t % S;
+          if (role == 0) {
+            // ---- MMA1: S^T_t = X_t Q'^T into the S^T buffer of tile t's group
+            const int sb = t & 1;
+            if (!mbar_wait(&x_full[st], (t / S) & 1u, abort_flag, sticky) ||
+                !mbar_wait(&s_empty[sb], ((t >> 1) & 1u) ^ 1u, abort_flag, sticky)) {
+              ok = false;
+              break;
             }
-          }
-        }
-        // ---- MMA2 + mass for tile t2
-        if (t2 < t1) {
-          const uint32_t desc = tile_ring[t2 % kRing];
-          const bool first = desc & 0x100u;
-          const bool last = desc & 0x200u;
-          const uint32_t sg = desc >> 10;
-          const int pb = t2 & 1;
-          if (mbar_test_wait(&p_full[pb], (t2 >> 1) & 1u) &&
-              (!first || mbar_test_wait(acc_empty, (sg & 1u) ^ 1u))) {
             tc_fence_after();
-            const int st = static_cast<int>(desc & 0xFFu);
-            const uint64_t pd = p_desc + ((pb * C::kPBytes) >> 4);
-            const uint64_t xd = xmn_desc + ((st * C::kXBytes) >> 4);
-            const uint32_t acc0 = (!first) ? 1u : 0u;
+            const uint32_t dcol = tmem + Pl::kColS + sb * KM;
 #pragma unroll
-            for (int ks = 0; ks < kTileRows / 16; ++ks)
-              mma_bf16_ss(tmem + C::kColAcc, pd + ((ks * 2048) >> 4), xd + ((ks * 2048) >> 4),
-                          idesc_x, ks > 0 ? 1u : acc0);
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_bf16_ss(dcol, xk_desc + ((Pl::box(st, ks >> 2) * kBlock + (ks & 3) * 32) >> 4),
+                          q_desc + (((ks >> 2) * (KM * 128) + (ks & 3) * 32) >> 4), idesc_s,
+                          ks > 0 ? 1u : 0u);
+            mma_commit(&s_full[sb]);
+          } else {
+            // ---- MMA2: [X~ | m] += A_t [X_t | 1]  (a segment's first tile overwrites)
+            const bool first = (r == s);
+            const bool last = (r + kTileRows >= e);
+            if (!mbar_wait(&p_full[t & 1u], (t >> 1) & 1u, abort_flag, sticky) ||
+                (first && !mbar_wait(acc_empty, (seg & 1u) ^ 1u, abort_flag, sticky))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t acc0 = first ? 0u : 1u;
+            const uint64_t bd0 = smem_desc(sbase + Pl::b_start(st, 0) * kBlock,
+                                           Pl::b_stride(st, 0) * kBlock, 1024, 2);
+            const uint64_t bd1 = smem_desc(sbase + Pl::b_start(st, 1) * kBlock,
+                                           Pl::b_stride(st, 1) * kBlock, 1024, 2);
 #pragma unroll
-            for (int ks = 0; ks < kTileRows / 16; ++ks)
-              mma_bf16_ss(tmem + C::kColMass, pd + ((ks * 2048) >> 4), ones_desc, idesc_m,
-                          ks > 0 ? 1u : acc0);
+            for (int ks = 0; ks < kTileRows / 16; ++ks) {
+              mma_bf16_ss(tmem + Pl::kColAcc, p_desc + ((ks * 2048) >> 4), bd0 + ((ks * 2048) >> 4),
+                          idesc_x0, ks > 0 ? 1u : acc0);
+              if (Pl::kParts == 2)
+                mma_bf16_ss(tmem + Pl::kColAcc + 128, p_desc + ((ks * 2048) >> 4),
+                            bd1 + ((ks * 2048) >> 4), idesc_x1, ks > 0 ? 1u : acc0);
+            }
             mma_commit(&x_empty[st]);
-            mma_commit(&p_empty[pb]);
-            if (last) mma_commit(&acc_full[sg & 1u]);
-            ++t2;
-            progressed = true;
+            mma_commit(&p_empty[t & 1u]);
+            if (last) mma_commit(&acc_full[seg & 1u]);
           }
         }
-        if (walker_done && t2 == t1) break;
-        if (progressed) {
-          idle_since = cycles_now();
-        } else if (!*abort_flag && cycles_now() - idle_since <= kWaitTimeoutCycles) {
-          // Nothing ready: back off briefly so that this polling thread does
-          // not take issue slots from the softmax warps on its SM sub-partition.
-          __nanosleep(64);
-        } else if (*abort_flag) {
-          ok = false;
-        } else if (cycles_now() - idle_since > kWaitTimeoutCycles) {
-          *abort_flag = 1u;
-          atomicOr(sticky, DEVFLAG_TIMEOUT);
-          ok = false;
-        }
+        ++seg;
       }
-      if (!ok) {  // make sure no MMA is still running when TMEM is released
-        mma_commit(drain);
-        mbar_wait_bounded(drain, 0);
+      if (!ok) {  // make sure none of this thread's MMAs still runs when TMEM is released
+        mma_commit(&drain[role]);
+        mbar_wait_bounded(&drain[role], 0);
       }
     }
   } else if (warp >= 4) {
@@ -321,72 +327,96 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t sr[KM / 32][32];
 #pragma unroll
         for (int cc = 0; cc < KM / 32; ++cc)
-          tmem_ld32(lane_addr + C::kColS + grp * KM + cc * 32, sr[cc]);
+          tmem_ld32(lane_addr + Pl::kColS + grp * KM + cc * 32, sr[cc]);
         tmem_wait_ld();
 #pragma unroll
         for (int cc = 0; cc < KM / 32; ++cc) tmem_pin32(sr[cc]);
         tc_fence_before();
-        mbar_arrive(&s_empty[grp]);
+        warp_arrive(&s_empty[grp], lane);
 
-        // stable softmax over the prototype axis (thread-local); eight
-        // independent max / sum chains keep the FP pipes busy
-        float mx8[8], sm8[8];
+        // Stable softmax over the prototype axis (thread-local): four
+        // independent max chains (three-input max) and four packed sums.
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+        for (int j = 0; j < KM; j += 8) {
 #pragma unroll
-        for (int j = 0; j < KM; ++j)
-          if (FULL || j < k) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(sr[j >> 5][j & 31]));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sm8[i] = 0.f;
-        float pv[KM];
-#pragma unroll
-        for (int j = 0; j < KM; ++j) {
-          const float ev = (FULL || j < k) ? ex2_approx(__uint_as_float(sr[j >> 5][j & 31]) - mx) : 0.f;
-          pv[j] = ev;
-          sm8[j & 7] += ev;
-        }
-        const float sum = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
-        const float inv = 1.0f / sum;
-
-        if (!warp_wait(&p_empty[grp], ((t >> 1) & 1u) ^ 1u, abort_flag, sticky)) { ok = false; break; }
-        // Row `row` of the probability tile, MN-major with 128-byte swizzle:
-        // 64-prototype blocks 16 KB apart, 8-row groups 1 KB apart, the
-        // 16-byte chunk index XOR-ed with (row mod 8).
-        const uint32_t prow = smem_u32(p_s + grp * C::kPBytes) + (row >> 3) * 1024 + (row & 7) * 128;
-#pragma unroll
-        for (int mb = 0; mb < KM / 64; ++mb) {
-#pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            const int j0 = mb * 64 + c8 * 8;
-            uint32_t wv[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h)
-              wv[h] = valid ? pack_bf16x2(pv[j0 + 2 * h] * inv, pv[j0 + 2 * h + 1] * inv) : 0u;
-            st_shared_v4(prow + mb * 16384 + ((c8 ^ (row & 7)) << 4), wv[0], wv[1], wv[2], wv[3]);
+          for (int u = 0; u < 4; ++u) {
+            const int ja = j + 2 * u, jb = ja + 1;
+            const float va = (FULL || ja < k) ? __uint_as_float(sr[ja >> 5][ja & 31]) : -INFINITY;
+            const float vb = (FULL || jb < k) ? __uint_as_float(sr[jb >> 5][jb & 31]) : -INFINITY;
+            mx4[u] = max3f(mx4[u], va, vb);
           }
         }
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        const uint64_t neg_m = f2_pack(-mx, -mx);
+        uint64_t z2[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int j = 0; j < KM; j += 2) {
+          float x0, x1;
+          f2_unpack(f2_add(f2_pack(__uint_as_float(sr[j >> 5][j & 31]),
+                                   __uint_as_float(sr[(j + 1) >> 5][(j + 1) & 31])),
+                           neg_m),
+                    x0, x1);
+          const float e0 = (FULL || j < k) ? ex2_approx(x0) : 0.f;
+          const float e1 = (FULL || j + 1 < k) ? ex2_approx(x1) : 0.f;
+          sr[j >> 5][j & 31] = __float_as_uint(e0);
+          sr[(j + 1) >> 5][(j + 1) & 31] = __float_as_uint(e1);
+          z2[(j >> 1) & 3] = f2_add(z2[(j >> 1) & 3], f2_pack(e0, e1));
+        }
+        float za, zb, zc, zd;
+        f2_unpack(f2_add(z2[0], z2[1]), za, zb);
+        f2_unpack(f2_add(z2[2], z2[3]), zc, zd);
+        const float inv = valid ? 1.0f / ((za + zb) + (zc + zd)) : 0.f;
+        const uint64_t inv2 = f2_pack(inv, inv);
+
+        // The probability buffer is free once the previous tile's MMA2 (of
+        // the other group) has completed.
+        if (t > 0 && !warp_wait(&p_empty[(t - 1) & 1u], ((t - 1) >> 1) & 1u, abort_flag, sticky)) {
+          ok = false;
+          break;
+        }
+        // Row `row` of the probability tile, MN-major with 128-byte swizzle:
+        // 64-prototype chunks kPStride blocks apart, 8-row groups 1 KB apart,
+        // the 16-byte unit index XOR-ed with (row mod 8).  Rows past the
+        // segment's end may hold NaN (another user's data): their weights
+        // are forced to zero, not scaled by zero.
+        const uint32_t prow = sbase + Pl::kP0 * kBlock + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+        for (int c8 = 0; c8 < KM / 8; ++c8) {
+          uint32_t pw[4];
+#pragma unroll
+          for (int hh = 0; hh < 4; ++hh) {
+            const int j = c8 * 8 + 2 * hh;
+            float p0, p1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(sr[j >> 5][j & 31]),
+                                     __uint_as_float(sr[(j + 1) >> 5][(j + 1) & 31])),
+                             inv2),
+                      p0, p1);
+            pw[hh] = valid ? pack_bf16x2(p0, p1) : 0u;
+          }
+          st_shared_v4(prow + (c8 >> 3) * (Pl::kPStride * kBlock) + (((c8 & 7) ^ (row & 7)) << 4),
+                       pw[0], pw[1], pw[2], pw[3]);
+        }
         if (!valid) {
-          // Rows past the segment's end hold another user's data (or TMA
-          // zero fill).  Their weights are zero, but 0 * NaN is NaN, so the
-          // rows themselves are cleared before the aggregation reads them.
-          const uint32_t xrow = smem_u32(x_s + st * C::kXBytes) + row * 128;
+          // The rows themselves are cleared too, because 0 * NaN is NaN in
+          // the aggregation (the block of ones is never touched).
 #pragma unroll
-          for (int cb = 0; cb < D / 64; ++cb)
+          for (int cb = 0; cb < D / 64; ++cb) {
+            const uint32_t xrow = sbase + Pl::box(st, cb) * kBlock + row * 128;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) st_shared_v4(xrow + cb * 16384 + i * 16, 0u, 0u, 0u, 0u);
+            for (int i = 0; i < 8; ++i) st_shared_v4(xrow + i * 16, 0u, 0u, 0u, 0u);
+          }
         }
         fence_proxy_async_smem();
-        mbar_arrive(&p_full[grp]);
+        warp_arrive(&p_full[grp], lane);
 
         if (last) {
           // ---------------------------------------------- drain X~ and m
           if (!warp_wait(&acc_full[seg & 1u], (seg >> 1) & 1u, abort_flag, sticky)) { ok = false; break; }
           tc_fence_after();
-          const int64_t slot = segment_slot(c, lo, hi, R0, R1);
-          float* dx = slot < 0 ? a.out_x + user * k * D : a.part_x + slot * k * D;
-          float* dm = slot < 0 ? a.out_m + user * k : a.part_m + slot * k;
+          const int64_t slotp = segment_slot(c, lo, hi, R0, R1);
+          float* dx = slotp < 0 ? a.out_x + user * k * D : a.part_x + slotp * k * D;
+          float* dm = slotp < 0 ? a.out_m + user * k : a.part_m + slotp * k;
           // M=128: prototype j sits in TMEM lane j.  M=64: prototypes
           // 16q..16q+15 sit in lanes 32q..32q+15.
           const int j = (KM == 128) ? row : q * 16 + lane;
@@ -394,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t v[32];
-            tmem_ld32(lane_addr + C::kColAcc + cc * 32, v);
+            tmem_ld32(lane_addr + Pl::kColAcc + cc * 32, v);
             tmem_wait_ld();
             tmem_pin32(v);
             if (has) {
@@ -406,12 +436,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           uint32_t mv;
-          tmem_ld1(lane_addr + C::kColMass, mv);
+          tmem_ld1(lane_addr + Pl::kColAcc + D, mv);
           tmem_wait_ld();
           tmem_pin1(mv);
           if (has) dm[j] = __uint_as_float(mv);
           tc_fence_before();
-          mbar_arrive(acc_empty);
+          warp_arrive(acc_empty, lane);
         }
       }
       ++seg;
@@ -431,9 +461,9 @@ cudaError_t launch_one(const CUtensorMap& tx, const CUtensorMap& tq, const PassA
                        int grid, cudaStream_t stream) {
   auto kern = a.k == KM ? fused_sa_kernel<D, KM, true> : fused_sa_kernel<D, KM, false>;
   cudaError_t err =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D, KM>::kSmem);
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Plan<D, KM>::kSmem);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kThreads, Cfg<D, KM>::kSmem, stream>>>(tx, tq, a);
+  kern<<<grid, kThreads, Plan<D, KM>::kSmem, stream>>>(tx, tq, a);
   return cudaGetLastError();
 }
 
@@ -445,9 +475,9 @@ bool fused_bf16_supported(int d, int k_pad) {
 }
 
 size_t fused_bf16_smem_bytes(int d, int k_pad) {
-  if (d == 64) return k_pad == 64 ? Cfg<64, 64>::kSmem : Cfg<64, 128>::kSmem;
-  if (d == 128) return k_pad == 64 ? Cfg<128, 64>::kSmem : Cfg<128, 128>::kSmem;
-  return Cfg<256, 64>::kSmem;
+  if (d == 64) return k_pad == 64 ? Plan<64, 64>::kSmem : Plan<64, 128>::kSmem;
+  if (d == 128) return k_pad == 64 ? Plan<128, 64>::kSmem : Plan<128, 128>::kSmem;
+  return Plan<256, 64>::kSmem;
 }
 
 cudaError_t launch_fused_bf16(const CUtensorMap& tx, const CUtensorMap& tq, int k_pad,

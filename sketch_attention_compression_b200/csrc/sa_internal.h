@@ -83,6 +83,27 @@ struct SegmentWalker {
   }
 };
 
+// Walks the tiles of one CTA's row range: each call yields the first row of
+// the next 128-row tile (tiles never straddle a segment start).
+struct TileCursor {
+  SegmentWalker w;
+  int64_t r = 0, e = 0;
+  bool have = false;
+  SA_HD bool next(int64_t& row) {
+    if (have && r + kTileRows < e) {
+      r += kTileRows;
+      row = r;
+      return true;
+    }
+    int64_t user, s, lo, hi;
+    have = w.next(user, s, e, lo, hi);
+    if (!have) return false;
+    r = s;
+    row = r;
+    return true;
+  }
+};
+
 // Partial slot of a split user's segment in CTA c, or -1 if the user lies
 // wholly inside the CTA's range (then it goes straight to the outputs).
 SA_HD int64_t segment_slot(int64_t c, int64_t lo, int64_t hi, int64_t R0, int64_t R1) {
