@@ -87,8 +87,9 @@ typedef struct sa_query_s* sa_query;
  * Allocates device memory (cudaMalloc) for Q'.  P, W_Q and W_K are read by
  * a kernel enqueued on `stream`; they must stay alive until it completes.
  * Returns SA_ERR_UNSUPPORTED for bf16 shapes without a tensor-core kernel
- * (currently bf16 needs k <= 128 for d = 64/128 and k <= 64 for d = 256) or
- * for a GPU other than sm_100.
+ * (bf16 supports k <= 128 for d = 64 and 128, and any k <= 256 for d = 256,
+ * where k > 64 runs on pairs of CTAs that split the prototypes) or for a
+ * GPU other than sm_100.
  */
 sa_status sa_prepare_query(const void* P, const void* W_Q, const void* W_K, int k, int d,
                            float scale, sa_dtype dtype, void* stream, sa_query* out);

@@ -21,7 +21,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "_lib", "libsa.so")
 SOURCES = ["sa_api.cu", "sa_prepare.cu", "sa_fused.cu", "sa_simt.cu", "sa_finalize.cu",
-           "sa_noalloc.cu"]
+           "sa_noalloc.cu", "sa_fused_pair.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
           "-I", os.path.join(ROOT, "include"), "-I", CSRC]

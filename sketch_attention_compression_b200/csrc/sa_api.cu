@@ -11,13 +11,15 @@
 struct sa_query_s {
   int device;
   int sms;
+  int pair_units;  // co-resident two-CTA clusters (k_pad == 256)
   int k;
   int d;
   int k_pad;  // prototype rows of the bf16 Q' copy (multiple of 64), 0 for fp32
   sa_dtype dtype;
   float* q_f32;      // [k][d]
   uint16_t* q_bf16;  // [k_pad][d], rows >= k zero
-  CUtensorMap tmap_q;
+  CUtensorMap tmap_q;       // boxes of k_pad rows (k_pad <= 128)
+  CUtensorMap tmap_q_half;  // boxes of 128 rows (k_pad == 256: one half per CTA of a pair)
 };
 
 namespace {
@@ -62,9 +64,12 @@ constexpr int64_t kMaxRows = (int64_t{1} << 31) - 256;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Number of CTA row ranges: one per SM, or one per pair of SMs for the
+// two-CTA pass (256 padded prototypes).
 int64_t grid_for(const sa_query_s* q, int64_t total_rows) {
   const int64_t T = sa::tiles_of(total_rows);
-  int64_t G = T < q->sms ? T : q->sms;
+  const int64_t units = (q->dtype == SA_BF16 && q->k_pad == 256) ? q->pair_units : q->sms;
+  int64_t G = T < units ? T : units;
   return G < 1 ? 1 : G;
 }
 
@@ -134,7 +139,8 @@ sa_status run(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
                           : make_tmap_bf16(&tmx, q->q_bf16, static_cast<uint64_t>(q->k_pad),
                                            static_cast<uint64_t>(q->d), 64);
       if (!ok) return SA_ERR_CUDA;
-      err = sa::launch_fused_bf16(tmx, q->tmap_q, q->k_pad, a, G, st);
+      err = q->k_pad == 256 ? sa::launch_fused_bf16_pair(tmx, q->tmap_q_half, a, G, st)
+                            : sa::launch_fused_bf16(tmx, q->tmap_q, q->k_pad, a, G, st);
     } else {
       err = sa::launch_simt_fp32(q->q_f32, static_cast<const float*>(X), a, G, st);
     }
@@ -183,7 +189,8 @@ sa_status sa_prepare_query(const void* P, const void* W_Q, const void* W_K, int 
 
   int k_pad = 0;
   if (dtype == SA_BF16) {
-    k_pad = k <= 64 ? 64 : (k <= 128 ? 128 : 256);
+    // d = 256 with more than 64 prototypes runs on CTA pairs (256 padded).
+    k_pad = k <= 64 ? 64 : ((k <= 128 && d != 256) ? 128 : 256);
     if (!sa::fused_bf16_supported(d, k_pad)) return SA_ERR_UNSUPPORTED;
   }
 
@@ -192,6 +199,14 @@ sa_status sa_prepare_query(const void* P, const void* W_Q, const void* W_K, int 
   memset(q, 0, sizeof(*q));
   q->device = dev;
   q->sms = sms;
+  if (dtype == SA_BF16 && k_pad == 256) {
+    const int n = sa::fused_bf16_pair_max_clusters();
+    if (n < 1) {
+      delete q;
+      return SA_ERR_UNSUPPORTED;
+    }
+    q->pair_units = n < sms / 2 ? n : sms / 2;
+  }
   q->k = k;
   q->d = d;
   q->k_pad = k_pad;
@@ -201,8 +216,9 @@ sa_status sa_prepare_query(const void* P, const void* W_Q, const void* W_K, int 
   if (ok && dtype == SA_BF16) {
     const size_t qb = static_cast<size_t>(k_pad) * d * sizeof(uint16_t);
     ok = cudaMalloc(&q->q_bf16, qb) == cudaSuccess && cudaMemsetAsync(q->q_bf16, 0, qb, st) == cudaSuccess;
-    ok = ok && make_tmap_bf16(&q->tmap_q, q->q_bf16, static_cast<uint64_t>(k_pad),
-                              static_cast<uint64_t>(d), static_cast<uint32_t>(k_pad));
+    ok = ok && make_tmap_bf16(k_pad == 256 ? &q->tmap_q_half : &q->tmap_q, q->q_bf16,
+                              static_cast<uint64_t>(k_pad), static_cast<uint64_t>(d),
+                              static_cast<uint32_t>(k_pad == 256 ? 128 : k_pad));
   }
   ok = ok && sa::launch_prepare_query(P, W_Q, W_K, k, d, static_cast<double>(scale),
                                       dtype == SA_BF16, q->q_f32, q->q_bf16, st) == cudaSuccess;

@@ -416,13 +416,8 @@ cudaError_t launch_one(const CUtensorMap& tx, const CUtensorMap& tq, const PassA
 
 bool fused_bf16_supported(int d, int k_pad) {
   return (d == 64 && (k_pad == 64 || k_pad == 128)) ||
-         (d == 128 && (k_pad == 64 || k_pad == 128)) || (d == 256 && k_pad == 64);
-}
-
-size_t fused_bf16_smem_bytes(int d, int k_pad) {
-  if (d == 64) return k_pad == 64 ? Plan<64, 64>::kSmem : Plan<64, 128>::kSmem;
-  if (d == 128) return k_pad == 64 ? Plan<128, 64>::kSmem : Plan<128, 128>::kSmem;
-  return Plan<256, 64>::kSmem;
+         (d == 128 && (k_pad == 64 || k_pad == 128)) ||
+         (d == 256 && (k_pad == 64 || k_pad == 256));  // 256: the two-CTA pass
 }
 
 cudaError_t launch_fused_bf16(const CUtensorMap& tx, const CUtensorMap& tq, int k_pad,

@@ -140,7 +140,14 @@ cudaError_t launch_prepare_query(const void* P, const void* W_Q, const void* W_K
 cudaError_t launch_fused_bf16(const CUtensorMap& tmap_x, const CUtensorMap& tmap_q,
                               int k_pad, const PassArgs& a, int grid, cudaStream_t stream);
 bool fused_bf16_supported(int d, int k_pad);
-size_t fused_bf16_smem_bytes(int d, int k_pad);
+
+// Tensor-core pass for d = 256 and 129..256 prototypes: clusters of two CTAs,
+// one per prototype half; `ranges` row ranges, 2 * ranges CTAs.  tmap_q_half
+// reads 128-row boxes of the padded Q' (256 x 256).
+cudaError_t launch_fused_bf16_pair(const CUtensorMap& tmap_x, const CUtensorMap& tmap_q_half,
+                                   const PassArgs& a, int ranges, cudaStream_t stream);
+// How many two-CTA clusters of that pass fit on the GPU at once (0 on error).
+int fused_bf16_pair_max_clusters();
 
 // fp32 CUDA-core pass.
 cudaError_t launch_simt_fp32(const float* q_f32, const float* X, const PassArgs& a, int grid,

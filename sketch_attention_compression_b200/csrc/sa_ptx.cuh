@@ -317,6 +317,71 @@ __device__ __forceinline__ void ld_shared_v2f(uint32_t addr, float& a, float& b)
   asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(a), "=f"(b) : "r"(addr) : "memory");
 }
 
+// ---------------------------------------------------------------- clusters
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// All threads of all CTAs of the cluster (every warp must execute it).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// The address of this CTA's shared variable at `local` in the shared memory
+// of CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_cta(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+
+// Stores two floats into another CTA's shared memory and signals them as
+// 8 transaction bytes on that CTA's mbarrier (both addresses from
+// map_to_cta).
+__device__ __forceinline__ void st_async_v2f(uint32_t remote, float a, float b,
+                                             uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
+          remote),
+      "f"(a), "f"(b), "r"(remote_bar)
+      : "memory");
+}
+
+// try_wait with cluster-scope acquire: for data that other CTAs of the
+// cluster delivered with st.async.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait with cluster-scope acquire (same contract as mbar_wait).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile uint32_t* abort_flag,
+                                                  uint32_t* sticky_flag) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const long long t0 = cycles_now();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (cycles_now() - t0 > kWaitTimeoutCycles) {
+      *abort_flag = 1u;
+      atomicOr(sticky_flag, DEVFLAG_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- packed fp32
 // sm_100 executes these on pairs of fp32 values held in one 64-bit register
 // pair, halving the instruction count of element-wise work.

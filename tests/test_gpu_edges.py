@@ -29,7 +29,8 @@ def _full_parity(inp):
 
 
 @pytest.mark.parametrize("d,k", [(64, 64), (64, 128), (128, 64), (128, 128), (256, 64),
-                                 (128, 5), (128, 100), (64, 1), (128, 33)])
+                                 (128, 5), (128, 100), (64, 1), (128, 33),
+                                 (256, 256), (256, 200), (256, 65)])
 def test_ragged_tails_bf16(d, k):
     _full_parity(make_inputs(RAGGED, d=d, k=k, dtype="bf16", seed=d * 1000 + k))
 
@@ -180,3 +181,15 @@ def test_partials_then_finalize_equals_forward():
     q.partials(dev["X"], dev["offsets"], Xt2, m2, ws)
     q.finalize(dev["X"], dev["offsets"], Xt2, m2, ws)
     assert torch.equal(Xt, Xt2) and torch.equal(m, m2)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_more_than_128_prototypes_needs_d256(d):
+    """bf16 with k > 128 has a kernel only for d = 256 (pairs of CTAs split
+    the prototypes); other widths report SA_ERR_UNSUPPORTED on the host."""
+    from sketch_attention_compression_b200 import SAError, SketchQuery
+    from sketch_attention_compression_b200.binding import SA_ERR_UNSUPPORTED
+    dev = to_device(make_inputs([10], d=d, k=129, dtype="bf16", seed=24))
+    with pytest.raises(SAError) as e:
+        SketchQuery(dev["P"], dev["W_Q"], dev["W_K"], 0.1)
+    assert e.value.status == SA_ERR_UNSUPPORTED
