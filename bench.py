@@ -47,6 +47,7 @@ DEFAULT_WORKLOAD = "batch16_n100k_d128_k128_mixture_bf16"
 L2_BYTES = 126e6
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 KERNEL_SOURCES = ["sketch_attention_compression_b200/csrc/sa_fused.cu",
+                  "sketch_attention_compression_b200/csrc/sa_plan.h",
                   "sketch_attention_compression_b200/csrc/sa_ptx.cuh",
                   "sketch_attention_compression_b200/csrc/sa_internal.h"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fused_sa_batch16_n100k_d128_k128.md")
@@ -87,59 +88,100 @@ def load_traffic():
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock, power draw and clock-event (throttle) reasons of
+    one GPU while the timed region runs.  Reads only; changes no setting.
+
+    NVML is polled about every millisecond from a thread, so that even a
+    timed region of a few milliseconds gets samples; without NVML it falls
+    back to nvidia-smi at 50 ms."""
+
+    REASONS = [("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap")]
 
     def __init__(self, uuid: str):
         self.uuid = uuid
-        self.proc = None
-        self.lines = []
+        self.samples = []  # (sm_mhz, max_mhz, watts, reason_bits)
+        self.stop_flag = threading.Event()
         self.thread = None
+        self.nvml = None
+        self.proc = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-            return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            pynvml.nvmlInit()
+            handle = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.nvml = (pynvml, handle)
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+        except Exception:
+            self.nvml = None
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "--query-gpu=uuid,clocks.sm,clocks.max.sm,power.draw,"
+                     "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                     "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                     "--format=csv,noheader,nounits", "-lms", "50"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                return
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
         self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _poll_nvml(self):
+        pynvml, h = self.nvml
+        bits = {name: getattr(pynvml, const, 0) for name, const in self.REASONS}
+        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self.stop_flag.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, mx, pw, {n for n, b in bits.items() if rs & b}))
+            except Exception:
+                pass
+            time.sleep(0.001)
 
-    def stop(self):
-        if self.proc is None:
-            return None
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.thread.join(timeout=5)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9 or (self.uuid and parts[0] != self.uuid):
+    def _read_smi(self):
+        names = [n for n, _ in self.REASONS]
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8 or (self.uuid and parts[0] != self.uuid):
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
+                self.samples.append((float(parts[1]), float(parts[2]), float(parts[3]),
+                                     {n for n, v in zip(names, parts[4:8]) if v.lower() == "active"}))
             except ValueError:
                 continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        if not sm:
+
+    def mark(self) -> int:
+        return len(self.samples)
+
+    def stop(self):
+        self.stop_flag.set()
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, first: int = 0, last=None):
+        rows = self.samples[first:last]
+        if not rows:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        reasons = set()
+        for r in rows:
+            reasons |= r[3]
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_median": round(statistics.median(r[2] for r in rows), 1),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "source": "nvml" if self.nvml else "nvidia-smi"}
 
 
 # ---------------------------------------------------------------------------
@@ -273,10 +315,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         uuid = str(torch.cuda.get_device_properties(dev).uuid)
         sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
         sampler.start()
-        time.sleep(0.3)
+        time.sleep(0.05)
 
     # -- timed region A: the product call, back to back -------------------
-    launches = 0
+    launches = 0  # kernels of this library launched in region A
+    mark_a = sampler.mark() if sampler else 0
     barrier()
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
@@ -289,6 +332,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize(dev)
     barrier()
     step_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    mark_a_end = sampler.mark() if sampler else 0
 
     # -- timed region B: the two passes split by events (kernel durations) --
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(3 * args.steps)]
@@ -330,7 +374,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     e2e_ms = max_over_ranks(h0.elapsed_time(h1) / e2e_steps)
 
     if sampler is not None:
-        clocks = sampler.stop()
+        sampler.stop()
+        # the kernel-only regions A and B (region C is mostly host copies)
+        clocks = sampler.summary(mark_a, mark_a_end) or sampler.summary(mark_a)
 
     # sanity on the last outputs: every behaviour spreads unit mass
     msum = m.sum(dim=1).double().cpu().numpy()
@@ -393,7 +439,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 "h2d_bytes_per_step": int(bytes_x + 8 * (B + 1)),
                 "d2h_bytes_per_step": int(4 * B * w.k * (w.d + 1)),
                 "ms_per_step": e2e_ms},
-        "gpu_launches": launches * 2 + 2 * e2e_steps + 2,
+        "gpu_launches": launches,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
