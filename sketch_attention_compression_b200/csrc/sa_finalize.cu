@@ -38,7 +38,18 @@ __global__ void __launch_bounds__(kFinThreads)
     const int ch = blockIdx.x % chunks;
     const int64_t Rc = cta_row_begin(cb, G, T, N);
     const int64_t Rp = cta_row_begin(cb - 1, G, T, N);
-    const int64_t b = user_at_or_before(a.offsets, B, Rc);
+    // The user whose rows contain Rc: with valid offsets only one non-empty
+    // user does, so one parallel pass over the offsets finds it (a binary
+    // search would chain its loads end to end).  With invalid offsets any
+    // match is taken; the outputs are then unspecified but stay in bounds.
+    __shared__ long long s_user;
+    if (threadIdx.x == 0) s_user = -1;
+    __syncthreads();
+    for (int64_t i = threadIdx.x; i < B; i += kFinThreads)
+      if (a.offsets[i] <= Rc && Rc < a.offsets[i + 1]) s_user = i;
+    __syncthreads();
+    if (s_user < 0) return;
+    const int64_t b = s_user;
     const int64_t lo = a.offsets[b], hi = a.offsets[b + 1];
     if (!(lo < Rc && lo >= Rp && hi > Rc)) return;  // not split here, or owned elsewhere
     int64_t c_hi = cta_of_row(hi - 1 < N - 1 ? hi - 1 : N - 1, G, T);
@@ -49,18 +60,36 @@ __global__ void __launch_bounds__(kFinThreads)
     const int64_t e0 = static_cast<int64_t>(ch) * kChunkFloats;
     const int64_t e1 = (e0 + kChunkFloats) < kd ? (e0 + kChunkFloats) : kd;
     float* out = a.out_x + b * kd;
+    // The slots are read in batches of independent loads (a user spans
+    // about ten CTA ranges; loading them one after another would put their
+    // latencies end to end) and added in ascending CTA order, the fixed order
+    // that makes the result bitwise reproducible.
+    constexpr int kBatch = 8;
     for (int64_t i = e0 + 4 * threadIdx.x; i < e1; i += 4 * kFinThreads) {
       float4 s = *reinterpret_cast<const float4*>(a.part_x + slot_lo * kd + i);
-      for (int64_t cc = c_lo + 1; cc <= c_hi; ++cc) {
-        const float4 v = *reinterpret_cast<const float4*>(a.part_x + (2 * cc) * kd + i);
-        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+      for (int64_t cc = c_lo + 1; cc <= c_hi; cc += kBatch) {
+        float4 v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+          if (cc + u <= c_hi) v[u] = *reinterpret_cast<const float4*>(a.part_x + (2 * (cc + u)) * kd + i);
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+          if (cc + u <= c_hi) { s.x += v[u].x; s.y += v[u].y; s.z += v[u].z; s.w += v[u].w; }
       }
       *reinterpret_cast<float4*>(out + i) = s;
     }
     if (ch == 0) {
       for (int j = threadIdx.x; j < k; j += kFinThreads) {
         float s = a.part_m[slot_lo * k + j];
-        for (int64_t cc = c_lo + 1; cc <= c_hi; ++cc) s += a.part_m[(2 * cc) * k + j];
+        for (int64_t cc = c_lo + 1; cc <= c_hi; cc += kBatch) {
+          float v[kBatch];
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u)
+            if (cc + u <= c_hi) v[u] = a.part_m[(2 * (cc + u)) * k + j];
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u)
+            if (cc + u <= c_hi) s += v[u];
+        }
         a.out_m[b * k + j] = s;
       }
     }
