@@ -67,11 +67,41 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar, int lane) {
   if (lane == 0) mbar_arrive(bar);
 }
 
+// MMA1 of tile t is issued only after MMA2 of tile t - kMma1Lead has been
+// issued.  The tensor pipe runs MMAs in issue order; MMA2 frees the X stage
+// and the probability buffer, so it must not queue behind affinities that no
+// softmax group needs yet.  The lead still leaves MMA1 of tile t about one
+// tile period ahead of the group that consumes it (that group is busy with
+// tile t - 2 until MMA2 of t - 2 can be issued).
+#ifndef SA_MMA1_LEAD
+#define SA_MMA1_LEAD 4
+#endif
+constexpr uint32_t kMma1Lead = SA_MMA1_LEAD;
+
+// Bounded wait until the counter `cnt` (a shared-memory word that only
+// grows) reaches `target`; same abort and timeout contract as mbar_wait.
+__device__ __forceinline__ bool wait_count(volatile uint32_t* cnt, uint32_t target,
+                                           volatile uint32_t* abort_flag, uint32_t* sticky_flag) {
+  if (*cnt >= target) return true;
+  const long long t0 = cycles_now();
+  while (*cnt < target) {
+    if (*abort_flag) return false;
+    if (cycles_now() - t0 > kWaitTimeoutCycles) {
+      *abort_flag = 1u;
+      atomicOr(sticky_flag, DEVFLAG_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
 // FULL: k == KM, so no prototype column needs masking.
 template <int D, int KM, bool FULL>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_sa_kernel(const __grid_constant__ CUtensorMap tm_x,
-                    const __grid_constant__ CUtensorMap tm_q, const PassArgs a) {
+                    const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_ox,
+                    const __grid_constant__ CUtensorMap tm_px, const PassArgs a) {
   using Pl = Plan<D, KM>;
   constexpr int S = Pl::S;
 
@@ -95,9 +125,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* q_full = acc_empty + 1;
   uint64_t* drain = q_full + 1;     // [issuer]: abort path, all of its MMAs done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  // [lane quarter]: the drain of segment s has finished reading its staging
+  // buffers (phase s), so the drain of segment s + 1 may refill them.
+  uint64_t* stage_free = drain + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stage_free + 4);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   int64_t* b0_slot = reinterpret_cast<int64_t*>(tmem_slot + 2);
+  volatile uint32_t* mma2_issued = tmem_slot + 4;  // tiles whose MMA2 has been issued
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -120,7 +154,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(acc_empty, 4);
     mbar_init(q_full, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&stage_free[i], 1);
     *abort_flag = 0u;
+    *mma2_issued = 0u;
     *b0_slot = (a.batch > 0 && R0 < R1) ? user_at_or_before(a.offsets, a.batch, R0) : a.batch;
     if (c == 0) { a.header->flags = 0u; a.header->timeout_flags = 0u; }
     fence_mbar_init();
@@ -201,7 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (role == 0) {
             // ---- MMA1: S^T_t = X_t Q'^T into the S^T buffer of tile t's group
             const int sb = t & 1;
-            if (!mbar_wait(&x_full[st], (t / S) & 1u, abort_flag, sticky) ||
+            if ((t >= kMma1Lead && !wait_count(mma2_issued, t + 1 - kMma1Lead, abort_flag, sticky)) ||
+                !mbar_wait(&x_full[st], (t / S) & 1u, abort_flag, sticky) ||
                 !mbar_wait(&s_empty[sb], ((t >> 1) & 1u) ^ 1u, abort_flag, sticky)) {
               ok = false;
               break;
@@ -240,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&x_empty[st]);
             mma_commit(&p_empty[t & 1u]);
             if (last) mma_commit(&acc_full[seg & 1u]);
+            *mma2_issued = t + 1;
           }
         }
         ++seg;
@@ -360,37 +398,86 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!warp_wait(&acc_full[seg & 1u], (seg >> 1) & 1u, abort_flag, sticky)) { ok = false; break; }
           tc_fence_after();
           const int64_t slotp = segment_slot(c, lo, hi, R0, R1);
-          float* dx = slotp < 0 ? a.out_x + user * k * D : a.part_x + slotp * k * D;
+          const CUtensorMap* tmo = slotp < 0 ? &tm_ox : &tm_px;
+          const int32_t zo = static_cast<int32_t>(slotp < 0 ? user : slotp);
           float* dm = slotp < 0 ? a.out_m + user * k : a.part_m + slotp * k;
           // M=128: prototype j sits in TMEM lane j.  M=64: prototypes
           // 16q..16q+15 sit in lanes 32q..32q+15.
-          const int j = (KM == 128) ? row : q * 16 + lane;
+          const int j0 = KM == 128 ? q * 32 : q * 16;
+          const int j = j0 + lane;
           const bool has = (KM == 128 ? true : lane < 16) && j < k;
+          if (seg > 0 && !warp_wait(&stage_free[q], (seg - 1) & 1u, abort_flag, sticky)) {
+            ok = false;
+            break;
+          }
+          // The accumulator is copied to registers in batches of up to 128
+          // columns; the last batch's loads release it (acc_empty), so the
+          // next segment's first MMA2 waits for TMEM reads only.  Each
+          // 16-column chunk is then staged in shared memory (one row per
+          // lane) and written by a TMA store: whole rows of X~ per request
+          // instead of one 16-byte piece of 32 different rows per warp
+          // store, which would hold up the other group's shared-memory
+          // stores behind it.  Rows >= k lie outside the map and are not
+          // written.
+          const uint32_t stage = sbase + Pl::kDrain + q * 2 * Pl::kDrainBuf;
+          constexpr int kDrainCols = D < 128 ? D : 128;
+          uint32_t mv = 0;
+          uint32_t chunk = 0;
 #pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(lane_addr + Pl::kColAcc + cc * 32, v);
-            tmem_wait_ld();
-            tmem_pin32(v);
-            if (has) {
-              float4* dst = reinterpret_cast<float4*>(dx + static_cast<int64_t>(j) * D + cc * 32);
+          for (int bt = 0; bt < D / kDrainCols; ++bt) {
+            const bool final_batch = bt == D / kDrainCols - 1;
+            uint32_t v[kDrainCols / 32][32];
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                     __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            for (int cc = 0; cc < kDrainCols / 32; ++cc)
+              tmem_ld32(lane_addr + Pl::kColAcc + bt * kDrainCols + cc * 32, v[cc]);
+            if (final_batch) tmem_ld1(lane_addr + Pl::kColAcc + D, mv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int cc = 0; cc < kDrainCols / 32; ++cc) tmem_pin32(v[cc]);
+            tmem_pin1(mv);
+            if (final_batch) {
+              tc_fence_before();
+              warp_arrive(acc_empty, lane);
+            }
+#pragma unroll
+            for (int h = 0; h < kDrainCols / 16; ++h, ++chunk) {
+              const uint32_t buf = stage + (chunk & 1u) * Pl::kDrainBuf;
+              if (chunk >= 2) {  // the store that read this buffer two chunks ago
+                if (lane == 0) bulk_wait_read<1>();
+                __syncwarp();
+              }
+              if (lane < Pl::kDrainRows) {
+                // 64-byte swizzle: 16-byte unit u of row r sits at unit
+                // u ^ ((r >> 1) & 3).
+                const uint32_t rowp = buf + lane * 64;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const int c0 = h * 16 + u * 4;
+                  st_shared_v4(rowp + ((u ^ ((lane >> 1) & 3)) << 4), v[c0 >> 5][c0 & 31],
+                               v[c0 >> 5][(c0 & 31) + 1], v[c0 >> 5][(c0 & 31) + 2],
+                               v[c0 >> 5][(c0 & 31) + 3]);
+                }
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(tmo, buf, bt * kDrainCols + h * 16, j0, zo);
+                bulk_commit();
+              }
             }
           }
-          uint32_t mv;
-          tmem_ld1(lane_addr + Pl::kColAcc + D, mv);
-          tmem_wait_ld();
-          tmem_pin1(mv);
+          if (lane == 0) {
+            bulk_wait_read<0>();
+            mbar_arrive(&stage_free[q]);
+          }
+          __syncwarp();
           if (has) dm[j] = __uint_as_float(mv);
-          tc_fence_before();
-          warp_arrive(acc_empty, lane);
         }
       }
       ++seg;
     }
+    // The X~ stores must be complete before the CTA exits.
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -402,13 +489,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D, int KM>
-cudaError_t launch_one(const CUtensorMap& tx, const CUtensorMap& tq, const PassArgs& a,
-                       int grid, cudaStream_t stream) {
+cudaError_t launch_one(const CUtensorMap& tx, const CUtensorMap& tq, const CUtensorMap& tox,
+                       const CUtensorMap& tpx, const PassArgs& a, int grid, cudaStream_t stream) {
   auto kern = a.k == KM ? fused_sa_kernel<D, KM, true> : fused_sa_kernel<D, KM, false>;
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Plan<D, KM>::kSmem);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kThreads, Plan<D, KM>::kSmem, stream>>>(tx, tq, a);
+  kern<<<grid, kThreads, Plan<D, KM>::kSmem, stream>>>(tx, tq, tox, tpx, a);
   return cudaGetLastError();
 }
 
@@ -420,13 +507,15 @@ bool fused_bf16_supported(int d, int k_pad) {
          (d == 256 && (k_pad == 64 || k_pad == 256));  // 256: the two-CTA pass
 }
 
-cudaError_t launch_fused_bf16(const CUtensorMap& tx, const CUtensorMap& tq, int k_pad,
+cudaError_t launch_fused_bf16(const CUtensorMap& tx, const CUtensorMap& tq,
+                              const CUtensorMap& tox, const CUtensorMap& tpx, int k_pad,
                               const PassArgs& a, int grid, cudaStream_t stream) {
-  if (a.d == 64 && k_pad == 64) return launch_one<64, 64>(tx, tq, a, grid, stream);
-  if (a.d == 64 && k_pad == 128) return launch_one<64, 128>(tx, tq, a, grid, stream);
-  if (a.d == 128 && k_pad == 64) return launch_one<128, 64>(tx, tq, a, grid, stream);
-  if (a.d == 128 && k_pad == 128) return launch_one<128, 128>(tx, tq, a, grid, stream);
-  if (a.d == 256 && k_pad == 64) return launch_one<256, 64>(tx, tq, a, grid, stream);
+  if (a.d == 64 && k_pad == 64) return launch_one<64, 64>(tx, tq, tox, tpx, a, grid, stream);
+  if (a.d == 64 && k_pad == 128) return launch_one<64, 128>(tx, tq, tox, tpx, a, grid, stream);
+  if (a.d == 128 && k_pad == 64) return launch_one<128, 64>(tx, tq, tox, tpx, a, grid, stream);
+  if (a.d == 128 && k_pad == 128)
+    return launch_one<128, 128>(tx, tq, tox, tpx, a, grid, stream);
+  if (a.d == 256 && k_pad == 64) return launch_one<256, 64>(tx, tq, tox, tpx, a, grid, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -135,9 +135,12 @@ cudaError_t launch_prepare_query(const void* P, const void* W_Q, const void* W_K
                                  int d, double scale, bool bf16_inputs, float* q_f32,
                                  uint16_t* q_bf16, cudaStream_t stream);
 
-// Tensor-core pass (bf16 X).  Returns cudaErrorInvalidValue for an
-// unsupported (d, k_pad) pair.
+// Tensor-core pass (bf16 X).  tmap_out / tmap_part are 3-D fp32 maps of
+// out_x [batch][k][d] and part_x [2G][k][d] with boxes of 16 columns x
+// (32 rows for k_pad = 128, 16 for k_pad = 64) x 1 and 64-byte swizzle.
+// Returns cudaErrorInvalidValue for an unsupported (d, k_pad) pair.
 cudaError_t launch_fused_bf16(const CUtensorMap& tmap_x, const CUtensorMap& tmap_q,
+                              const CUtensorMap& tmap_out, const CUtensorMap& tmap_part,
                               int k_pad, const PassArgs& a, int grid, cudaStream_t stream);
 bool fused_bf16_supported(int d, int k_pad);
 

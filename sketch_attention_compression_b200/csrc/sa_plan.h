@@ -37,7 +37,13 @@ struct Plan {
   static constexpr int kPStride = D == 128 ? 2 : 1;  // blocks between the 64-prototype chunks
   static constexpr int kPlanBlocks = D == 128 ? 13 : 12;
   static constexpr int kBars = kPlanBlocks * kPlanBlock;     // barriers and scheduler state after the blocks
-  static constexpr int kSmem = kBars + 512;
+  // Staging of the accumulator drain: each softmax lane quarter owns two
+  // buffers of kDrainRows rows x 16 fp32 columns (64-byte rows, 64-byte
+  // swizzle, so 512-byte aligned) that TMA stores read.
+  static constexpr int kDrainRows = KM == 128 ? 32 : 16;
+  static constexpr int kDrainBuf = 32 * 64;
+  static constexpr int kDrain = kBars + 512;
+  static constexpr int kSmem = kDrain + 4 * 2 * kDrainBuf;
   static_assert(kSmem <= kPlanMaxSmem, "shared memory budget");
   // TMEM columns: two S^T buffers (one per softmax group), then the
   // accumulator [X~ | m] with D + 16 columns; the masses are column D.
