@@ -117,11 +117,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* x_empty = bars + S;
   uint64_t* s_full = bars + 2 * S;  // [group]
   uint64_t* s_empty = s_full + 2;   // [group]
-  uint64_t* p_full = s_empty + 2;   // [group]: the group's probabilities are stored
-  uint64_t* p_empty = p_full + 2;   // [parity of the tile whose MMA2 freed the buffer]
+  // The probability buffer is handed over in four slices: slice q holds the
+  // tile rows 32q..32q+31 that softmax warp q computes, which are K-steps
+  // 2q and 2q+1 of MMA2.
+  uint64_t* p_full = s_empty + 2;   // [group][slice]: the warp's probabilities are stored
+  uint64_t* p_empty = p_full + 8;   // [tile parity][slice]: that tile's MMA2 has read the slice
   // Two acc_full barriers, used by segment parity, so that no wait can
   // confuse the phase of segment s with that of segment s - 2.
-  uint64_t* acc_full = p_empty + 2;
+  uint64_t* acc_full = p_empty + 8;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* q_full = acc_empty + 1;
   uint64_t* drain = q_full + 1;     // [issuer]: abort path, all of its MMAs done
@@ -147,8 +150,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 4);
-      mbar_init(&p_full[i], 4);
-      mbar_init(&p_empty[i], 1);
+      for (int sq = 0; sq < 4; ++sq) {
+        mbar_init(&p_full[i * 4 + sq], 1);
+        mbar_init(&p_empty[i * 4 + sq], 1);
+      }
       mbar_init(&acc_full[i], 1);
       mbar_init(&drain[i], 1);
     }
@@ -255,27 +260,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ---- MMA2: [X~ | m] += A_t [X_t | 1]  (a segment's first tile overwrites)
             const bool first = (r == s);
             const bool last = (r + kTileRows >= e);
-            if (!mbar_wait(&p_full[t & 1u], (t >> 1) & 1u, abort_flag, sticky) ||
-                (first && !mbar_wait(acc_empty, (seg & 1u) ^ 1u, abort_flag, sticky))) {
+            if (first && !mbar_wait(acc_empty, (seg & 1u) ^ 1u, abort_flag, sticky)) {
               ok = false;
               break;
             }
-            tc_fence_after();
             const uint32_t acc0 = first ? 0u : 1u;
             const uint64_t bd0 = smem_desc(sbase + Pl::b_start(st, 0) * kBlock,
                                            Pl::b_stride(st, 0) * kBlock, 1024, 2);
             const uint64_t bd1 = smem_desc(sbase + Pl::b_start(st, 1) * kBlock,
                                            Pl::b_stride(st, 1) * kBlock, 1024, 2);
+            // Slice by slice: K-steps 2q and 2q+1 as soon as warp q's rows
+            // are stored, then a commit that frees that slice for the next
+            // tile.
 #pragma unroll
-            for (int ks = 0; ks < kTileRows / 16; ++ks) {
-              mma_bf16_ss(tmem + Pl::kColAcc, p_desc + ((ks * 2048) >> 4), bd0 + ((ks * 2048) >> 4),
-                          idesc_x0, ks > 0 ? 1u : acc0);
-              if (Pl::kParts == 2)
-                mma_bf16_ss(tmem + Pl::kColAcc + 128, p_desc + ((ks * 2048) >> 4),
-                            bd1 + ((ks * 2048) >> 4), idesc_x1, ks > 0 ? 1u : acc0);
+            for (int sq = 0; sq < 4; ++sq) {
+              if (!mbar_wait(&p_full[(t & 1u) * 4 + sq], (t >> 1) & 1u, abort_flag, sticky)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < 2; ++kk) {
+                const int ks = 2 * sq + kk;
+                mma_bf16_ss(tmem + Pl::kColAcc, p_desc + ((ks * 2048) >> 4),
+                            bd0 + ((ks * 2048) >> 4), idesc_x0, ks > 0 ? 1u : acc0);
+                if (Pl::kParts == 2)
+                  mma_bf16_ss(tmem + Pl::kColAcc + 128, p_desc + ((ks * 2048) >> 4),
+                              bd1 + ((ks * 2048) >> 4), idesc_x1, ks > 0 ? 1u : acc0);
+              }
+              mma_commit(&p_empty[(t & 1u) * 4 + sq]);
             }
+            if (!ok) break;
             mma_commit(&x_empty[st]);
-            mma_commit(&p_empty[t & 1u]);
             if (last) mma_commit(&acc_full[seg & 1u]);
             *mma2_issued = t + 1;
           }
@@ -352,9 +368,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float inv = valid ? 1.0f / ((za + zb) + (zc + zd)) : 0.f;
         const uint64_t inv2 = f2_pack(inv, inv);
 
-        // The probability buffer is free once the previous tile's MMA2 (of
-        // the other group) has completed.
-        if (t > 0 && !warp_wait(&p_empty[(t - 1) & 1u], ((t - 1) >> 1) & 1u, abort_flag, sticky)) {
+        // This warp's slice of the probability buffer is free once the
+        // previous tile's MMA2 (of the other group) has read it.
+        if (t > 0 &&
+            !warp_wait(&p_empty[((t - 1) & 1u) * 4 + q], ((t - 1) >> 1) & 1u, abort_flag, sticky)) {
           ok = false;
           break;
         }
@@ -391,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         fence_proxy_async_smem();
-        warp_arrive(&p_full[grp], lane);
+        warp_arrive(&p_full[grp * 4 + q], lane);
 
         if (last) {
           // ---------------------------------------------- drain X~ and m

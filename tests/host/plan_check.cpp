@@ -37,11 +37,12 @@ static int check() {
   for (int s = 0; s < P::S; ++s)
     for (int b = 0; b < D / 64; ++b)
       bad |= take(P::box(s, b), "X" + std::to_string(s) + "." + std::to_string(b));
-  // Barrier area (x_full/x_empty per stage; s_full, s_empty, p_full,
-  // p_empty, acc_full, drain per group; acc_empty, q_full; stage_free per
-  // lane quarter) and the scheduler words must fit the 512 bytes before
-  // the drain staging, which the 64-byte swizzle wants 512-byte aligned.
-  const int bar_bytes = (2 * P::S + 6 * 2 + 2 + 4) * 8 + 4 * 4 + 8;
+  // Barrier area (x_full/x_empty per stage; s_full, s_empty, acc_full,
+  // drain per group; p_full, p_empty per group and slice; acc_empty,
+  // q_full; stage_free per lane quarter) and the scheduler words must fit
+  // the 512 bytes before the drain staging, which the 64-byte swizzle wants
+  // 512-byte aligned.
+  const int bar_bytes = (2 * P::S + 4 * 2 + 2 * 8 + 2 + 4) * 8 + 4 * 4 + 8;
   if (bar_bytes > P::kDrain - P::kBars || P::kDrain % 512 != 0 || P::kDrainBuf % 512 != 0 ||
       P::kDrainRows * 64 > P::kDrainBuf) {
     std::printf("FAIL D=%d KM=%d: barrier area or drain staging\n", D, KM);
