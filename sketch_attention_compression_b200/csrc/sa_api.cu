@@ -60,22 +60,6 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
   return r == CUDA_SUCCESS;
 }
 
-// 3-D fp32 map of a [n][k][d] sketch array, written by the fused pass's
-// drain in boxes of 16 columns x box_rows prototypes x 1 sketch.
-bool make_tmap_sketch(CUtensorMap* m, float* base, uint64_t d, uint64_t k, uint64_t n,
-                      uint32_t box_rows) {
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[3] = {d, k, n};
-  cuuint64_t strides[2] = {d * 4, k * d * 4};
-  cuuint32_t box[3] = {16, box_rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 constexpr int64_t kMaxRows = (int64_t{1} << 31) - 256;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -155,18 +139,8 @@ sa_status run(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
                           : make_tmap_bf16(&tmx, q->q_bf16, static_cast<uint64_t>(q->k_pad),
                                            static_cast<uint64_t>(q->d), 64);
       if (!ok) return SA_ERR_CUDA;
-      if (q->k_pad == 256) {
-        err = sa::launch_fused_bf16_pair(tmx, q->tmap_q_half, a, G, st);
-      } else {
-        CUtensorMap tmo, tmp;
-        const uint32_t box_rows = q->k_pad == 128 ? 32u : 16u;
-        if (!make_tmap_sketch(&tmo, X_tilde, static_cast<uint64_t>(q->d),
-                              static_cast<uint64_t>(q->k), static_cast<uint64_t>(batch), box_rows) ||
-            !make_tmap_sketch(&tmp, a.part_x, static_cast<uint64_t>(q->d),
-                              static_cast<uint64_t>(q->k), static_cast<uint64_t>(2 * G), box_rows))
-          return SA_ERR_CUDA;
-        err = sa::launch_fused_bf16(tmx, q->tmap_q, tmo, tmp, q->k_pad, a, G, st);
-      }
+      err = q->k_pad == 256 ? sa::launch_fused_bf16_pair(tmx, q->tmap_q_half, a, G, st)
+                            : sa::launch_fused_bf16(tmx, q->tmap_q, q->k_pad, a, G, st);
     } else {
       err = sa::launch_simt_fp32(q->q_f32, static_cast<const float*>(X), a, G, st);
     }

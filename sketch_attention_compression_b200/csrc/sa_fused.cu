@@ -78,6 +78,7 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar, int lane) {
 #endif
 constexpr uint32_t kMma1Lead = SA_MMA1_LEAD;
 
+
 // Bounded wait until the counter `cnt` (a shared-memory word that only
 // grows) reaches `target`; same abort and timeout contract as mbar_wait.
 __device__ __forceinline__ bool wait_count(volatile uint32_t* cnt, uint32_t target,
@@ -99,9 +100,7 @@ __device__ __forceinline__ bool wait_count(volatile uint32_t* cnt, uint32_t targ
 template <int D, int KM, bool FULL>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_sa_kernel(const __grid_constant__ CUtensorMap tm_x,
-                    const __grid_constant__ CUtensorMap tm_q,
-                    const __grid_constant__ CUtensorMap tm_ox,
-                    const __grid_constant__ CUtensorMap tm_px, const PassArgs a) {
+                    const __grid_constant__ CUtensorMap tm_q, const PassArgs a) {
   using Pl = Plan<D, KM>;
   constexpr int S = Pl::S;
 
@@ -145,26 +144,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t R1 = cta_row_begin(c + 1, G, a.tiles, N);
   uint32_t* sticky = &a.header->timeout_flags;
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
-      for (int sq = 0; sq < 4; ++sq) {
-        mbar_init(&p_full[i * 4 + sq], 1);
-        mbar_init(&p_empty[i * 4 + sq], 1);
+  int64_t* off_cache = reinterpret_cast<int64_t*>(smem + Pl::kOffs);
+  if (warp == 0) {
+    int64_t b0v = 0;
+    if (lane == 0) {
+      for (int i = 0; i < S; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&s_full[i], 1);
+        mbar_init(&s_empty[i], 4);
+        for (int sq = 0; sq < 4; ++sq) {
+          mbar_init(&p_full[i * 4 + sq], 1);
+          mbar_init(&p_empty[i * 4 + sq], 1);
+        }
+        mbar_init(&acc_full[i], 1);
+        mbar_init(&drain[i], 1);
       }
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&drain[i], 1);
+      mbar_init(acc_empty, 4);
+      mbar_init(q_full, 1);
+      for (int i = 0; i < 4; ++i) mbar_init(&stage_free[i], 1);
+      *abort_flag = 0u;
+      *mma2_issued = 0u;
+      b0v = (a.batch > 0 && R0 < R1) ? user_at_or_before(a.offsets, a.batch, R0) : a.batch;
+      *b0_slot = b0v;
+      if (c == 0) { a.header->flags = 0u; a.header->timeout_flags = 0u; }
+      fence_mbar_init();
     }
-    mbar_init(acc_empty, 4);
-    mbar_init(q_full, 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&stage_free[i], 1);
-    *abort_flag = 0u;
-    *mma2_issued = 0u;
-    *b0_slot = (a.batch > 0 && R0 < R1) ? user_at_or_before(a.offsets, a.batch, R0) : a.batch;
-    if (c == 0) { a.header->flags = 0u; a.header->timeout_flags = 0u; }
-    fence_mbar_init();
+    // Offsets from the CTA's first user on, in shared memory: every role
+    // walks them at each segment change, and a global load there (a
+    // round trip through a loaded memory system) would stall the role.
+    b0v = __shfl_sync(0xFFFFFFFFu, b0v, 0);
+    for (int i = lane; i < Pl::kOffCache && b0v + i <= a.batch; i += 32)
+      off_cache[i] = a.offsets[b0v + i];
   }
   {  // the block of bf16 ones read as MMA2's extra 16 columns
     const uint32_t ones = sbase + Pl::kOnes * kBlock;
@@ -181,6 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int64_t b0 = *b0_slot;
+  const int64_t n_cached =
+      (a.batch + 1 - b0) < Pl::kOffCache ? (a.batch + 1 - b0) : Pl::kOffCache;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -190,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int cb = 0; cb < D / 64; ++cb)
         tma_load_2d(q_s + cb * KM * 128, &tm_q, q_full, cb * 64, 0);
-      TileCursor cur{SegmentWalker{a.offsets, a.batch, R0, R1, b0}};
+      TileCursor cur{SegmentWalker{a.offsets, a.batch, R0, R1, b0, off_cache, b0, n_cached}};
       int64_t r;
       uint32_t t = 0;
       bool ok = true;
@@ -233,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_x0 = idesc_bf16_f32(KM, Pl::kPartN0, 1, 1);
       constexpr uint32_t idesc_x1 = idesc_bf16_f32(KM, 144, 1, 1);
       bool ok = role == 1 || mbar_wait(q_full, 0, abort_flag, sticky);
-      SegmentWalker w{a.offsets, a.batch, R0, R1, b0};
+      SegmentWalker w{a.offsets, a.batch, R0, R1, b0, off_cache, b0, n_cached};
       int64_t user, s, e, lo, hi;
       uint32_t t = 0, seg = 0;
       while (ok && w.next(user, s, e, lo, hi)) {
@@ -310,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = q * 32 + lane;         // tile row = TMEM lane of S^T
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int k = a.k;
-    SegmentWalker w{a.offsets, a.batch, R0, R1, b0};
+    SegmentWalker w{a.offsets, a.batch, R0, R1, b0, off_cache, b0, n_cached};
     int64_t user, s, e, lo, hi;
     uint32_t t = 0, seg = 0;
     bool ok = true;
@@ -415,9 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!warp_wait(&acc_full[seg & 1u], (seg >> 1) & 1u, abort_flag, sticky)) { ok = false; break; }
           tc_fence_after();
           const int64_t slotp = segment_slot(c, lo, hi, R0, R1);
-          const CUtensorMap* tmo = slotp < 0 ? &tm_ox : &tm_px;
-          const int32_t zo = static_cast<int32_t>(slotp < 0 ? user : slotp);
           float* dm = slotp < 0 ? a.out_m + user * k : a.part_m + slotp * k;
+          float* dxo = slotp < 0 ? a.out_x + user * k * D : a.part_x + slotp * k * D;
           // M=128: prototype j sits in TMEM lane j.  M=64: prototypes
           // 16q..16q+15 sit in lanes 32q..32q+15.
           const int j0 = KM == 128 ? q * 32 : q * 16;
@@ -430,13 +441,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           // The accumulator is copied to registers in batches of up to 128
           // columns; the last batch's loads release it (acc_empty), so the
           // next segment's first MMA2 waits for TMEM reads only.  Each
-          // 16-column chunk is then staged in shared memory (one row per
-          // lane) and written by a TMA store: whole rows of X~ per request
-          // instead of one 16-byte piece of 32 different rows per warp
-          // store, which would hold up the other group's shared-memory
-          // stores behind it.  Rows >= k lie outside the map and are not
-          // written.
-          const uint32_t stage = sbase + Pl::kDrain + q * 2 * Pl::kDrainBuf;
+          // 32-column chunk is then staged in shared memory (one row per
+          // lane) and read back so that every warp store writes four whole
+          // 128-byte rows of X~, instead of a 16-byte piece of 32 different
+          // rows, which would hold up the other group's shared-memory
+          // stores behind it.
+          const uint32_t stage = sbase + Pl::kDrain + q * Pl::kDrainBuf;
           constexpr int kDrainCols = D < 128 ? D : 128;
           uint32_t mv = 0;
           uint32_t chunk = 0;
@@ -456,45 +466,36 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_fence_before();
               warp_arrive(acc_empty, lane);
             }
+            // 32-column chunks: each lane stages its row (128 bytes, the
+            // 16-byte unit index XOR-ed with row mod 8), then the warp
+            // writes four whole rows per store.
 #pragma unroll
-            for (int h = 0; h < kDrainCols / 16; ++h, ++chunk) {
-              const uint32_t buf = stage + (chunk & 1u) * Pl::kDrainBuf;
-              if (chunk >= 2) {  // the store that read this buffer two chunks ago
-                if (lane == 0) bulk_wait_read<1>();
-                __syncwarp();
-              }
+            for (int cc = 0; cc < kDrainCols / 32; ++cc, ++chunk) {
+              if (chunk > 0) __syncwarp();  // the previous chunk's reads are done
               if (lane < Pl::kDrainRows) {
-                // 64-byte swizzle: 16-byte unit u of row r sits at unit
-                // u ^ ((r >> 1) & 3).
-                const uint32_t rowp = buf + lane * 64;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  const int c0 = h * 16 + u * 4;
-                  st_shared_v4(rowp + ((u ^ ((lane >> 1) & 3)) << 4), v[c0 >> 5][c0 & 31],
-                               v[c0 >> 5][(c0 & 31) + 1], v[c0 >> 5][(c0 & 31) + 2],
-                               v[c0 >> 5][(c0 & 31) + 3]);
-                }
+                for (int u = 0; u < 8; ++u)
+                  st_shared_v4(stage + lane * 128 + ((u ^ (lane & 7)) << 4), v[cc][4 * u],
+                               v[cc][4 * u + 1], v[cc][4 * u + 2], v[cc][4 * u + 3]);
               }
-              fence_proxy_async_smem();
               __syncwarp();
-              if (lane == 0) {
-                tma_store_3d(tmo, buf, bt * kDrainCols + h * 16, j0, zo);
-                bulk_commit();
+#pragma unroll
+              for (int i = 0; i < Pl::kDrainRows / 4; ++i) {
+                const int rr = 4 * i + (lane >> 3), uu = lane & 7;
+                const float4 w = ld_shared_v4f(stage + rr * 128 + ((uu ^ (rr & 7)) << 4));
+                if (j0 + rr < k)
+                  *reinterpret_cast<float4*>(dxo + static_cast<int64_t>(j0 + rr) * D +
+                                             bt * kDrainCols + cc * 32 + uu * 4) = w;
               }
             }
           }
-          if (lane == 0) {
-            bulk_wait_read<0>();
-            mbar_arrive(&stage_free[q]);
-          }
           __syncwarp();
+          if (lane == 0) mbar_arrive(&stage_free[q]);
           if (has) dm[j] = __uint_as_float(mv);
         }
       }
       ++seg;
     }
-    // The X~ stores must be complete before the CTA exits.
-    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -506,13 +507,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D, int KM>
-cudaError_t launch_one(const CUtensorMap& tx, const CUtensorMap& tq, const CUtensorMap& tox,
-                       const CUtensorMap& tpx, const PassArgs& a, int grid, cudaStream_t stream) {
+cudaError_t launch_one(const CUtensorMap& tx, const CUtensorMap& tq, const PassArgs& a,
+                       int grid, cudaStream_t stream) {
   auto kern = a.k == KM ? fused_sa_kernel<D, KM, true> : fused_sa_kernel<D, KM, false>;
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Plan<D, KM>::kSmem);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kThreads, Plan<D, KM>::kSmem, stream>>>(tx, tq, tox, tpx, a);
+  kern<<<grid, kThreads, Plan<D, KM>::kSmem, stream>>>(tx, tq, a);
   return cudaGetLastError();
 }
 
@@ -524,15 +525,13 @@ bool fused_bf16_supported(int d, int k_pad) {
          (d == 256 && (k_pad == 64 || k_pad == 256));  // 256: the two-CTA pass
 }
 
-cudaError_t launch_fused_bf16(const CUtensorMap& tx, const CUtensorMap& tq,
-                              const CUtensorMap& tox, const CUtensorMap& tpx, int k_pad,
+cudaError_t launch_fused_bf16(const CUtensorMap& tx, const CUtensorMap& tq, int k_pad,
                               const PassArgs& a, int grid, cudaStream_t stream) {
-  if (a.d == 64 && k_pad == 64) return launch_one<64, 64>(tx, tq, tox, tpx, a, grid, stream);
-  if (a.d == 64 && k_pad == 128) return launch_one<64, 128>(tx, tq, tox, tpx, a, grid, stream);
-  if (a.d == 128 && k_pad == 64) return launch_one<128, 64>(tx, tq, tox, tpx, a, grid, stream);
-  if (a.d == 128 && k_pad == 128)
-    return launch_one<128, 128>(tx, tq, tox, tpx, a, grid, stream);
-  if (a.d == 256 && k_pad == 64) return launch_one<256, 64>(tx, tq, tox, tpx, a, grid, stream);
+  if (a.d == 64 && k_pad == 64) return launch_one<64, 64>(tx, tq, a, grid, stream);
+  if (a.d == 64 && k_pad == 128) return launch_one<64, 128>(tx, tq, a, grid, stream);
+  if (a.d == 128 && k_pad == 64) return launch_one<128, 64>(tx, tq, a, grid, stream);
+  if (a.d == 128 && k_pad == 128) return launch_one<128, 128>(tx, tq, a, grid, stream);
+  if (a.d == 256 && k_pad == 64) return launch_one<256, 64>(tx, tq, a, grid, stream);
   return cudaErrorInvalidValue;
 }
 

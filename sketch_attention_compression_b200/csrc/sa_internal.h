@@ -70,9 +70,17 @@ SA_HD int64_t user_at_or_before(const int64_t* off, int64_t B, int64_t r) {
 struct SegmentWalker {
   const int64_t* off;
   int64_t B, R0, R1, b;
+  // Optional copy of off[cb0, cb0 + ncache) (the fused pass keeps one in
+  // shared memory); other entries are read from `off`.
+  const int64_t* cache = nullptr;
+  int64_t cb0 = 0, ncache = 0;
+  SA_HD int64_t at(int64_t i) const {
+    const int64_t ci = i - cb0;
+    return (cache != nullptr && ci >= 0 && ci < ncache) ? cache[ci] : off[i];
+  }
   SA_HD bool next(int64_t& user, int64_t& s, int64_t& e, int64_t& lo, int64_t& hi) {
     while (b < B) {
-      const int64_t l = off[b], h = off[b + 1];
+      const int64_t l = at(b), h = at(b + 1);
       if (l >= R1) { b = B; return false; }
       const int64_t cur = b++;
       const int64_t ss = l > R0 ? l : R0;
@@ -135,12 +143,9 @@ cudaError_t launch_prepare_query(const void* P, const void* W_Q, const void* W_K
                                  int d, double scale, bool bf16_inputs, float* q_f32,
                                  uint16_t* q_bf16, cudaStream_t stream);
 
-// Tensor-core pass (bf16 X).  tmap_out / tmap_part are 3-D fp32 maps of
-// out_x [batch][k][d] and part_x [2G][k][d] with boxes of 16 columns x
-// (32 rows for k_pad = 128, 16 for k_pad = 64) x 1 and 64-byte swizzle.
-// Returns cudaErrorInvalidValue for an unsupported (d, k_pad) pair.
+// Tensor-core pass (bf16 X).  Returns cudaErrorInvalidValue for an
+// unsupported (d, k_pad) pair.
 cudaError_t launch_fused_bf16(const CUtensorMap& tmap_x, const CUtensorMap& tmap_q,
-                              const CUtensorMap& tmap_out, const CUtensorMap& tmap_part,
                               int k_pad, const PassArgs& a, int grid, cudaStream_t stream);
 bool fused_bf16_supported(int d, int k_pad);
 

@@ -37,13 +37,16 @@ struct Plan {
   static constexpr int kPStride = D == 128 ? 2 : 1;  // blocks between the 64-prototype chunks
   static constexpr int kPlanBlocks = D == 128 ? 13 : 12;
   static constexpr int kBars = kPlanBlocks * kPlanBlock;     // barriers and scheduler state after the blocks
-  // Staging of the accumulator drain: each softmax lane quarter owns two
-  // buffers of kDrainRows rows x 16 fp32 columns (64-byte rows, 64-byte
-  // swizzle, so 512-byte aligned) that TMA stores read.
+  // Staging of the accumulator drain: each softmax lane quarter owns
+  // kDrainRows rows x 32 fp32 columns (128-byte rows, the 16-byte unit
+  // index XOR-ed with the row mod 8).
   static constexpr int kDrainRows = KM == 128 ? 32 : 16;
-  static constexpr int kDrainBuf = 32 * 64;
+  static constexpr int kDrainBuf = 32 * 128;
   static constexpr int kDrain = kBars + 512;
-  static constexpr int kSmem = kDrain + 4 * 2 * kDrainBuf;
+  // Copy of the offsets from the CTA's first user on (kOffCache entries).
+  static constexpr int kOffCache = 64;
+  static constexpr int kOffs = kDrain + 4 * kDrainBuf;
+  static constexpr int kSmem = kOffs + kOffCache * 8;
   static_assert(kSmem <= kPlanMaxSmem, "shared memory budget");
   // TMEM columns: two S^T buffers (one per softmax group), then the
   // accumulator [X~ | m] with D + 16 columns; the masses are column D.

@@ -40,11 +40,10 @@ static int check() {
   // Barrier area (x_full/x_empty per stage; s_full, s_empty, acc_full,
   // drain per group; p_full, p_empty per group and slice; acc_empty,
   // q_full; stage_free per lane quarter) and the scheduler words must fit
-  // the 512 bytes before the drain staging, which the 64-byte swizzle wants
-  // 512-byte aligned.
+  // the 512 bytes before the drain staging (128-byte rows).
   const int bar_bytes = (2 * P::S + 4 * 2 + 2 * 8 + 2 + 4) * 8 + 4 * 4 + 8;
-  if (bar_bytes > P::kDrain - P::kBars || P::kDrain % 512 != 0 || P::kDrainBuf % 512 != 0 ||
-      P::kDrainRows * 64 > P::kDrainBuf) {
+  if (bar_bytes > P::kDrain - P::kBars || P::kDrain % 128 != 0 ||
+      P::kDrainRows * 128 > P::kDrainBuf) {
     std::printf("FAIL D=%d KM=%d: barrier area or drain staging\n", D, KM);
     bad = 1;
   }
