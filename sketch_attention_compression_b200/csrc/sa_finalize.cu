@@ -29,6 +29,7 @@ constexpr int kValidateBlocks = 32;
 __global__ void __launch_bounds__(kFinThreads)
     finalize_kernel(const PassArgs a, int64_t G, int chunks, int64_t reduce_blocks) {
   grid_dependency_wait();
+  grid_dependency_launch();  // the next call's fused pass may start its local set-up
   const int64_t N = a.total_rows, T = a.tiles, B = a.batch;
   const int k = a.k, d = a.d;
   const int64_t kd = static_cast<int64_t>(k) * d;

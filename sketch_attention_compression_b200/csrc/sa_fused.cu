@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0u) {  // the 128-byte swizzle needs 1024-byte alignment
+    grid_dependency_wait();
     if (threadIdx.x == 0) atomicOr(&a.header->timeout_flags, DEVFLAG_SMEM_ALIGN);
     return;
   }
@@ -145,36 +146,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* sticky = &a.header->timeout_flags;
 
   int64_t* off_cache = reinterpret_cast<int64_t*>(smem + Pl::kOffs);
-  if (warp == 0) {
-    int64_t b0v = 0;
-    if (lane == 0) {
-      for (int i = 0; i < S; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(&s_full[i], 1);
-        mbar_init(&s_empty[i], 4);
-        for (int sq = 0; sq < 4; ++sq) {
-          mbar_init(&p_full[i * 4 + sq], 1);
-          mbar_init(&p_empty[i * 4 + sq], 1);
-        }
-        mbar_init(&acc_full[i], 1);
-        mbar_init(&drain[i], 1);
+  // Set-up in two parts.  The launch may overlap the end of the preceding
+  // kernel in the stream (programmatic dependent launch), so the first part
+  // touches shared and tensor memory only; grid_dependency_wait then makes
+  // everything that kernel wrote visible before any global access.
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);
+      for (int sq = 0; sq < 4; ++sq) {
+        mbar_init(&p_full[i * 4 + sq], 1);
+        mbar_init(&p_empty[i * 4 + sq], 1);
       }
-      mbar_init(acc_empty, 4);
-      mbar_init(q_full, 1);
-      for (int i = 0; i < 4; ++i) mbar_init(&stage_free[i], 1);
-      *abort_flag = 0u;
-      *mma2_issued = 0u;
-      b0v = (a.batch > 0 && R0 < R1) ? user_at_or_before(a.offsets, a.batch, R0) : a.batch;
-      *b0_slot = b0v;
-      if (c == 0) { a.header->flags = 0u; a.header->timeout_flags = 0u; }
-      fence_mbar_init();
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&drain[i], 1);
     }
-    // Offsets from the CTA's first user on, in shared memory: every role
-    // walks them at each segment change, and a global load there (a
-    // round trip through a loaded memory system) would stall the role.
-    b0v = __shfl_sync(0xFFFFFFFFu, b0v, 0);
-    for (int i = lane; i < Pl::kOffCache && b0v + i <= a.batch; i += 32)
-      off_cache[i] = a.offsets[b0v + i];
+    mbar_init(acc_empty, 4);
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&stage_free[i], 1);
+    *abort_flag = 0u;
+    *mma2_issued = 0u;
+    fence_mbar_init();
   }
   {  // the block of bf16 ones read as MMA2's extra 16 columns
     const uint32_t ones = sbase + Pl::kOnes * kBlock;
@@ -185,6 +178,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 2) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
+  }
+  grid_dependency_wait();
+  if (warp == 0) {
+    int64_t b0v = 0;
+    if (lane == 0) {
+      b0v = (a.batch > 0 && R0 < R1) ? user_at_or_before(a.offsets, a.batch, R0) : a.batch;
+      *b0_slot = b0v;
+      if (c == 0) { a.header->flags = 0u; a.header->timeout_flags = 0u; }
+    }
+    // Offsets from the CTA's first user on, in shared memory: every role
+    // walks them at each segment change, and a global load there (a
+    // round trip through a loaded memory system) would stall the role.
+    b0v = __shfl_sync(0xFFFFFFFFu, b0v, 0);
+    for (int i = lane; i < Pl::kOffCache && b0v + i <= a.batch; i += 32)
+      off_cache[i] = a.offsets[b0v + i];
   }
   tc_fence_before();
   __syncthreads();
@@ -513,8 +521,17 @@ cudaError_t launch_one(const CUtensorMap& tx, const CUtensorMap& tq, const PassA
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Plan<D, KM>::kSmem);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kThreads, Plan<D, KM>::kSmem, stream>>>(tx, tq, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Plan<D, KM>::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tx, tq, a);
 }
 
 }  // namespace

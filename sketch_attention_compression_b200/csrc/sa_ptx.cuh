@@ -435,4 +435,12 @@ __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// Programmatic dependent launch: the next grid in the stream (launched with
+// programmatic stream serialization) may be scheduled once every CTA of
+// this grid has issued this or exited; it still waits in
+// grid_dependency_wait before touching what this grid writes.
+__device__ __forceinline__ void grid_dependency_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace sa
