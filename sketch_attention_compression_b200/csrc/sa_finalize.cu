@@ -30,31 +30,32 @@ __global__ void __launch_bounds__(kFinThreads)
     finalize_kernel(const PassArgs a, int64_t G, int chunks, int64_t reduce_blocks) {
   grid_dependency_wait();
   grid_dependency_launch();  // the next call's fused pass may start its local set-up
-  const int64_t N = a.total_rows, T = a.tiles, B = a.batch;
+  const int64_t N = a.total_rows, B = a.batch;
   const int k = a.k, d = a.d;
   const int64_t kd = static_cast<int64_t>(k) * d;
 
   if (static_cast<int64_t>(blockIdx.x) < reduce_blocks) {
     const int64_t cb = blockIdx.x / chunks + 1;  // boundary between CTAs cb-1 and cb
     const int ch = blockIdx.x % chunks;
-    const int64_t Rc = cta_row_begin(cb, G, T, N);
-    const int64_t Rp = cta_row_begin(cb - 1, G, T, N);
-    // The user whose rows contain Rc: with valid offsets only one non-empty
-    // user does, so one parallel pass over the offsets finds it (a binary
-    // search would chain its loads end to end).  With invalid offsets any
-    // match is taken; the outputs are then unspecified but stay in bounds.
-    __shared__ long long s_user;
-    if (threadIdx.x == 0) s_user = -1;
+    // The two range starts, and the user found for R_cb: if it starts
+    // before R_cb, it is the user whose rows contain R_cb.
+    __shared__ long long s_rc, s_rp, s_user;
+    if (threadIdx.x < 32) {
+      int64_t bc, bp;
+      const int64_t rc = warp_range_begin(a.offsets, B, N, cb, G, threadIdx.x, &bc);
+      const int64_t rp = warp_range_begin(a.offsets, B, N, cb - 1, G, threadIdx.x, &bp);
+      if (threadIdx.x == 0) {
+        s_rc = rc;
+        s_rp = rp;
+        s_user = bc;
+      }
+    }
     __syncthreads();
-    for (int64_t i = threadIdx.x; i < B; i += kFinThreads)
-      if (a.offsets[i] <= Rc && Rc < a.offsets[i + 1]) s_user = i;
-    __syncthreads();
-    if (s_user < 0) return;
-    const int64_t b = s_user;
+    const int64_t Rc = s_rc, Rp = s_rp, b = s_user;
+    if (b >= B) return;
     const int64_t lo = a.offsets[b], hi = a.offsets[b + 1];
     if (!(lo < Rc && lo >= Rp && hi > Rc)) return;  // not split here, or owned elsewhere
-    int64_t c_hi = cta_of_row(hi - 1 < N - 1 ? hi - 1 : N - 1, G, T);
-    if (c_hi > G - 1) c_hi = G - 1;
+    const int64_t c_hi = cta_of_row(a.offsets, b, B, N, G, hi - 1 < N - 1 ? hi - 1 : N - 1);
     const int64_t c_lo = cb - 1;
     const int64_t slot_lo = 2 * c_lo + (lo <= Rp ? 0 : 1);
 

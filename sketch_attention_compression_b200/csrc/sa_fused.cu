@@ -135,14 +135,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* abort_flag = tmem_slot + 1;
   int64_t* b0_slot = reinterpret_cast<int64_t*>(tmem_slot + 2);
   volatile uint32_t* mma2_issued = tmem_slot + 4;  // tiles whose MMA2 has been issued
+  int64_t* range_slot = reinterpret_cast<int64_t*>(tmem_slot + 6);  // R0, R1
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t G = gridDim.x;
   const int64_t c = blockIdx.x;
   const int64_t N = a.total_rows;
-  const int64_t R0 = cta_row_begin(c, G, a.tiles, N);
-  const int64_t R1 = cta_row_begin(c + 1, G, a.tiles, N);
   uint32_t* sticky = &a.header->timeout_flags;
 
   int64_t* off_cache = reinterpret_cast<int64_t*>(smem + Pl::kOffs);
@@ -181,16 +180,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   grid_dependency_wait();
   if (warp == 0) {
-    int64_t b0v = 0;
+    // This CTA's row range and its first user (the work split of
+    // sa_internal.h, searched by the whole warp).
+    int64_t b0v, b1v;
+    const int64_t r0 = warp_range_begin(a.offsets, a.batch, N, c, G, lane, &b0v);
+    const int64_t r1 = warp_range_begin(a.offsets, a.batch, N, c + 1, G, lane, &b1v);
+    if (!(r0 < r1)) b0v = a.batch;
     if (lane == 0) {
-      b0v = (a.batch > 0 && R0 < R1) ? user_at_or_before(a.offsets, a.batch, R0) : a.batch;
+      range_slot[0] = r0;
+      range_slot[1] = r1;
       *b0_slot = b0v;
       if (c == 0) { a.header->flags = 0u; a.header->timeout_flags = 0u; }
     }
     // Offsets from the CTA's first user on, in shared memory: every role
     // walks them at each segment change, and a global load there (a
     // round trip through a loaded memory system) would stall the role.
-    b0v = __shfl_sync(0xFFFFFFFFu, b0v, 0);
     for (int i = lane; i < Pl::kOffCache && b0v + i <= a.batch; i += 32)
       off_cache[i] = a.offsets[b0v + i];
   }
@@ -199,6 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int64_t b0 = *b0_slot;
+  const int64_t R0 = range_slot[0], R1 = range_slot[1];
   const int64_t n_cached =
       (a.batch + 1 - b0) < Pl::kOffCache ? (a.batch + 1 - b0) : Pl::kOffCache;
 

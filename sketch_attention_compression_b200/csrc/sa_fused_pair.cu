@@ -89,14 +89,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xslot + 256);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   int64_t* b0_slot = reinterpret_cast<int64_t*>(tmem_slot + 2);
+  int64_t* range_slot = reinterpret_cast<int64_t*>(tmem_slot + 4);  // R0, R1
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t G = gridDim.x / 2;             // row ranges (one per cluster)
   const int64_t c = blockIdx.x / 2;
   const int64_t N = a.total_rows;
-  const int64_t R0 = cta_row_begin(c, G, a.tiles, N);
-  const int64_t R1 = cta_row_begin(c + 1, G, a.tiles, N);
   uint32_t* sticky = &a.header->timeout_flags;
 
   if (aligned && threadIdx.x == 0) {
@@ -115,7 +114,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     mbar_init(acc_empty, 4);
     mbar_init(q_full, 1);
     *abort_flag = 0u;
-    *b0_slot = (a.batch > 0 && R0 < R1) ? user_at_or_before(a.offsets, a.batch, R0) : a.batch;
+    int64_t b0u;
+    const int64_t r0 = range_begin(a.offsets, a.batch, N, c, G, &b0u);
+    const int64_t r1 = range_begin(a.offsets, a.batch, N, c + 1, G);
+    range_slot[0] = r0;
+    range_slot[1] = r1;
+    *b0_slot = r0 < r1 ? b0u : a.batch;
     if (c == 0 && h == 0) { a.header->flags = 0u; a.header->timeout_flags = 0u; }
     fence_mbar_init();
   }
@@ -140,6 +144,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   if (aligned) {
     const uint32_t tmem = *tmem_slot;
     const int64_t b0 = *b0_slot;
+    const int64_t R0 = range_slot[0], R1 = range_slot[1];
     if (warp == 0) {
       // ---------------------------------------------------------- producer
       if (lane == 0) {

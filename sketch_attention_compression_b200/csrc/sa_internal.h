@@ -1,11 +1,15 @@
 // Internal declarations shared by the kernels and the C-ABI layer.
 //
 // Work split (all kernels of one call agree on it):
-//   The N concatenated history rows are cut into T = ceil(N / 128) row tiles.
-//   CTA c of a G-CTA grid (G <= T) owns rows [R_c, R_{c+1}) with
-//   R_c = floor(c * T / G) * 128 (clipped to N), so every CTA has at least
-//   one tile and the ranges are contiguous.  Inside its range a CTA walks
-//   the users in order; user b's part of the range is one "segment".
+//   Splitting the N concatenated history rows over the G CTAs of a pass
+//   charges each row 1 and each user start kUserStartCost rows: a user that
+//   ends inside a CTA's range costs that range the drain of its sketch and
+//   a part-filled last tile.  CTA c owns rows [R_c, R_{c+1}), where R_c is
+//   the row at which the cost reaches c/G of the total C = N +
+//   kUserStartCost * B, moved back to the user's first row or to a whole
+//   number of 128-row tiles into the user, so every user's tiles are
+//   aligned to its own first row.  Inside its range a CTA walks the users
+//   in order; user b's part of the range is one "segment".
 //   * A user that lies wholly inside one CTA's range is written straight to
 //     the outputs by that CTA.
 //   * A user that crosses a CTA boundary is "split".  Each CTA writes its
@@ -43,16 +47,60 @@ constexpr size_t kWsHeaderBytes = 256;
 
 SA_HD int64_t tiles_of(int64_t rows) { return (rows + kTileRows - 1) / kTileRows; }
 
-// First row of CTA c (c in [0, G]); R_G == N.
-SA_HD int64_t cta_row_begin(int64_t c, int64_t G, int64_t T, int64_t N) {
-  int64_t r = ((c * T) / G) * kTileRows;
-  return r < N ? r : N;
+// Cost, in rows, charged to each user start by the work split.
+constexpr int64_t kUserStartCost = 640;
+
+// Cost of everything before user b's first row.
+SA_HD int64_t cost_before_user(const int64_t* off, int64_t b) { return off[b] + kUserStartCost * b; }
+
+// Cost position at which CTA range c starts (0 < c < G).
+SA_HD int64_t range_target(int64_t B, int64_t N, int64_t c, int64_t G) {
+  return (c * (N + kUserStartCost * B)) / G;
 }
 
-// The CTA whose range holds row r (0 <= r < N); requires G <= T.
-SA_HD int64_t cta_of_row(int64_t r, int64_t G, int64_t T) {
-  int64_t u = r / kTileRows;
-  return ((u + 1) * G - 1) / T;
+// First row of CTA range c, given user b with cost_before_user(b) <= tau <
+// cost_before_user(b + 1) for tau = range_target(c): the user's first row,
+// or a whole number of tiles into it.  Clipped to [0, N] and to the user's
+// rows (which only matters for invalid offsets).
+SA_HD int64_t range_row(const int64_t* off, int64_t b, int64_t N, int64_t tau) {
+  const int64_t into = tau - cost_before_user(off, b) - kUserStartCost;
+  int64_t r = off[b] + (into > 0 ? (into / kTileRows) * kTileRows : 0);
+  if (r > off[b + 1]) r = off[b + 1];
+  if (r > N) r = N;
+  return r < 0 ? 0 : r;
+}
+
+// First row of CTA range c (c in [0, G]; R_0 = 0, R_G = N).  *user, if
+// given, receives the user found for it (range_row's b).  Serial binary
+// search; the fused pass uses a warp-wide search with the same result.
+SA_HD int64_t range_begin(const int64_t* off, int64_t B, int64_t N, int64_t c, int64_t G,
+                          int64_t* user = nullptr) {
+  if (c <= 0 || B <= 0 || c >= G) {
+    if (user) *user = c <= 0 || B <= 0 ? 0 : B;
+    return c <= 0 ? 0 : N;
+  }
+  const int64_t tau = range_target(B, N, c, G);
+  int64_t lo = 0, hi = B - 1;  // largest b in [0, B) with cost_before_user(b) <= tau
+  while (lo < hi) {
+    const int64_t mid = (lo + hi + 1) >> 1;
+    if (cost_before_user(off, mid) <= tau) lo = mid; else hi = mid - 1;
+  }
+  if (user) *user = lo;
+  return range_row(off, lo, N, tau);
+}
+
+// The CTA range that holds row r of user b (off[b] <= r < off[b + 1]): the
+// largest c with R_c <= r, from b's offsets alone.
+SA_HD int64_t cta_of_row(const int64_t* off, int64_t b, int64_t B, int64_t N, int64_t G,
+                         int64_t r) {
+  const int64_t C = N + kUserStartCost * B;
+  int64_t X = cost_before_user(off, b) + kUserStartCost +
+              kTileRows * ((r - off[b]) / kTileRows + 1);
+  const int64_t next = cost_before_user(off, b + 1);
+  if (X > next) X = next;
+  int64_t c = (X * G + C - 1) / C - 1;  // largest c with floor(c C / G) < X
+  if (c < 0) c = 0;
+  return c > G - 1 ? G - 1 : c;
 }
 
 // Largest b in [0, B) with off[b] <= r (off[0] <= r assumed; with invalid

@@ -429,6 +429,33 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// range_begin (sa_internal.h) computed by a whole warp: every lane passes
+// the same arguments and gets the same row and user.  A 32-way search over
+// the users, one round of loads per factor of 32 in the batch size; for
+// valid offsets the cost of the users' starts is strictly increasing, so
+// the result equals the serial binary search's.
+__device__ __forceinline__ int64_t warp_range_begin(const int64_t* off, int64_t B, int64_t N,
+                                                    int64_t c, int64_t G, int lane,
+                                                    int64_t* user) {
+  if (c <= 0 || B <= 0 || c >= G) {
+    *user = (c <= 0 || B <= 0) ? 0 : B;
+    return c <= 0 ? 0 : N;
+  }
+  const int64_t tau = range_target(B, N, c, G);
+  int64_t lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int64_t step = (hi - lo + 32) / 32;
+    const int64_t b = lo + lane * step;
+    const bool pred = b <= hi && cost_before_user(off, b) <= tau;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, pred);
+    const int64_t nlo = lo + (m ? 31 - __clz(static_cast<int>(m)) : 0) * step;
+    hi = (nlo + step - 1) < hi ? (nlo + step - 1) : hi;
+    lo = nlo;
+  }
+  *user = lo;
+  return range_row(off, lo, N, tau);
+}
+
 // Programmatic dependent launch: block until the preceding grid in the
 // stream has completed and its memory operations are visible.
 __device__ __forceinline__ void grid_dependency_wait() {

@@ -1,9 +1,13 @@
 // Host-side check of the row-range schedule in sa_internal.h (the code the
-// kernels run), on random ragged batches: every row of every user is
-// covered by exactly one segment; users inside one CTA range go straight to
-// the outputs; split users use distinct partial slots below 2G; the
-// finalize pass reduces every split user exactly once, over exactly the
-// slots that the partial pass wrote for it, in ascending CTA order.
+// kernels run), on random ragged batches: the ranges are ordered and start
+// at a user's first row or a whole number of tiles into the user; every row
+// of every user is covered by exactly one segment; cta_of_row names the CTA
+// that covered each row; users inside one CTA range go straight to the
+// outputs; split users use distinct partial slots below 2G; the finalize
+// pass reduces every split user exactly once, over exactly the slots that
+// the partial pass wrote for it, in ascending CTA order.  The 32-way search
+// the kernels use (warp_range_begin) is replayed here step by step and must
+// agree with the serial search.
 #include <cstdio>
 #include <cstdlib>
 #include <map>
@@ -20,27 +24,63 @@ static int fail(const char* what, long long a, long long b) {
   return 1;
 }
 
+// Host replay of warp_range_begin (sa_ptx.cuh): 32 lanes test evenly
+// spaced users, the highest lane whose user's start cost is <= tau narrows
+// the range, until one user is left.
+static int64_t warp_search_replay(const int64_t* off, int64_t B, int64_t N, int64_t c, int64_t G,
+                                  int64_t* user) {
+  if (c <= 0 || B <= 0 || c >= G) {
+    *user = (c <= 0 || B <= 0) ? 0 : B;
+    return c <= 0 ? 0 : N;
+  }
+  const int64_t tau = range_target(B, N, c, G);
+  int64_t lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int64_t step = (hi - lo + 32) / 32;
+    int last = -1;
+    for (int lane = 0; lane < 32; ++lane) {
+      const int64_t b = lo + lane * step;
+      if (b <= hi && cost_before_user(off, b) <= tau) last = lane;
+    }
+    const int64_t nlo = lo + (last < 0 ? 0 : last) * step;
+    hi = (nlo + step - 1) < hi ? (nlo + step - 1) : hi;
+    lo = nlo;
+  }
+  *user = lo;
+  return range_row(off, lo, N, tau);
+}
+
 static int check(const std::vector<int64_t>& off, int64_t sms) {
   const int64_t B = static_cast<int64_t>(off.size()) - 1, N = off.back();
   const int64_t T = tiles_of(N);
   int64_t G = T < sms ? T : sms;
   if (G < 1) G = 1;
   std::vector<int> covered(N, 0);
+  std::vector<int64_t> owner(N, -1);
   std::map<int64_t, std::set<int64_t>> written;  // user -> slots
   std::map<int64_t, int64_t> slot_owner;          // slot -> user
   std::vector<int> direct(B, 0);
   for (int64_t c = 0; c < G; ++c) {
-    const int64_t R0 = cta_row_begin(c, G, T, N), R1 = cta_row_begin(c + 1, G, T, N);
-    if (N > 0 && R0 >= R1) return fail("empty CTA range", c, R0);
-    if (R0 % kTileRows) return fail("unaligned range", c, R0);
-    if (R0 < R1 && cta_of_row(R0, G, T) != c) return fail("cta_of_row(R0)", c, R0);
-    if (R0 < R1 && cta_of_row(R1 - 1, G, T) != c) return fail("cta_of_row(R1-1)", c, R1);
-    const int64_t b0 = (B > 0 && R0 < R1) ? user_at_or_before(off.data(), B, R0) : B;
+    int64_t bu, bw, bu1;
+    const int64_t R0 = range_begin(off.data(), B, N, c, G, &bu);
+    const int64_t R1 = range_begin(off.data(), B, N, c + 1, G, &bu1);
+    if (warp_search_replay(off.data(), B, N, c, G, &bw) != R0 || bw != bu)
+      return fail("warp search != serial search", c, R0);
+    if (R0 > R1) return fail("ranges out of order", c, R0);
+    if (R0 < R1 && B > 0) {
+      const int64_t u = user_at_or_before(off.data(), B, R0);
+      if (off[u] < R0 && (R0 - off[u]) % kTileRows) return fail("range not tile-aligned in its user", c, R0);
+      if (off[bu] > R0) return fail("walker start after R0", c, bu);
+    }
+    const int64_t b0 = (B > 0 && R0 < R1) ? bu : B;
     SegmentWalker w{off.data(), B, R0, R1, b0};
     int64_t u, s, e, lo, hi;
     while (w.next(u, s, e, lo, hi)) {
       if (s < R0 || e > R1 || s < lo || e > hi) return fail("segment bounds", s, e);
-      for (int64_t r = s; r < e; ++r) covered[r]++;
+      for (int64_t r = s; r < e; ++r) {
+        covered[r]++;
+        owner[r] = c;
+      }
       const int64_t slot = segment_slot(c, lo, hi, R0, R1);
       if (slot < 0) {
         direct[u]++;
@@ -54,16 +94,23 @@ static int check(const std::vector<int64_t>& off, int64_t sms) {
   }
   for (int64_t r = 0; r < N; ++r)
     if (covered[r] != 1) return fail("row coverage", r, covered[r]);
+  // cta_of_row against the owner of every row (a sample of rows for big N)
+  const int64_t stride = N > 200000 ? 97 : 1;
+  for (int64_t r = 0, u = 0; r < N; r += stride) {
+    while (off[u + 1] <= r) ++u;
+    if (cta_of_row(off.data(), u, B, N, G, r) != owner[r]) return fail("cta_of_row", r, owner[r]);
+  }
   // finalize ownership, same arithmetic as finalize_kernel
   std::map<int64_t, std::vector<int64_t>> reduced;
   for (int64_t cb = 1; cb < G; ++cb) {
-    const int64_t Rc = cta_row_begin(cb, G, T, N), Rp = cta_row_begin(cb - 1, G, T, N);
-    const int64_t b = user_at_or_before(off.data(), B, Rc);
+    int64_t b, bp;
+    const int64_t Rc = range_begin(off.data(), B, N, cb, G, &b);
+    const int64_t Rp = range_begin(off.data(), B, N, cb - 1, G, &bp);
+    if (b >= B) continue;
     const int64_t lo = off[b], hi = off[b + 1];
     if (!(lo < Rc && lo >= Rp && hi > Rc)) continue;
     if (reduced.count(b)) return fail("user reduced twice", b, cb);
-    int64_t c_hi = cta_of_row(hi - 1 < N - 1 ? hi - 1 : N - 1, G, T);
-    if (c_hi > G - 1) c_hi = G - 1;
+    const int64_t c_hi = cta_of_row(off.data(), b, B, N, G, hi - 1 < N - 1 ? hi - 1 : N - 1);
     std::vector<int64_t> slots{2 * (cb - 1) + (lo <= Rp ? 0 : 1)};
     for (int64_t cc = cb; cc <= c_hi; ++cc) slots.push_back(2 * cc);
     reduced[b] = slots;
@@ -108,6 +155,17 @@ int main() {
     }
     if (check(off, sms)) {
       std::printf("case iter=%d B=%d N=%lld sms=%lld\n", iter, B, (long long)off.back(), (long long)sms);
+      return 1;
+    }
+    ++cases;
+  }
+  // large batches: several rounds of the 32-way search
+  for (int iter = 0; iter < 40; ++iter) {
+    const int B = 1000 + static_cast<int>(rng() % 40000);
+    std::vector<int64_t> off{0};
+    for (int b = 0; b < B; ++b) off.push_back(off.back() + ((rng() % 3 == 0) ? 0 : 1 + rng() % 900));
+    if (check(off, 148)) {
+      std::printf("case large iter=%d B=%d\n", iter, B);
       return 1;
     }
     ++cases;
