@@ -4,6 +4,7 @@
 // from a compiled library.
 #pragma once
 
+#include "sa_internal.h"
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
