@@ -230,6 +230,62 @@ def workload_inputs(args, seed=None) -> dict:
     return inp
 
 
+class RankGroup:
+    """The ranks of one bench run: one process per GPU, with
+    torch.distributed only for the barrier around each timed region and the
+    reductions of the timings and row counts (the path itself has no
+    collective).  The reduction tensors live on `device`: the rank's GPU
+    with NCCL, the CPU with gloo."""
+
+    def __init__(self, world: int, device):
+        self.world = world
+        self.device = device
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def _reduce(self, x: float, op: str) -> float:
+        if self.world == 1:
+            return float(x)
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+        return float(t.item())
+
+    def max(self, x: float) -> float:
+        return self._reduce(x, "max")
+
+    def sum(self, x: float) -> float:
+        return self._reduce(x, "sum")
+
+
+def init_rank_group(world: int, local_rank: int, backend: str = "nccl") -> RankGroup:
+    """Joins the process group of a torchrun launch (env:// rendezvous) and
+    returns the bench's view of it; a single process needs no group."""
+    import torch
+    if world == 1:
+        return RankGroup(1, torch.device("cuda", local_rank) if backend == "nccl" else "cpu")
+    import datetime
+
+    import torch.distributed as dist
+    if backend == "nccl":
+        torch.cuda.set_device(local_rank)
+        device = torch.device("cuda", local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    else:
+        device = torch.device("cpu")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return RankGroup(world, device)
+
+
+def rank_seed(workload: str, rank: int) -> int:
+    """Each rank draws its own batch of the workload (weak scaling)."""
+    return WORKLOADS[workload].seed + rank
+
+
 def run_reference(args, rank: int):
     if rank != 0:
         return
@@ -267,9 +323,8 @@ def run_reference(args, rank: int):
 # our arm
 # ---------------------------------------------------------------------------
 
-def run_ours(args, rank: int, world: int, local_rank: int):
+def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
     import torch
-    import torch.distributed as dist
 
     from sketch_attention_compression_b200 import SketchQuery, load_library, read_device_status
 
@@ -277,7 +332,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = WORKLOADS[args.workload]
-    inp = workload_inputs(args, seed=w.seed + rank)  # each rank: its own batch
+    inp = workload_inputs(args, seed=rank_seed(args.workload, rank))
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     X = torch.from_numpy(inp["X"]).to(dev).to(tdt)
     P, W_Q, W_K = (torch.from_numpy(inp[k]).to(dev).to(tdt) for k in ("P", "W_Q", "W_K"))
@@ -292,16 +347,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     Xt = torch.empty((B, w.k, w.d), dtype=torch.float32, device=dev)
     m = torch.empty((B, w.k), dtype=torch.float32, device=dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier = ranks.barrier
+    max_over_ranks = ranks.max
 
     # warm-up (also checks the device flags once)
     for _ in range(max(args.warmup, 1)):
@@ -402,7 +449,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     else:
         achieved, peak, unit = flops / fused_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
     traffic = load_traffic()
-    rows_total = N * world
+    rows_total = ranks.sum(N)  # rows of all ranks' batches
     value = rows_total / (step_ms * 1e-3)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -476,16 +523,9 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank)
         return
-    if world > 1:
-        import datetime
-
-        import torch
-        import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
+    ranks = init_rank_group(world, local_rank, "nccl")
     try:
-        run_ours(args, rank, world, local_rank)
+        run_ours(args, rank, world, local_rank, ranks)
     finally:
         if world > 1:
             import torch.distributed as dist

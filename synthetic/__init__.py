@@ -27,4 +27,5 @@ from .workloads import (  # noqa: F401
     generate,
     round_to_bf16,
     ragged_lengths,
+    workload_lengths,
 )

@@ -166,16 +166,26 @@ def _finish(rng, lengths, d, k, dtype, x_kind, mix_components, mix_sd, scale):
                 dtype=dtype, d=d, k=k)
 
 
+def _draw_lengths(rng: np.random.Generator, w: "Workload") -> np.ndarray:
+    if w.lengths == "uniform":
+        return np.full(w.batch, w.n, dtype=np.int64)
+    if w.lengths == "loguniform":
+        return ragged_lengths(rng, w.batch, w.lo, w.hi)
+    raise ValueError(w.lengths)
+
+
+def workload_lengths(name: str, seed: Optional[int] = None) -> np.ndarray:
+    """The per-user lengths that ``generate(name, seed)`` draws (its first
+    draws), without drawing the rest of the batch."""
+    w = WORKLOADS[name]
+    return _draw_lengths(np.random.default_rng(w.seed if seed is None else seed), w)
+
+
 def generate(name: str, seed: Optional[int] = None) -> dict:
     """Draw the named workload (see ``WORKLOADS``) with its own seed."""
     w = WORKLOADS[name]
     rng = np.random.default_rng(w.seed if seed is None else seed)
-    if w.lengths == "uniform":
-        lengths = np.full(w.batch, w.n, dtype=np.int64)
-    elif w.lengths == "loguniform":
-        lengths = ragged_lengths(rng, w.batch, w.lo, w.hi)
-    else:
-        raise ValueError(w.lengths)
+    lengths = _draw_lengths(rng, w)
     out = _finish(rng, lengths, w.d, w.k, w.dtype, w.x_kind, w.mix_components,
                   w.mix_sd, None)
     out["workload"] = w.name

@@ -56,3 +56,16 @@ def test_small_workload_generation():
     assert list(inp["offsets"]) == [0, 1024]
     # W ~ N(0, 1/d): sample sd near 1/8
     assert abs(inp["W_K"].std() - 1 / 8) < 0.01
+
+
+def test_workload_lengths_are_generate_first_draws():
+    """workload_lengths (used by the bench to count each rank's rows) draws
+    exactly the lengths that generate draws first."""
+    import numpy as np
+    from synthetic import WORKLOADS, generate, ragged_lengths, workload_lengths
+    for name in ("single_n1024_d64_k16_fp32", "batch32_n10k_d128_k64_bf16"):
+        assert np.array_equal(workload_lengths(name), np.diff(generate(name)["offsets"]))
+        assert np.array_equal(workload_lengths(name, seed=7), np.diff(generate(name, seed=7)["offsets"]))
+    w = WORKLOADS["ragged256_loguniform_1k_100k_d128_k64_bf16"]
+    want = ragged_lengths(np.random.default_rng(w.seed + 1), w.batch, w.lo, w.hi)
+    assert np.array_equal(workload_lengths(w.name, seed=w.seed + 1), want)
