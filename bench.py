@@ -27,6 +27,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import re
 import statistics
@@ -340,6 +341,12 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
     B = len(inp["offsets"]) - 1
     N = int(inp["offsets"][-1])
     elem = 2 if w.dtype == "bf16" else 4
+    # An X that fits in L2 would let timed iterations hit in L2: the timed
+    # loops then rotate over enough copies that each iteration's X was
+    # evicted since its last use (copies x size > 2 x L2).
+    x_bytes = float(N) * w.d * elem
+    n_copies = 1 if x_bytes > L2_BYTES else int(math.ceil(2 * L2_BYTES / max(x_bytes, 1.0)))
+    Xs = [X] + [X.clone() for _ in range(n_copies - 1)]
 
     stream = torch.cuda.current_stream(dev)
     q = SketchQuery(P, W_Q, W_K, inp["scale"], stream=stream)
@@ -351,8 +358,8 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
     max_over_ranks = ranks.max
 
     # warm-up (also checks the device flags once)
-    for _ in range(max(args.warmup, 1)):
-        q.forward(X, offsets, Xt, m, ws, stream=stream)
+    for i in range(max(args.warmup, 1)):
+        q.forward(Xs[i % n_copies], offsets, Xt, m, ws, stream=stream)
     if read_device_status(ws, stream) != 0:
         raise RuntimeError("device flags raised during warm-up")
 
@@ -372,8 +379,8 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        q.forward(X, offsets, Xt, m, ws, stream=stream)
+    for i in range(args.steps):
+        q.forward(Xs[i % n_copies], offsets, Xt, m, ws, stream=stream)
         launches += 2
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -392,15 +399,15 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
         barrier()
         torch.cuda.synchronize(dev)
         ea.record(stream)
-        for _ in range(args.steps):
-            fn()
+        for i in range(args.steps):
+            fn(Xs[i % n_copies])
         eb.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
         return max_over_ranks(ea.elapsed_time(eb) / args.steps)
 
-    fused_ms = time_pass(lambda: q.partials(X, offsets, Xt, m, ws, stream=stream))
-    fin_ms = time_pass(lambda: q.finalize(X, offsets, Xt, m, ws, stream=stream))
+    fused_ms = time_pass(lambda x: q.partials(x, offsets, Xt, m, ws, stream=stream))
+    fin_ms = time_pass(lambda x: q.finalize(x, offsets, Xt, m, ws, stream=stream))
     if read_device_status(ws, stream) != 0:
         raise RuntimeError("device flags raised during the timed region")
 
@@ -472,7 +479,10 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
         "config": {
             "workload": args.workload, "users_per_gpu": B, "rows_per_gpu": N,
             "d": w.d, "k": w.k, "x_bytes_per_gpu": bytes_x,
-            "l2": f"inputs larger than L2 (X {bytes_x / 1e6:.1f} MB > {L2_BYTES / 1e6:.0f} MB)",
+            "l2": (f"inputs larger than L2 (X {bytes_x / 1e6:.1f} MB > {L2_BYTES / 1e6:.0f} MB)"
+                   if n_copies == 1 else
+                   f"X {bytes_x / 1e6:.1f} MB fits in L2: timed iterations rotate over "
+                   f"{n_copies} copies ({n_copies * bytes_x / 1e6:.0f} MB > 2 x L2)"),
             "parallelism": f"independent batch per GPU x{world}",
         },
         "roofline": {
