@@ -1,4 +1,5 @@
-"""Builds libsa.so in-tree with nvcc for sm_100a.
+"""Builds libsa.so (and libsa_inject.so, the fault-injection build the tests
+use) in-tree with nvcc for sm_100a.
 
     python -m sketch_attention_compression_b200.build [--verbose]
 
@@ -20,6 +21,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "_lib", "libsa.so")
+# Fault-injection build for the tests: same sources, a 2e8-cycle wait limit
+# and a device switch that stalls one copy (sa_debug_inject_stall).
+INJECT_LIB = os.path.join(PKG, "_lib", "libsa_inject.so")
+INJECT_DEFINES = ["-DSA_FAULT_INJECT", "-DSA_WAIT_TIMEOUT_CYCLES=200000000ll"]
 SOURCES = ["sa_api.cu", "sa_prepare.cu", "sa_fused.cu", "sa_simt.cu", "sa_finalize.cu",
            "sa_noalloc.cu", "sa_fused_pair.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -34,21 +39,25 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
-    os.makedirs(os.path.dirname(LIB), exist_ok=True)
+def build(verbose: bool = False, force: bool = False, inject: bool = False) -> str:
+    """Builds libsa.so, or with inject=True the fault-injection library."""
+    out_lib = INJECT_LIB if inject else LIB
+    obj_dir = os.path.join(BUILD, "inject") if inject else BUILD
+    defines = INJECT_DEFINES if inject else []
+    os.makedirs(obj_dir, exist_ok=True)
+    os.makedirs(os.path.dirname(out_lib), exist_ok=True)
     headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
     headers.append(os.path.join(ROOT, "include", "sa.h"))
     newest_header = max(os.path.getmtime(h) for h in headers)
     objs = []
     for src in SOURCES:
         spath = os.path.join(CSRC, src)
-        obj = os.path.join(BUILD, src.replace(".cu", ".o"))
+        obj = os.path.join(obj_dir, src.replace(".cu", ".o"))
         objs.append(obj)
         if (not force and os.path.exists(obj)
                 and os.path.getmtime(obj) >= max(os.path.getmtime(spath), newest_header)):
             continue
-        cmd = [nvcc(), "-c", spath, "-o", obj] + ARCH + CFLAGS
+        cmd = [nvcc(), "-c", spath, "-o", obj] + ARCH + CFLAGS + defines
         if verbose:
             cmd += ["-Xptxas", "-v"]
         res = subprocess.run(cmd, capture_output=True, text=True)
@@ -56,13 +65,19 @@ def build(verbose: bool = False, force: bool = False) -> str:
             sys.stderr.write(res.stdout + res.stderr)
         if res.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}")
-    cmd = [nvcc(), "-shared", "-o", LIB] + objs + ARCH + ["-Xcompiler", "-fPIC"]
+    cmd = [nvcc(), "-shared", "-o", out_lib] + objs + ARCH + ["-Xcompiler", "-fPIC"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
         raise RuntimeError("link failed")
-    return LIB
+    return out_lib
+
+
+def build_all(verbose: bool = False, force: bool = False) -> list:
+    """Both libraries: libsa.so and the fault-injection build."""
+    return [build(verbose, force), build(verbose, force, inject=True)]
 
 
 if __name__ == "__main__":
-    print(build(verbose="--verbose" in sys.argv, force="--force" in sys.argv))
+    for path in build_all(verbose="--verbose" in sys.argv, force="--force" in sys.argv):
+        print(path)

@@ -47,6 +47,18 @@
 #include "sa_plan.h"
 #include "sa_ptx.cuh"
 
+#ifdef SA_FAULT_INJECT
+// Fault-injection build only (libsa_inject.so, for the tests): when
+// sa_debug_inject_stall(t) has set a tile index >= 0, CTA 0's producer never
+// issues the copy of its tile t, so MMA1 waits on a barrier that nothing
+// completes until the (shortened) wait limit runs out, and the pass must
+// report DEVFLAG_TIMEOUT and leave the context usable.
+__device__ int g_inject_stall_tile = -1;
+extern "C" int sa_debug_inject_stall(int tile) {
+  return static_cast<int>(cudaMemcpyToSymbol(g_inject_stall_tile, &tile, sizeof(int)));
+}
+#endif
+
 namespace sa {
 namespace {
 
@@ -207,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t n_cached =
       (a.batch + 1 - b0) < Pl::kOffCache ? (a.batch + 1 - b0) : Pl::kOffCache;
 
+  uint32_t tiles_issued = 0;  // producer thread: X tiles whose TMA copy was issued
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -218,13 +231,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       TileCursor cur{SegmentWalker{a.offsets, a.batch, R0, R1, b0, off_cache, b0, n_cached}};
       int64_t r;
       uint32_t t = 0;
-      bool ok = true;
       while (cur.next(r)) {
         const int st = t % S;
-        if (!mbar_wait(&x_empty[st], ((t / S) & 1u) ^ 1u, abort_flag, sticky)) {
-          ok = false;
-          break;
+#ifdef SA_FAULT_INJECT
+        if (c == 0 && static_cast<int>(t) == g_inject_stall_tile) {
+          ++t;
+          continue;
         }
+#endif
+        if (!mbar_wait(&x_empty[st], ((t / S) & 1u) ^ 1u, abort_flag, sticky)) break;
         mbar_arrive_expect_tx(&x_full[st], kTileRows * D * 2);
 #pragma unroll
         for (int cb = 0; cb < D / 64; ++cb)
@@ -232,11 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            static_cast<int32_t>(r), pol);
         ++t;
       }
-      if (!ok) {  // let the copies in flight land before the CTA exits
-        for (uint32_t u = (t > static_cast<uint32_t>(S) ? t - S : 0u); u < t; ++u)
-          mbar_wait_bounded(&x_full[u % S], (u / S) & 1u);
-        mbar_wait_bounded(q_full, 0);
-      }
+      tiles_issued = t;
     }
   } else if (warp == 1 || warp == 3) {
     // ------------------------------------------------------------ MMA issuers
@@ -322,10 +333,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         ++seg;
-      }
-      if (!ok) {  // make sure none of this thread's MMAs still runs when TMEM is released
-        mma_commit(&drain[role]);
-        mbar_wait_bounded(&drain[role], 0);
       }
     }
   } else if (warp >= 4) {
@@ -513,6 +520,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (*abort_flag) {
+    // A role gave up (a bounded wait ran out): every role has now stopped,
+    // but copies and MMAs that the others issued may still be in flight.
+    // They must finish before the tensor memory is released and the CTA's
+    // shared memory is handed to the next CTA.
+    if (warp == 0 && lane == 0) {
+      const uint32_t t = tiles_issued;
+      for (uint32_t u = (t > static_cast<uint32_t>(S) ? t - S : 0u); u < t; ++u)
+        mbar_wait_bounded(&x_full[u % S], (u / S) & 1u);
+      mbar_wait_bounded(q_full, 0);
+    }
+    if ((warp == 1 || warp == 3) && lane == 0) {
+      const int role = warp == 1 ? 0 : 1;
+      mma_commit(&drain[role]);
+      mbar_wait_bounded(&drain[role], 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -141,6 +141,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   cluster_sync();
   tc_fence_after();
 
+  uint32_t tiles_issued = 0;  // producer thread: X tiles whose TMA copy was issued
   if (aligned) {
     const uint32_t tmem = *tmem_slot;
     const int64_t b0 = *b0_slot;
@@ -157,13 +158,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         TileCursor cur{SegmentWalker{a.offsets, a.batch, R0, R1, b0}};
         int64_t r;
         uint32_t t = 0;
-        bool ok = true;
         while (cur.next(r)) {
           const int st = t % S;
-          if (!mbar_wait(&x_empty[st], ((t / S) & 1u) ^ 1u, abort_flag, sticky)) {
-            ok = false;
-            break;
-          }
+          if (!mbar_wait(&x_empty[st], ((t / S) & 1u) ^ 1u, abort_flag, sticky)) break;
           mbar_arrive_expect_tx(&x_full[st], kTileRows * D * 2);
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb)
@@ -171,11 +168,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                         static_cast<int32_t>(r));
           ++t;
         }
-        if (!ok) {
-          for (uint32_t u = (t > static_cast<uint32_t>(S) ? t - S : 0u); u < t; ++u)
-            mbar_wait_bounded(&x_full[u % S], (u / S) & 1u);
-          mbar_wait_bounded(q_full, 0);
-        }
+        tiles_issued = t;
       }
     } else if (warp == 1 || warp == 3) {
       // ---------------------------------------------------------- MMA issuers
@@ -248,10 +241,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             }
           }
           ++seg;
-        }
-        if (!ok) {
-          mma_commit(&drain[role]);
-          mbar_wait_bounded(&drain[role], 0);
         }
       }
     } else if (warp >= 4) {
@@ -412,6 +401,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (aligned && *abort_flag) {
+    // A role gave up (a bounded wait ran out): let the copies and MMAs that
+    // other roles issued finish before the tensor memory is released.
+    if (warp == 0 && lane == 0) {
+      const uint32_t t = tiles_issued;
+      for (uint32_t u = (t > static_cast<uint32_t>(S) ? t - S : 0u); u < t; ++u)
+        mbar_wait_bounded(&x_full[u % S], (u / S) & 1u);
+      mbar_wait_bounded(q_full, 0);
+    }
+    if ((warp == 1 || warp == 3) && lane == 0) {
+      const int role = warp == 1 ? 0 : 1;
+      mma_commit(&drain[role]);
+      mbar_wait_bounded(&drain[role], 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
   if (aligned && warp == 2) {
     tc_fence_after();
     tmem_dealloc(*tmem_slot, 512);

@@ -26,7 +26,10 @@ enum : uint32_t {
 // Elapsed time is read from the per-SM cycle counter: %globaltimer is a slow
 // special register, and reading it inside polling loops costs hundreds of
 // cycles per iteration.
-constexpr long long kWaitTimeoutCycles = 4000000000ll;
+#ifndef SA_WAIT_TIMEOUT_CYCLES
+#define SA_WAIT_TIMEOUT_CYCLES 4000000000ll
+#endif
+constexpr long long kWaitTimeoutCycles = SA_WAIT_TIMEOUT_CYCLES;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

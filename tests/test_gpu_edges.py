@@ -47,6 +47,15 @@ def test_many_ctas_many_users_bf16():
     _full_parity(make_inputs(lens, d=128, k=128, dtype="bf16", seed=11))
 
 
+def test_many_tiny_users_per_cta():
+    # More users in a CTA's range than the shared-memory copy of the offsets
+    # holds (64 entries), so the segment walkers also read offsets from
+    # global memory; the 32-way range search takes three rounds.
+    rng = np.random.default_rng(21)
+    lens = rng.integers(0, 40, size=12000)
+    _full_parity(make_inputs(lens, d=128, k=64, dtype="bf16", seed=21))
+
+
 def test_one_long_user_split_across_all_ctas():
     _full_parity(make_inputs([200_000], d=128, k=64, dtype="bf16", seed=12))
 
