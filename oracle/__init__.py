@@ -15,6 +15,7 @@ from .sa_oracle import (  # noqa: F401
     prototype_mass,
     prototype_softmax,
     sa_batch,
+    sa_batch_user_queries,
     sa_user,
 )
 from .brute import sa_user_bruteforce  # noqa: F401

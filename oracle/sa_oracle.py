@@ -34,6 +34,8 @@ Readings where the page is silent (each also listed in the design doc):
   R5  a user with no rows has X~ = 0 and m = 0; rows outside a user's range
       contribute nothing to it (section 3.1: padding must not be assigned
       mass).
+  R12 (section 2.2) a refinement layer's SA step queries user b's rows with
+      that user's previous sketch in place of P^(0) (sa_batch_user_queries).
 
 Every function works in float64; float32 / bf16 inputs are upcast exactly.
 """
@@ -143,6 +145,33 @@ def sa_batch(X: np.ndarray, offsets: Sequence[int], P: np.ndarray,
     for b in (range(B) if users is None else users):
         lo, hi = int(offsets[b]), int(offsets[b + 1])
         Xt[b], m[b] = sa_user(X[lo:hi], P, W_Q, W_K, scale, steps=steps)
+    return Xt, m
+
+
+def sa_batch_user_queries(X: np.ndarray, offsets: Sequence[int], queries: np.ndarray,
+                          W_Q: np.ndarray, W_K: np.ndarray, scale: float,
+                          users: Optional[Sequence[int]] = None
+                          ) -> Tuple[np.ndarray, np.ndarray]:
+    """SA with a query matrix per user: user b's rows are queried by
+    ``queries[b]`` (k x d) in place of the shared P^(0).
+
+    Section 2.2 "Stacked Refinement" of the same notes: refinement layer l
+    starts from X~^(0) = P^(0) and each layer still reads the original X,
+    queried by the previous layer's sketch.  Reading R12: layer l's SA step
+    for user b is the section 2.1 computation with X~_b^(l-1) in place of
+    P^(0), with the same W_Q, W_K and scale arguments (whether the
+    projections differ per layer is left to the caller, who passes them).
+    Returns X~ (B x k x d) and m (B x k) in float64.
+    """
+    offsets = np.asarray(offsets, np.int64)
+    queries = np.asarray(queries)
+    B = len(offsets) - 1
+    _, k, d = queries.shape
+    Xt = np.zeros((B, k, d), F64)
+    m = np.zeros((B, k), F64)
+    for b in (range(B) if users is None else users):
+        lo, hi = int(offsets[b]), int(offsets[b + 1])
+        Xt[b], m[b] = sa_user(X[lo:hi], queries[b], W_Q, W_K, scale)
     return Xt, m
 
 
