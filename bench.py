@@ -41,7 +41,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synthetic import WORKLOADS, generate  # noqa: E402
+from synthetic import WORKLOADS, generate, user_queries  # noqa: E402
 
 METRIC = "SA history rows/sec and % of roofline (max(HBM, bf16 TC)) on 1 B200"
 DEFAULT_WORKLOAD = "batch16_n100k_d128_k128_mixture_bf16"
@@ -200,9 +200,10 @@ def blas_threads() -> int:
     return len(os.sched_getaffinity(0))
 
 
-def oracle_rows_per_s(inp: dict, budget_s: float, users=None):
+def oracle_rows_per_s(inp: dict, budget_s: float, users=None, queries=None):
     """Runs the oracle user by user until `budget_s` has elapsed (at least one
-    user); returns (rows/s, rows, seconds, users)."""
+    user); returns (rows/s, rows, seconds, users).  With `queries` (B, k, d),
+    user b is queried by queries[b] in place of P."""
     from oracle import sa_user
     offs = inp["offsets"]
     order = list(range(len(offs) - 1)) if users is None else users
@@ -211,7 +212,8 @@ def oracle_rows_per_s(inp: dict, budget_s: float, users=None):
     t0 = time.perf_counter()
     for b in order:
         lo, hi = int(offs[b]), int(offs[b + 1])
-        sa_user(inp["X"][lo:hi], inp["P"], inp["W_Q"], inp["W_K"], inp["scale"])
+        sa_user(inp["X"][lo:hi], inp["P"] if queries is None else queries[b], inp["W_Q"],
+                inp["W_K"], inp["scale"])
         rows += hi - lo
         done.append(b)
         if time.perf_counter() - t0 >= budget_s:
@@ -350,16 +352,38 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
 
     stream = torch.cuda.current_stream(dev)
     q = SketchQuery(P, W_Q, W_K, inp["scale"], stream=stream)
-    ws = q.new_workspace(B, N)
     Xt = torch.empty((B, w.k, w.d), dtype=torch.float32, device=dev)
     m = torch.empty((B, w.k), dtype=torch.float32, device=dev)
+    uq = args.user_queries
+    if uq:
+        # The SA step of a refinement layer: every user queried by its own
+        # k x d matrix (seeded like P), the same X and weights.
+        Q_host = torch.from_numpy(user_queries(B, w.k, w.d, seed=rank_seed(args.workload, rank)
+                                               + 100)).pin_memory()
+        Qd = Q_host.to(dev)
+        ws = torch.empty(q.workspace_bytes_user_queries(B, N), dtype=torch.uint8, device=dev)
+
+        def step(x):
+            q.forward_user_queries(Qd, x, offsets, Xt, m, ws, stream=stream)
+
+        def first_pass(x):
+            q.partials_user_queries(Qd, x, offsets, Xt, m, ws, stream=stream)
+    else:
+        ws = q.new_workspace(B, N)
+
+        def step(x):
+            q.forward(x, offsets, Xt, m, ws, stream=stream)
+
+        def first_pass(x):
+            q.partials(x, offsets, Xt, m, ws, stream=stream)
+    kernels_per_step = 3 if uq else 2
 
     barrier = ranks.barrier
     max_over_ranks = ranks.max
 
     # warm-up (also checks the device flags once)
     for i in range(max(args.warmup, 1)):
-        q.forward(Xs[i % n_copies], offsets, Xt, m, ws, stream=stream)
+        step(Xs[i % n_copies])
     if read_device_status(ws, stream) != 0:
         raise RuntimeError("device flags raised during warm-up")
 
@@ -380,8 +404,8 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(args.steps):
-        q.forward(Xs[i % n_copies], offsets, Xt, m, ws, stream=stream)
-        launches += 2
+        step(Xs[i % n_copies])
+        launches += kernels_per_step
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -406,7 +430,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
         barrier()
         return max_over_ranks(ea.elapsed_time(eb) / args.steps)
 
-    fused_ms = time_pass(lambda x: q.partials(x, offsets, Xt, m, ws, stream=stream))
+    fused_ms = time_pass(first_pass)
     fin_ms = time_pass(lambda x: q.finalize(x, offsets, Xt, m, ws, stream=stream))
     if read_device_status(ws, stream) != 0:
         raise RuntimeError("device flags raised during the timed region")
@@ -414,18 +438,37 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
     # -- timed region C: end to end on host buffers ----------------------
     X_host = X.cpu().pin_memory()
     offs_host = np.ascontiguousarray(inp["offsets"])
-    dev_buf = torch.empty(q.host_path_device_bytes(B, N), dtype=torch.uint8, device=dev)
-    out_x = torch.empty((B, w.k, w.d), dtype=torch.float32).pin_memory().numpy()
-    out_m = torch.empty((B, w.k), dtype=torch.float32).pin_memory().numpy()
+    out_x = torch.empty((B, w.k, w.d), dtype=torch.float32).pin_memory()
+    out_m = torch.empty((B, w.k), dtype=torch.float32).pin_memory()
     e2e_steps = max(3, min(args.steps, 20))
-    q.forward_host(X_host, offs_host, dev_buf, stream=stream, out_x=out_x, out_m=out_m)
+    if uq:
+        # Per-user queries have no host-buffer entry point: pinned host
+        # copies of X, the offsets and the queries on the same stream, the
+        # device call, and the copies of the results back.
+        offs_pinned = torch.from_numpy(offs_host).pin_memory()
+        X_e, off_e, Q_e = torch.empty_like(X), torch.empty_like(offsets), torch.empty_like(Qd)
+
+        def e2e_step():
+            X_e.copy_(X_host, non_blocking=True)
+            off_e.copy_(offs_pinned, non_blocking=True)
+            Q_e.copy_(Q_host, non_blocking=True)
+            q.forward_user_queries(Q_e, X_e, off_e, Xt, m, ws, stream=stream)
+            out_x.copy_(Xt, non_blocking=True)
+            out_m.copy_(m, non_blocking=True)
+    else:
+        dev_buf = torch.empty(q.host_path_device_bytes(B, N), dtype=torch.uint8, device=dev)
+        ox, om = out_x.numpy(), out_m.numpy()
+
+        def e2e_step():
+            q.forward_host(X_host, offs_host, dev_buf, stream=stream, out_x=ox, out_m=om)
+    e2e_step()
     barrier()
     torch.cuda.synchronize(dev)
     h0 = torch.cuda.Event(enable_timing=True)
     h1 = torch.cuda.Event(enable_timing=True)
     h0.record(stream)
     for _ in range(e2e_steps):
-        q.forward_host(X_host, offs_host, dev_buf, stream=stream, out_x=out_x, out_m=out_m)
+        e2e_step()
     h1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -455,12 +498,13 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
         achieved, peak, unit = bytes_x / fused_s / 1e9, peaks["hbm_gbs"], "GB/s"
     else:
         achieved, peak, unit = flops / fused_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-    traffic = load_traffic()
+    traffic = None if uq else load_traffic()  # the capture covers the shared-query pass
     rows_total = ranks.sum(N)  # rows of all ranks' batches
     value = rows_total / (step_ms * 1e-3)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        rps, rows, dt, users = oracle_rows_per_s(inp, args.cpu_budget)
+        rps, rows, dt, users = oracle_rows_per_s(inp, args.cpu_budget,
+                                                 queries=Q_host.numpy() if uq else None)
         cpu = {"value": rps, "unit": "rows/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"users {users[0]}..{users[-1]} ({rows} rows, {dt:.1f} s, numpy fp64)"}
     line = {
@@ -484,11 +528,14 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
                    f"X {bytes_x / 1e6:.1f} MB fits in L2: timed iterations rotate over "
                    f"{n_copies} copies ({n_copies * bytes_x / 1e6:.0f} MB > 2 x L2)"),
             "parallelism": f"independent batch per GPU x{world}",
+            "queries": ("per user: B x k x d fp32, the SA step of a refinement layer"
+                        if uq else "shared prototypes P"),
         },
         "roofline": {
             "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": achieved / peak, "traffic": traffic,
-            "kernel": ("simt_fp32_kernel" if w.dtype != "bf16" else
+            "kernel": ("user_query_kernel + " if uq else "") +
+                      ("simt_fp32_kernel" if w.dtype != "bf16" else
                        "fused_sa_pair_kernel" if w.k > (64 if w.d == 256 else 128) else
                        f"fused_sa_kernel<{w.d},{64 if w.k <= 64 else 128}>"),
             "kernel_ms": fused_ms, "finalize_ms": fin_ms,
@@ -501,7 +548,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
             "algorithmic": f"{2 * w.d} B and {4 * w.k * w.d} flop per row x {N} rows",
         },
         "e2e": {"value": rows_total / (e2e_ms * 1e-3), "unit": "rows/s",
-                "h2d_bytes_per_step": int(bytes_x + 8 * (B + 1)),
+                "h2d_bytes_per_step": int(bytes_x + 8 * (B + 1) + (4 * B * w.k * w.d if uq else 0)),
                 "d2h_bytes_per_step": int(4 * B * w.k * (w.d + 1)),
                 "ms_per_step": e2e_ms},
         "gpu_launches": launches,
@@ -521,6 +568,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0,
                     help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--user-queries", action="store_true",
+                    help="query every user with its own k x d matrix (refinement-layer SA step)")
     ap.add_argument("--users", type=int, default=0,
                     help="use only the first U users of the workload (smaller case)")
     args = ap.parse_args()

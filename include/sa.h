@@ -84,7 +84,8 @@ typedef struct sa_query_s* sa_query;
  *   stream                              the precompute kernel runs on it
  *   out   host; receives the handle
  *
- * Allocates device memory (cudaMalloc) for Q'.  P, W_Q and W_K are read by
+ * Allocates device memory (cudaMalloc) for Q' and for W_Q W_K^T * scale
+ * (d x d fp32, used by sa_sketch_forward_user_queries).  P, W_Q and W_K are read by
  * a kernel enqueued on `stream`; they must stay alive until it completes.
  * Returns SA_ERR_UNSUPPORTED for bf16 shapes without a tensor-core kernel
  * (bf16 supports k <= 128 for d = 64 and 128, and any k <= 256 for d = 256,
@@ -100,7 +101,8 @@ void sa_sketch_free(sa_query q);
 
 /* Bytes of device workspace sa_sketch_forward needs for a batch of `batch`
  * users and `total_rows` rows.  Independent of the batch size beyond a fixed
- * bound (it scales with the number of SMs, not with the number of users). */
+ * bound (it scales with the number of SMs, not with the number of users).
+ * Per-user queries need more: sa_workspace_bytes_user_queries. */
 size_t sa_workspace_bytes(sa_query q, int64_t batch, int64_t total_rows);
 
 /*
@@ -128,6 +130,48 @@ size_t sa_workspace_bytes(sa_query q, int64_t batch, int64_t total_rows);
 sa_status sa_sketch_forward(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
                             int64_t total_rows, float* X_tilde, float* mass, void* workspace,
                             size_t workspace_bytes, void* stream);
+
+/*
+ * sa_sketch_forward_user_queries -- the SA step of a refinement layer: user
+ * b's rows are queried by its own k x d matrix Q_b in place of P (section
+ * 2.2 "Stacked Refinement" of the same notes: layer l starts from the shared
+ * prototypes and queries the original X with the previous layer's sketch).
+ * For each user b:
+ *
+ *     S_b = (Q_b W_Q)(X_b W_K)^T * scale,  A_b = softmax over prototypes,
+ *     X~_b = A_b X_b,  m_b = A_b 1
+ *
+ * with W_Q, W_K and scale those of `q` (its P is not used).  The library
+ * forms Q'_b = Q_b (W_Q W_K^T * scale) in fp32 for every user (a kernel on
+ * `stream`, into the workspace) and runs the same fused pass, which loads
+ * each user's Q'_b where that user's rows begin.
+ *
+ *   q           prepared query (supplies d, k, dtype, W_Q, W_K, scale)
+ *   queries     device, B x k x d fp32 (4-byte aligned): Q_b for every user
+ *               (for example the previous layer's X~, or a function of it);
+ *               not modified
+ *   X, offsets, batch, total_rows, X_tilde, mass, stream
+ *               as for sa_sketch_forward
+ *   workspace   device, >= sa_workspace_bytes_user_queries(q, B, N) bytes,
+ *               256-byte aligned; one call at a time
+ *
+ * Returns SA_ERR_UNSUPPORTED for queries run on pairs of CTAs (bf16, d = 256,
+ * k > 64), SA_ERR_INVALID_ARG if queries is NULL with B > 0 or if B * k_pad
+ * reaches 2^31 (k_pad as sa_query_info reports), otherwise as
+ * sa_sketch_forward.  An empty user gets X~ = 0 and m = 0 whatever its Q_b.
+ */
+size_t sa_workspace_bytes_user_queries(sa_query q, int64_t batch, int64_t total_rows);
+/* The first two of the three kernels (Q'_b for every user, then the fused
+ * pass); sa_sketch_finalize with the same arguments (minus `queries`)
+ * completes the layer, as for sa_sketch_partials. */
+sa_status sa_sketch_partials_user_queries(sa_query q, const float* queries, const void* X,
+                                          const int64_t* offsets, int64_t batch,
+                                          int64_t total_rows, float* X_tilde, float* mass,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+sa_status sa_sketch_forward_user_queries(sa_query q, const float* queries, const void* X,
+                                         const int64_t* offsets, int64_t batch,
+                                         int64_t total_rows, float* X_tilde, float* mass,
+                                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * The two kernels sa_sketch_forward enqueues, for callers that schedule (or

@@ -34,6 +34,9 @@ SIGNATURES = {
     "sa_sketch_forward": (_i32, _FWD_ARGS),
     "sa_sketch_partials": (_i32, _FWD_ARGS),
     "sa_sketch_finalize": (_i32, _FWD_ARGS),
+    "sa_workspace_bytes_user_queries": (_sz, [_vp, _i64, _i64]),
+    "sa_sketch_forward_user_queries": (_i32, [_vp, _vp] + _FWD_ARGS[1:]),
+    "sa_sketch_partials_user_queries": (_i32, [_vp, _vp] + _FWD_ARGS[1:]),
     "sa_host_path_device_bytes": (_sz, [_vp, _i64, _i64]),
     "sa_sketch_forward_host": (_i32, _FWD_ARGS),
     "sa_sketch_forward_noalloc": (_i32, [_vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp]),
@@ -184,6 +187,38 @@ class SketchQuery:
         if check:
             read_device_status(workspace, stream)
         return X_tilde, mass
+
+    def workspace_bytes_user_queries(self, batch: int, total_rows: int) -> int:
+        return int(self._lib.sa_workspace_bytes_user_queries(self._h, batch, total_rows))
+
+    def forward_user_queries(self, queries, X, offsets, X_tilde=None, mass=None, workspace=None,
+                             stream=None, check: bool = False) -> Tuple[object, object]:
+        """The SA step of a refinement layer: user b's rows queried by
+        ``queries[b]`` ((B, k, d) fp32 CUDA tensor) with this query's W_Q,
+        W_K and scale.  Returns X~ (B, k, d) and m (B, k)."""
+        torch = _torch()
+        B = int(offsets.shape[0]) - 1
+        if queries.dtype != torch.float32 or tuple(queries.shape) != (B, self.k, self.d):
+            raise ValueError(f"queries must be float32 of shape ({B}, {self.k}, {self.d})")
+        if workspace is None:
+            workspace = torch.empty(self.workspace_bytes_user_queries(B, int(X.shape[0])),
+                                    dtype=torch.uint8, device=X.device)
+        args, X_tilde, mass, workspace = self._args(X, offsets, X_tilde, mass, workspace)
+        qp = _dev_ptr(queries, "queries") if B > 0 else ctypes.c_void_p(0)
+        sh = ctypes.c_void_p(_stream_handle(stream))
+        _check(self._lib.sa_sketch_forward_user_queries(self._h, qp, *args, sh),
+               "sa_sketch_forward_user_queries")
+        if check:
+            read_device_status(workspace, stream)
+        return X_tilde, mass
+
+    def partials_user_queries(self, queries, X, offsets, X_tilde, mass, workspace,
+                              stream=None) -> None:
+        """Q'_b and the fused pass of forward_user_queries (finalize() completes it)."""
+        args, *_ = self._args(X, offsets, X_tilde, mass, workspace)
+        _check(self._lib.sa_sketch_partials_user_queries(
+            self._h, _dev_ptr(queries, "queries"), *args, ctypes.c_void_p(_stream_handle(stream))),
+            "sa_sketch_partials_user_queries")
 
     def partials(self, X, offsets, X_tilde, mass, workspace, stream=None) -> None:
         args, *_ = self._args(X, offsets, X_tilde, mass, workspace)

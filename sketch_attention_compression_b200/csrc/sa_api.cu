@@ -18,6 +18,7 @@ struct sa_query_s {
   sa_dtype dtype;
   float* q_f32;      // [k][d]
   uint16_t* q_bf16;  // [k_pad][d], rows >= k zero
+  float* m_f32;      // [d][d]: W_Q W_K^T * scale * log2(e), for per-user queries
   CUtensorMap tmap_q;       // boxes of k_pad rows (k_pad <= 128)
   CUtensorMap tmap_q_half;  // boxes of 128 rows (k_pad == 256: one half per CTA of a pair)
 };
@@ -86,6 +87,15 @@ WsLayout ws_layout(const sa_query_s* q, int64_t total_rows) {
   return l;
 }
 
+// Per-user queries: rows per user of the per-call Q' array (k_pad for the
+// bf16 copy the tensor-core pass reads, k for fp32) and its bytes, placed
+// after the common workspace.
+int uq_rows(const sa_query_s* q) { return q->dtype == SA_BF16 ? q->k_pad : q->k; }
+size_t uq_bytes(const sa_query_s* q, int64_t batch) {
+  const size_t elem = q->dtype == SA_BF16 ? 2 : 4;
+  return round_up(static_cast<size_t>(batch) * uq_rows(q) * q->d * elem, 256);
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 bool same_device(const sa_query_s* q) {
@@ -95,8 +105,10 @@ bool same_device(const sa_query_s* q) {
 
 enum class Phase { kBoth, kPartials, kFinalize };
 
-sa_status run(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
-              int64_t total_rows, float* X_tilde, float* mass, void* workspace,
+// `queries` (device, [batch][k][d] fp32) selects per-user queries; nullptr
+// queries every user with the prepared Q'.
+sa_status run(sa_query q, const float* queries, const void* X, const int64_t* offsets,
+              int64_t batch, int64_t total_rows, float* X_tilde, float* mass, void* workspace,
               size_t workspace_bytes, void* stream, Phase phase) {
   if (q == nullptr) return SA_ERR_INVALID_ARG;
   if (batch < 0 || total_rows < 0 || total_rows > kMaxRows) return SA_ERR_INVALID_ARG;
@@ -105,11 +117,18 @@ sa_status run(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
     return SA_ERR_INVALID_ARG;
   if (total_rows > 0 && X == nullptr) return SA_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(X_tilde, 16) || !aligned(mass, 4) || !aligned(offsets, 8) ||
-      !aligned(workspace, 256))
+      !aligned(workspace, 256) || !aligned(queries, 4))
     return SA_ERR_INVALID_ARG;
   if (!same_device(q)) return SA_ERR_INVALID_ARG;
+  const bool user_q = queries != nullptr;
+  if (user_q) {
+    // The two-CTA pass (d = 256, k > 64) keeps its one Q' per CTA half; and
+    // the tensor map's row coordinate b * k_pad is a 32-bit integer.
+    if (q->dtype == SA_BF16 && q->k_pad == 256) return SA_ERR_UNSUPPORTED;
+    if (batch > (int64_t{1} << 31) / (q->k_pad > 0 ? q->k_pad : 1) - 1) return SA_ERR_INVALID_ARG;
+  }
   const WsLayout l = ws_layout(q, total_rows);
-  if (workspace_bytes < l.total) return SA_ERR_WORKSPACE;
+  if (workspace_bytes < l.total + (user_q ? uq_bytes(q, batch) : 0)) return SA_ERR_WORKSPACE;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -125,11 +144,23 @@ sa_status run(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
   a.part_x = reinterpret_cast<float*>(ws + l.part_x_off);
   a.part_m = reinterpret_cast<float*>(ws + l.part_m_off);
   a.header = reinterpret_cast<sa::WsHeader*>(ws);
+  a.user_queries = user_q ? 1 : 0;
   const int G = static_cast<int>(grid_for(q, total_rows));
 
   if (phase != Phase::kFinalize) {
     cudaError_t err;
+    void* uq = ws + l.total;  // per-call Q'_b array (per-user queries)
+    if (user_q &&
+        sa::launch_user_query(queries, q->m_f32, batch, q->k, uq_rows(q), q->d,
+                              q->dtype == SA_BF16 ? nullptr : static_cast<float*>(uq),
+                              q->dtype == SA_BF16 ? static_cast<uint16_t*>(uq) : nullptr,
+                              st) != cudaSuccess)
+      return SA_ERR_CUDA;
     if (q->dtype == SA_BF16) {
+      CUtensorMap tmq;
+      if (user_q && !make_tmap_bf16(&tmq, uq, static_cast<uint64_t>(batch) * q->k_pad,
+                                    static_cast<uint64_t>(q->d), static_cast<uint32_t>(q->k_pad)))
+        return SA_ERR_CUDA;
       CUtensorMap tmx;
       // A zero-row tensor map is not encodable; with N == 0 the kernel
       // issues no loads, so Q' stands in as a valid dummy.
@@ -140,9 +171,11 @@ sa_status run(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
                                            static_cast<uint64_t>(q->d), 64);
       if (!ok) return SA_ERR_CUDA;
       err = q->k_pad == 256 ? sa::launch_fused_bf16_pair(tmx, q->tmap_q_half, a, G, st)
-                            : sa::launch_fused_bf16(tmx, q->tmap_q, q->k_pad, a, G, st);
+                            : sa::launch_fused_bf16(tmx, user_q ? tmq : q->tmap_q, q->k_pad, a,
+                                                    G, st);
     } else {
-      err = sa::launch_simt_fp32(q->q_f32, static_cast<const float*>(X), a, G, st);
+      err = sa::launch_simt_fp32(user_q ? static_cast<const float*>(uq) : q->q_f32,
+                                 static_cast<const float*>(X), a, G, st);
     }
     if (err != cudaSuccess) return SA_ERR_CUDA;
   }
@@ -220,11 +253,15 @@ sa_status sa_prepare_query(const void* P, const void* W_Q, const void* W_K, int 
                               static_cast<uint64_t>(k_pad), static_cast<uint64_t>(d),
                               static_cast<uint32_t>(k_pad == 256 ? 128 : k_pad));
   }
+  ok = ok && cudaMalloc(&q->m_f32, static_cast<size_t>(d) * d * sizeof(float)) == cudaSuccess;
   ok = ok && sa::launch_prepare_query(P, W_Q, W_K, k, d, static_cast<double>(scale),
                                       dtype == SA_BF16, q->q_f32, q->q_bf16, st) == cudaSuccess;
+  ok = ok && sa::launch_prepare_projection(W_Q, W_K, d, static_cast<double>(scale),
+                                           dtype == SA_BF16, q->m_f32, st) == cudaSuccess;
   if (!ok) {
     cudaFree(q->q_f32);
     cudaFree(q->q_bf16);
+    cudaFree(q->m_f32);
     delete q;
     return SA_ERR_CUDA;
   }
@@ -236,6 +273,7 @@ void sa_sketch_free(sa_query q) {
   if (q == nullptr) return;
   cudaFree(q->q_f32);
   cudaFree(q->q_bf16);
+  cudaFree(q->m_f32);
   delete q;
 }
 
@@ -257,22 +295,45 @@ size_t sa_workspace_bytes(sa_query q, int64_t batch, int64_t total_rows) {
 sa_status sa_sketch_forward(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
                             int64_t total_rows, float* X_tilde, float* mass, void* workspace,
                             size_t workspace_bytes, void* stream) {
-  return run(q, X, offsets, batch, total_rows, X_tilde, mass, workspace, workspace_bytes, stream,
-             Phase::kBoth);
+  return run(q, nullptr, X, offsets, batch, total_rows, X_tilde, mass, workspace, workspace_bytes,
+             stream, Phase::kBoth);
 }
 
 sa_status sa_sketch_partials(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
                              int64_t total_rows, float* X_tilde, float* mass, void* workspace,
                              size_t workspace_bytes, void* stream) {
-  return run(q, X, offsets, batch, total_rows, X_tilde, mass, workspace, workspace_bytes, stream,
-             Phase::kPartials);
+  return run(q, nullptr, X, offsets, batch, total_rows, X_tilde, mass, workspace, workspace_bytes,
+             stream, Phase::kPartials);
 }
 
 sa_status sa_sketch_finalize(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
                              int64_t total_rows, float* X_tilde, float* mass, void* workspace,
                              size_t workspace_bytes, void* stream) {
-  return run(q, X, offsets, batch, total_rows, X_tilde, mass, workspace, workspace_bytes, stream,
-             Phase::kFinalize);
+  return run(q, nullptr, X, offsets, batch, total_rows, X_tilde, mass, workspace, workspace_bytes,
+             stream, Phase::kFinalize);
+}
+
+size_t sa_workspace_bytes_user_queries(sa_query q, int64_t batch, int64_t total_rows) {
+  if (q == nullptr || batch < 0 || total_rows < 0) return 0;
+  return ws_layout(q, total_rows).total + uq_bytes(q, batch);
+}
+
+sa_status sa_sketch_forward_user_queries(sa_query q, const float* queries, const void* X,
+                                         const int64_t* offsets, int64_t batch,
+                                         int64_t total_rows, float* X_tilde, float* mass,
+                                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (batch > 0 && queries == nullptr) return SA_ERR_INVALID_ARG;
+  return run(q, queries, X, offsets, batch, total_rows, X_tilde, mass, workspace,
+             workspace_bytes, stream, Phase::kBoth);
+}
+
+sa_status sa_sketch_partials_user_queries(sa_query q, const float* queries, const void* X,
+                                          const int64_t* offsets, int64_t batch,
+                                          int64_t total_rows, float* X_tilde, float* mass,
+                                          void* workspace, size_t workspace_bytes, void* stream) {
+  if (batch > 0 && queries == nullptr) return SA_ERR_INVALID_ARG;
+  return run(q, queries, X, offsets, batch, total_rows, X_tilde, mass, workspace,
+             workspace_bytes, stream, Phase::kPartials);
 }
 
 size_t sa_host_path_device_bytes(sa_query q, int64_t batch, int64_t total_rows) {
@@ -325,8 +386,8 @@ sa_status sa_sketch_forward_host(sa_query q, const void* X_host, const int64_t* 
     return SA_ERR_CUDA;
   if (cudaMemcpyAsync(o_dev, offsets_host, o_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return SA_ERR_CUDA;
-  sa_status s = run(q, x_dev, o_dev, batch, total_rows, xt_dev, m_dev, ws, ws_bytes, stream,
-                    Phase::kBoth);
+  sa_status s = run(q, nullptr, x_dev, o_dev, batch, total_rows, xt_dev, m_dev, ws, ws_bytes,
+                    stream, Phase::kBoth);
   if (s != SA_OK) return s;
   if (cudaMemcpyAsync(X_tilde_host, xt_dev, xt_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
       cudaMemcpyAsync(mass_host, m_dev, m_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)

@@ -31,7 +31,9 @@
 //   warp 0      TMA producer (X ring of Plan::S tiles; Q' once)
 //   warp 1      MMA1 issuer (one thread): as soon as an X stage has landed
 //               and its group's S^T buffer has been read out
-//   warp 2      TMEM allocation / release
+//   warp 2      TMEM allocation / release; with per-user queries, one
+//               thread loads each segment's Q'_b once MMA1 has finished
+//               with the previous user's
 //   warp 3      MMA2 issuer (one thread): as soon as the probabilities are
 //               stored (and, for a segment's first tile, X~ was drained)
 //   warps 4-7   softmax group 0 (even tiles), one thread per row
@@ -43,6 +45,13 @@
 // probability buffer.  The group that finishes a segment's last tile drains
 // X~ and m to the outputs (or to a partial slot for a user that crosses CTA
 // ranges).
+//
+// Per-user queries (the SA step of a refinement layer, section 2.2 "Stacked
+// Refinement" of the notes): the one Q' buffer is reloaded per segment.
+// MMA1 waits for Q'_b before a segment's first tile and commits q_empty
+// after its last, which lets warp 2 fetch the next user's Q' (from L2: the
+// per-call Q' array was just written).  The reload costs one TMA round trip
+// per segment boundary, partly hidden behind the two S^T buffers.
 #include "sa_internal.h"
 #include "sa_plan.h"
 #include "sa_ptx.cuh"
@@ -143,7 +152,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // [lane quarter]: the drain of segment s has finished reading its staging
   // buffers (phase s), so the drain of segment s + 1 may refill them.
   uint64_t* stage_free = drain + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stage_free + 4);
+  uint64_t* q_empty = stage_free + 4;  // per-user queries: MMA1 is done with this segment's Q'
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   int64_t* b0_slot = reinterpret_cast<int64_t*>(tmem_slot + 2);
   volatile uint32_t* mma2_issued = tmem_slot + 4;  // tiles whose MMA2 has been issued
@@ -175,6 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(acc_empty, 4);
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&stage_free[i], 1);
     *abort_flag = 0u;
     *mma2_issued = 0u;
@@ -219,15 +230,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t n_cached =
       (a.batch + 1 - b0) < Pl::kOffCache ? (a.batch + 1 - b0) : Pl::kOffCache;
 
+  const bool user_q = a.user_queries != 0;
   uint32_t tiles_issued = 0;  // producer thread: X tiles whose TMA copy was issued
+  uint32_t q_loads = 0;       // Q' loader thread (per-user queries): Q'_b copies issued
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      mbar_arrive_expect_tx(q_full, KM * D * 2);
+      if (!user_q) {
+        mbar_arrive_expect_tx(q_full, KM * D * 2);
 #pragma unroll
-      for (int cb = 0; cb < D / 64; ++cb)
-        tma_load_2d(q_s + cb * KM * 128, &tm_q, q_full, cb * 64, 0);
+        for (int cb = 0; cb < D / 64; ++cb)
+          tma_load_2d(q_s + cb * KM * 128, &tm_q, q_full, cb * 64, 0);
+      }
       TileCursor cur{SegmentWalker{a.offsets, a.batch, R0, R1, b0, off_cache, b0, n_cached}};
       int64_t r;
       uint32_t t = 0;
@@ -249,6 +264,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tiles_issued = t;
     }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ Q'_b loader
+    // Segment g's Q' (phase g of q_full) is copied once MMA1 has finished
+    // segment g - 1 (phase g - 1 of q_empty); rows user * KM.. of the
+    // per-call array (KM == k_pad on this pass).
+    if (lane == 0 && user_q) {
+      SegmentWalker w{a.offsets, a.batch, R0, R1, b0, off_cache, b0, n_cached};
+      int64_t user, s, e, lo, hi;
+      uint32_t g = 0;
+      while (w.next(user, s, e, lo, hi)) {
+        if (g > 0 && !mbar_wait(q_empty, (g - 1) & 1u, abort_flag, sticky)) break;
+        mbar_arrive_expect_tx(q_full, KM * D * 2);
+#pragma unroll
+        for (int cb = 0; cb < D / 64; ++cb)
+          tma_load_2d(q_s + cb * KM * 128, &tm_q, q_full, cb * 64, static_cast<int32_t>(user * KM));
+        ++g;
+      }
+      q_loads = g;
+    }
   } else if (warp == 1 || warp == 3) {
     // ------------------------------------------------------------ MMA issuers
     // A commit covers the MMAs of its own thread only: MMA1's commits
@@ -268,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = idesc_bf16_f32(kTileRows, KM, 0, 0);
       constexpr uint32_t idesc_x0 = idesc_bf16_f32(KM, Pl::kPartN0, 1, 1);
       constexpr uint32_t idesc_x1 = idesc_bf16_f32(KM, 144, 1, 1);
-      bool ok = role == 1 || mbar_wait(q_full, 0, abort_flag, sticky);
+      bool ok = true;
       SegmentWalker w{a.offsets, a.batch, R0, R1, b0, off_cache, b0, n_cached};
       int64_t user, s, e, lo, hi;
       uint32_t t = 0, seg = 0;
@@ -278,7 +312,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (role == 0) {
             // ---- MMA1: S^T_t = X_t Q'^T into the S^T buffer of tile t's group
             const int sb = t & 1;
-            if ((t >= kMma1Lead && !wait_count(mma2_issued, t + 1 - kMma1Lead, abort_flag, sticky)) ||
+            // Q' for this segment: loaded once (phase 0) for shared
+            // queries, phase seg of the per-user reloads otherwise.
+            if ((r == s && !mbar_wait(q_full, user_q ? (seg & 1u) : 0u, abort_flag, sticky)) ||
+                (t >= kMma1Lead && !wait_count(mma2_issued, t + 1 - kMma1Lead, abort_flag, sticky)) ||
                 !mbar_wait(&x_full[st], (t / S) & 1u, abort_flag, sticky) ||
                 !mbar_wait(&s_empty[sb], ((t >> 1) & 1u) ^ 1u, abort_flag, sticky)) {
               ok = false;
@@ -292,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           q_desc + (((ks >> 2) * (KM * 128) + (ks & 3) * 32) >> 4), idesc_s,
                           ks > 0 ? 1u : 0u);
             mma_commit(&s_full[sb]);
+            if (user_q && r + kTileRows >= e) mma_commit(q_empty);
           } else {
             // ---- MMA2: [X~ | m] += A_t [X_t | 1]  (a segment's first tile overwrites)
             const bool first = (r == s);
@@ -529,8 +567,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t t = tiles_issued;
       for (uint32_t u = (t > static_cast<uint32_t>(S) ? t - S : 0u); u < t; ++u)
         mbar_wait_bounded(&x_full[u % S], (u / S) & 1u);
-      mbar_wait_bounded(q_full, 0);
+      if (!user_q) mbar_wait_bounded(q_full, 0);
     }
+    if (warp == 2 && lane == 0 && q_loads > 0) mbar_wait_bounded(q_full, (q_loads - 1) & 1u);
     if ((warp == 1 || warp == 3) && lane == 0) {
       const int role = warp == 1 ? 0 : 1;
       mma_commit(&drain[role]);

@@ -180,6 +180,10 @@ struct PassArgs {
   float* part_x;     // [2G][k][d]
   float* part_m;     // [2G][k]
   WsHeader* header;
+  // 0: one Q' for every user.  1: user b's rows are queried by its own Q'_b
+  // (the tensor-core pass reads rows b * k_pad.. of its Q' tensor map, the
+  // fp32 pass the k x d block at b * k * d).
+  int user_queries;
 };
 
 // ---------------------------------------------------------------- launchers
@@ -190,6 +194,16 @@ struct PassArgs {
 cudaError_t launch_prepare_query(const void* P, const void* W_Q, const void* W_K, int k,
                                  int d, double scale, bool bf16_inputs, float* q_f32,
                                  uint16_t* q_bf16, cudaStream_t stream);
+
+// M = W_Q W_K^T * scale * log2(e) (d x d, fp32), for per-user queries.
+cudaError_t launch_prepare_projection(const void* W_Q, const void* W_K, int d, double scale,
+                                      bool bf16_inputs, float* m_f32, cudaStream_t stream);
+
+// Q'_b = Q_b M for b < batch: queries [batch][k][d] fp32 -> rows of k_rows
+// (>= k; rows k.. zero) written to out_f32 and/or out_bf16 ([batch][k_rows][d]).
+cudaError_t launch_user_query(const float* queries, const float* M, int64_t batch, int k,
+                              int k_rows, int d, float* out_f32, uint16_t* out_bf16,
+                              cudaStream_t stream);
 
 // Tensor-core pass (bf16 X).  Returns cudaErrorInvalidValue for an
 // unsupported (d, k_pad) pair.

@@ -10,7 +10,8 @@
 // Per CTA (256 threads), per 32-row tile of one user:
 //   1. the tile's rows (all d columns) are staged in shared memory;
 //   2. thread j < k computes s_ji = q'_j . x_i for the 32 rows (Q' rows come
-//      through the L1 cache; log2 e is folded into Q');
+//      through the L1 cache; log2 e is folded into Q'; with per-user queries
+//      the rows of the user's own Q'_b);
 //   3. each warp normalises 4 rows over the k prototypes: exp2(s - max) /
 //      sum (section 2.1: the normaliser runs over prototypes);
 //   4. every thread accumulates its (prototype, column) outputs
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(kThreadsSimt)
         float sacc[kRowsPerTile];
 #pragma unroll
         for (int rr = 0; rr < kRowsPerTile; ++rr) sacc[rr] = 0.f;
-        const float* qrow = qf + static_cast<int64_t>(tid) * d;
+        const float* qrow = qf + (a.user_queries ? user * k * d : 0) + static_cast<int64_t>(tid) * d;
         for (int f = 0; f < d; ++f) {
           const float qv = __ldg(qrow + f);
 #pragma unroll

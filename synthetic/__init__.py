@@ -17,6 +17,8 @@ Conventions (the notation of section 2.1 of that page):
   offsets  (B+1,)   int64, user b owns rows [offsets[b], offsets[b+1])
   P        (k, d)   shared prototypes P^(0)
   W_Q, W_K (d, d)   projections, used as  S = (P W_Q)(X W_K)^T * scale
+  queries  (B, k, d) per-user query matrices of a refinement layer's SA step
+                     (section 2.2), in place of P
 """
 
 from .workloads import (  # noqa: F401
@@ -27,5 +29,6 @@ from .workloads import (  # noqa: F401
     generate,
     round_to_bf16,
     ragged_lengths,
+    user_queries,
     workload_lengths,
 )

@@ -190,3 +190,13 @@ def generate(name: str, seed: Optional[int] = None) -> dict:
                   w.mix_sd, None)
     out["workload"] = w.name
     return out
+
+
+def user_queries(batch: int, k: int, d: int, seed: int) -> np.ndarray:
+    """Per-user query matrices Q_b (batch, k, d) float32 ~ N(0, 1), the same
+    distribution as the shared prototypes P, from their own generator (so a
+    workload's other arrays do not change).  They stand in for the previous
+    layer's sketch that a refinement layer queries with; they are fp32 (the
+    sketch's own type) and not rounded to bf16."""
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((batch, k, d), dtype=np.float32)
