@@ -536,7 +536,9 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
             "frac": achieved / peak, "traffic": traffic,
             "kernel": ("user_query_kernel + " if uq else "") +
                       ("simt_fp32_kernel" if w.dtype != "bf16" else
-                       "fused_sa_pair_kernel" if w.k > (64 if w.d == 256 else 128) else
+                       "fused_sa_pair_kernel" if w.d == 256 and w.k > 64 else
+                       f"fused_sa_kernel<{w.d},128> on clusters of {-(-w.k // 128)} CTAs"
+                       if w.k > 128 else
                        f"fused_sa_kernel<{w.d},{64 if w.k <= 64 else 128}>"),
             "kernel_ms": fused_ms, "finalize_ms": fin_ms,
             "kernel_timing": f"mean over {args.steps} back-to-back launches of the pass, "

@@ -77,7 +77,7 @@ typedef struct sa_query_s* sa_query;
  *   P     device, k x d, dtype          shared prototypes P^(0)
  *   W_Q   device, d x d, dtype          query projection
  *   W_K   device, d x d, dtype          key projection
- *   k     1 <= k <= 256                 number of prototypes
+ *   k     1 <= k <= 1024                number of prototypes
  *   d     64, 128 or 256                embedding width
  *   scale finite                        affinity scale (1/sqrt(d) in the paper's setting)
  *   dtype SA_BF16 or SA_FP32            element type of P, W_Q, W_K and of X later
@@ -87,10 +87,11 @@ typedef struct sa_query_s* sa_query;
  * Allocates device memory (cudaMalloc) for Q' and for W_Q W_K^T * scale
  * (d x d fp32, used by sa_sketch_forward_user_queries).  P, W_Q and W_K are read by
  * a kernel enqueued on `stream`; they must stay alive until it completes.
- * Returns SA_ERR_UNSUPPORTED for bf16 shapes without a tensor-core kernel
- * (bf16 supports k <= 128 for d = 64 and 128, and any k <= 256 for d = 256,
- * where k > 64 runs on pairs of CTAs that split the prototypes) or for a
- * GPU other than sm_100.
+ * Returns SA_ERR_UNSUPPORTED for shapes without a kernel, or for a GPU
+ * other than sm_100.  bf16: d = 64 and 128 take any k <= 1024 (k > 128 runs
+ * on clusters of ceil(k / 128) CTAs, each holding 128 prototypes; section
+ * 2.2 of the notes puts the final layers at about a thousand prototypes),
+ * d = 256 takes k <= 256 (k > 64 on pairs of CTAs).  fp32: k <= 256.
  */
 sa_status sa_prepare_query(const void* P, const void* W_Q, const void* W_K, int k, int d,
                            float scale, sa_dtype dtype, void* stream, sa_query* out);
@@ -156,7 +157,7 @@ sa_status sa_sketch_forward(sa_query q, const void* X, const int64_t* offsets, i
  *               256-byte aligned; one call at a time
  *
  * Returns SA_ERR_UNSUPPORTED for queries run on pairs of CTAs (bf16, d = 256,
- * k > 64), SA_ERR_INVALID_ARG if queries is NULL with B > 0 or if B * k_pad
+ * k > 64; the clusters of d = 64 and 128 take per-user queries), SA_ERR_INVALID_ARG if queries is NULL with B > 0 or if B * k_pad
  * reaches 2^31 (k_pad as sa_query_info reports), otherwise as
  * sa_sketch_forward.  An empty user gets X~ = 0 and m = 0 whatever its Q_b.
  */

@@ -11,7 +11,9 @@
 struct sa_query_s {
   int device;
   int sms;
-  int pair_units;  // co-resident two-CTA clusters (k_pad == 256)
+  int pair_units;  // co-resident two-CTA clusters (d == 256, k_pad == 256)
+  int ncl;         // CTAs per prototype-split cluster (d <= 128, k > 128), else 1
+  int cluster_units;  // co-resident clusters of ncl CTAs
   int k;
   int d;
   int k_pad;  // prototype rows of the bf16 Q' copy (multiple of 64), 0 for fp32
@@ -19,7 +21,7 @@ struct sa_query_s {
   float* q_f32;      // [k][d]
   uint16_t* q_bf16;  // [k_pad][d], rows >= k zero
   float* m_f32;      // [d][d]: W_Q W_K^T * scale * log2(e), for per-user queries
-  CUtensorMap tmap_q;       // boxes of k_pad rows (k_pad <= 128)
+  CUtensorMap tmap_q;       // boxes of k_pad rows (k_pad <= 128), of 128 rows for clusters
   CUtensorMap tmap_q_half;  // boxes of 128 rows (k_pad == 256: one half per CTA of a pair)
 };
 
@@ -69,7 +71,9 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // two-CTA pass (256 padded prototypes).
 int64_t grid_for(const sa_query_s* q, int64_t total_rows) {
   const int64_t T = sa::tiles_of(total_rows);
-  const int64_t units = (q->dtype == SA_BF16 && q->k_pad == 256) ? q->pair_units : q->sms;
+  const int64_t units = q->ncl > 1 ? q->cluster_units
+                        : (q->dtype == SA_BF16 && q->k_pad == 256) ? q->pair_units
+                                                                   : q->sms;
   int64_t G = T < units ? T : units;
   return G < 1 ? 1 : G;
 }
@@ -124,7 +128,7 @@ sa_status run(sa_query q, const float* queries, const void* X, const int64_t* of
   if (user_q) {
     // The two-CTA pass (d = 256, k > 64) keeps its one Q' per CTA half; and
     // the tensor map's row coordinate b * k_pad is a 32-bit integer.
-    if (q->dtype == SA_BF16 && q->k_pad == 256) return SA_ERR_UNSUPPORTED;
+    if (q->dtype == SA_BF16 && q->d == 256 && q->k_pad == 256) return SA_ERR_UNSUPPORTED;
     if (batch > (int64_t{1} << 31) / (q->k_pad > 0 ? q->k_pad : 1) - 1) return SA_ERR_INVALID_ARG;
   }
   const WsLayout l = ws_layout(q, total_rows);
@@ -159,7 +163,8 @@ sa_status run(sa_query q, const float* queries, const void* X, const int64_t* of
     if (q->dtype == SA_BF16) {
       CUtensorMap tmq;
       if (user_q && !make_tmap_bf16(&tmq, uq, static_cast<uint64_t>(batch) * q->k_pad,
-                                    static_cast<uint64_t>(q->d), static_cast<uint32_t>(q->k_pad)))
+                                    static_cast<uint64_t>(q->d),
+                                    static_cast<uint32_t>(q->ncl > 1 ? 128 : q->k_pad)))
         return SA_ERR_CUDA;
       CUtensorMap tmx;
       // A zero-row tensor map is not encodable; with N == 0 the kernel
@@ -170,9 +175,10 @@ sa_status run(sa_query q, const float* queries, const void* X, const int64_t* of
                           : make_tmap_bf16(&tmx, q->q_bf16, static_cast<uint64_t>(q->k_pad),
                                            static_cast<uint64_t>(q->d), 64);
       if (!ok) return SA_ERR_CUDA;
-      err = q->k_pad == 256 ? sa::launch_fused_bf16_pair(tmx, q->tmap_q_half, a, G, st)
-                            : sa::launch_fused_bf16(tmx, user_q ? tmq : q->tmap_q, q->k_pad, a,
-                                                    G, st);
+      const CUtensorMap& tq = user_q ? tmq : q->tmap_q;
+      err = q->ncl > 1 ? sa::launch_fused_bf16_cluster(tmx, tq, a, G, q->ncl, st)
+            : q->k_pad == 256 ? sa::launch_fused_bf16_pair(tmx, q->tmap_q_half, a, G, st)
+                              : sa::launch_fused_bf16(tmx, tq, q->k_pad, a, G, st);
     } else {
       err = sa::launch_simt_fp32(user_q ? static_cast<const float*>(uq) : q->q_f32,
                                  static_cast<const float*>(X), a, G, st);
@@ -206,7 +212,7 @@ sa_status sa_prepare_query(const void* P, const void* W_Q, const void* W_K, int 
   if (out == nullptr) return SA_ERR_INVALID_ARG;
   *out = nullptr;
   if (P == nullptr || W_Q == nullptr || W_K == nullptr) return SA_ERR_INVALID_ARG;
-  if (k < 1 || k > 256 || !(d == 64 || d == 128 || d == 256) || !isfinite(scale))
+  if (k < 1 || k > 1024 || !(d == 64 || d == 128 || d == 256) || !isfinite(scale))
     return SA_ERR_INVALID_ARG;
   if (dtype != SA_BF16 && dtype != SA_FP32) return SA_ERR_INVALID_ARG;
   const size_t elem = dtype == SA_BF16 ? 2 : 4;
@@ -221,10 +227,19 @@ sa_status sa_prepare_query(const void* P, const void* W_Q, const void* W_K, int 
   if (major != 10 || minor != 0) return SA_ERR_UNSUPPORTED;  // built for sm_100a only
 
   int k_pad = 0;
+  int ncl = 1;
   if (dtype == SA_BF16) {
-    // d = 256 with more than 64 prototypes runs on CTA pairs (256 padded).
-    k_pad = k <= 64 ? 64 : ((k <= 128 && d != 256) ? 128 : 256);
-    if (!sa::fused_bf16_supported(d, k_pad)) return SA_ERR_UNSUPPORTED;
+    // d = 256 with more than 64 prototypes runs on CTA pairs (256 padded);
+    // d = 64 or 128 with more than 128 on clusters of ceil(k / 128) CTAs.
+    if (d != 256 && k > 128) {
+      ncl = (k + 127) / 128;
+      k_pad = 128 * ncl;
+    } else {
+      k_pad = k <= 64 ? 64 : ((k <= 128 && d != 256) ? 128 : 256);
+      if (k > 256 || !sa::fused_bf16_supported(d, k_pad)) return SA_ERR_UNSUPPORTED;
+    }
+  } else if (k > 256) {
+    return SA_ERR_UNSUPPORTED;  // the fp32 pass keeps k <= 256 accumulators per thread row
   }
 
   sa_query_s* q = new (std::nothrow) sa_query_s;
@@ -232,7 +247,15 @@ sa_status sa_prepare_query(const void* P, const void* W_Q, const void* W_K, int 
   memset(q, 0, sizeof(*q));
   q->device = dev;
   q->sms = sms;
-  if (dtype == SA_BF16 && k_pad == 256) {
+  q->ncl = ncl;
+  if (ncl > 1) {
+    const int n = sa::fused_bf16_cluster_max_clusters(d, ncl);
+    if (n < 1) {
+      delete q;
+      return SA_ERR_UNSUPPORTED;
+    }
+    q->cluster_units = n < sms / ncl ? n : sms / ncl;
+  } else if (dtype == SA_BF16 && k_pad == 256) {
     const int n = sa::fused_bf16_pair_max_clusters();
     if (n < 1) {
       delete q;
@@ -249,9 +272,10 @@ sa_status sa_prepare_query(const void* P, const void* W_Q, const void* W_K, int 
   if (ok && dtype == SA_BF16) {
     const size_t qb = static_cast<size_t>(k_pad) * d * sizeof(uint16_t);
     ok = cudaMalloc(&q->q_bf16, qb) == cudaSuccess && cudaMemsetAsync(q->q_bf16, 0, qb, st) == cudaSuccess;
-    ok = ok && make_tmap_bf16(k_pad == 256 ? &q->tmap_q_half : &q->tmap_q, q->q_bf16,
+    const bool pair = ncl == 1 && k_pad == 256;
+    ok = ok && make_tmap_bf16(pair ? &q->tmap_q_half : &q->tmap_q, q->q_bf16,
                               static_cast<uint64_t>(k_pad), static_cast<uint64_t>(d),
-                              static_cast<uint32_t>(k_pad == 256 ? 128 : k_pad));
+                              static_cast<uint32_t>(k_pad > 128 ? 128 : k_pad));
   }
   ok = ok && cudaMalloc(&q->m_f32, static_cast<size_t>(d) * d * sizeof(float)) == cudaSuccess;
   ok = ok && sa::launch_prepare_query(P, W_Q, W_K, k, d, static_cast<double>(scale),

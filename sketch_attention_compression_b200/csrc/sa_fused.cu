@@ -46,6 +46,24 @@
 // X~ and m to the outputs (or to a partial slot for a user that crosses CTA
 // ranges).
 //
+// More than 128 prototypes (CLU): a cluster of C = k_pad / 128 CTAs (up to
+// 8, so k <= 1024; section 2.2 of the notes puts the final layers at about
+// a thousand prototypes) shares each row range.  CTA h holds prototypes
+// [128 h, 128 h + 128): its slice of Q', its S^T columns, its rows of the
+// accumulator; every CTA reads every X tile of the range (HBM once, L2 for
+// the others).  The softmax over all k prototypes of a row combines the
+// slices: each CTA computes its slice's maximum m_h and sum
+// z_h = sum_j exp2(s_j - m_h), publishes (m_h, z_h) in its own shared
+// memory and signals the other CTAs; each then reads all C pairs (in rank
+// order, so every CTA gets the same M and Z bit for bit) and scales its
+// exponentials by exp2(m_h - M) / Z, with M = max_h m_h and
+// Z = sum_h z_h exp2(m_h - M).  Each CTA sends its (m_h, z_h) of every row
+// to the others with st.async (the data and its arrival on the receiver's
+// barrier in one hop) into slots that take the place of the drain staging
+// (cluster CTAs drain straight from registers: they hold few segments); a
+// sender writes a group's slots again only after every receiver has
+// signalled that it read them (slot_free).
+//
 // Per-user queries (the SA step of a refinement layer, section 2.2 "Stacked
 // Refinement" of the notes): the one Q' buffer is reloaded per segment.
 // MMA1 waits for Q'_b before a segment's first tile and commits q_empty
@@ -117,13 +135,24 @@ __device__ __forceinline__ bool wait_count(volatile uint32_t* cnt, uint32_t targ
   return true;
 }
 
-// FULL: k == KM, so no prototype column needs masking.
-template <int D, int KM, bool FULL>
+// Warp-wide wait with cluster-scope acquire (data published by other CTAs).
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile uint32_t* abort_flag, uint32_t* sticky) {
+  const bool ok = mbar_wait_cluster(bar, parity, abort_flag, sticky);
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
+constexpr int kMaxCluster = 8;
+
+// FULL: no prototype column needs masking (k == KM, or k == KM * C for a
+// cluster).  CLU: prototype-split cluster of C CTAs (KM == 128 each).
+template <int D, int KM, bool FULL, bool CLU>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_sa_kernel(const __grid_constant__ CUtensorMap tm_x,
                     const __grid_constant__ CUtensorMap tm_q, const PassArgs a) {
   using Pl = Plan<D, KM>;
   constexpr int S = Pl::S;
+  static_assert(!CLU || KM == 128, "clusters split the prototypes in slices of 128");
 
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0u) {  // the 128-byte swizzle needs 1024-byte alignment
@@ -153,7 +182,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // buffers (phase s), so the drain of segment s + 1 may refill them.
   uint64_t* stage_free = drain + 2;
   uint64_t* q_empty = stage_free + 4;  // per-user queries: MMA1 is done with this segment's Q'
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + 1);
+  // Clusters: [group][lane quarter] the other CTAs' row statistics of this
+  // tile have arrived; [group] the other CTAs have read the ones we sent.
+  uint64_t* stats_full = q_empty + 1;
+  uint64_t* slot_free = stats_full + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(slot_free + 2);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   int64_t* b0_slot = reinterpret_cast<int64_t*>(tmem_slot + 2);
   volatile uint32_t* mma2_issued = tmem_slot + 4;  // tiles whose MMA2 has been issued
@@ -161,9 +194,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t G = gridDim.x;
-  const int64_t c = blockIdx.x;
+  // Row ranges: one per CTA, or one per cluster (whose CTAs are
+  // consecutive blocks; CTA h = rank h holds prototype slice h).
+  const uint32_t ncl = CLU ? cluster_size() : 1u;
+  const uint32_t h = CLU ? cluster_rank() : 0u;
+  const int64_t G = gridDim.x / ncl;
+  const int64_t c = blockIdx.x / ncl;
   const int64_t N = a.total_rows;
+  const int k_loc = CLU ? min(KM, a.k - static_cast<int>(h) * KM) : a.k;  // this CTA's prototypes
   uint32_t* sticky = &a.header->timeout_flags;
 
   int64_t* off_cache = reinterpret_cast<int64_t*>(smem + Pl::kOffs);
@@ -187,6 +225,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&stage_free[i], 1);
+    if (CLU) {
+      for (int i = 0; i < 8; ++i) mbar_init(&stats_full[i], 1);
+      for (int i = 0; i < 2; ++i) mbar_init(&slot_free[i], 4 * (ncl - 1));
+    }
     *abort_flag = 0u;
     *mma2_issued = 0u;
     fence_mbar_init();
@@ -222,7 +264,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       off_cache[i] = a.offsets[b0v + i];
   }
   tc_fence_before();
-  __syncthreads();
+  // With a cluster, the other CTAs' barriers must be initialised before
+  // this CTA signals them: the cluster barrier also covers the CTA's own.
+  if (CLU) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int64_t b0 = *b0_slot;
@@ -241,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(q_full, KM * D * 2);
 #pragma unroll
         for (int cb = 0; cb < D / 64; ++cb)
-          tma_load_2d(q_s + cb * KM * 128, &tm_q, q_full, cb * 64, 0);
+          tma_load_2d(q_s + cb * KM * 128, &tm_q, q_full, cb * 64, static_cast<int32_t>(h * KM));
       }
       TileCursor cur{SegmentWalker{a.offsets, a.batch, R0, R1, b0, off_cache, b0, n_cached}};
       int64_t r;
@@ -267,8 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 2) {
     // ------------------------------------------------------------ Q'_b loader
     // Segment g's Q' (phase g of q_full) is copied once MMA1 has finished
-    // segment g - 1 (phase g - 1 of q_empty); rows user * KM.. of the
-    // per-call array (KM == k_pad on this pass).
+    // segment g - 1 (phase g - 1 of q_empty): rows user * k_pad + h * KM..
+    // of the per-call array (k_pad = KM * C).
     if (lane == 0 && user_q) {
       SegmentWalker w{a.offsets, a.batch, R0, R1, b0, off_cache, b0, n_cached};
       int64_t user, s, e, lo, hi;
@@ -278,7 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(q_full, KM * D * 2);
 #pragma unroll
         for (int cb = 0; cb < D / 64; ++cb)
-          tma_load_2d(q_s + cb * KM * 128, &tm_q, q_full, cb * 64, static_cast<int32_t>(user * KM));
+          tma_load_2d(q_s + cb * KM * 128, &tm_q, q_full, cb * 64,
+                      static_cast<int32_t>((user * ncl + h) * KM));
         ++g;
       }
       q_loads = g;
@@ -378,8 +423,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int grp = (warp - 4) >> 2;       // 0: even tiles, 1: odd tiles
     const int q = warp & 3;                // TMEM lane quarter of this warp
     const int row = q * 32 + lane;         // tile row = TMEM lane of S^T
+    const uint32_t xch_a = sbase + Pl::kXch;  // clusters: received row statistics [group][src][row]
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    const int k = a.k;
+    const int k = k_loc;
     SegmentWalker w{a.offsets, a.batch, R0, R1, b0, off_cache, b0, n_cached};
     int64_t user, s, e, lo, hi;
     uint32_t t = 0, seg = 0;
@@ -403,6 +449,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         warp_arrive(&s_empty[grp], lane);
 
+        // Padded prototypes (j >= k) get logit -inf, so they add nothing
+        // to the maximum and exp2 gives them exactly 0.  Only 32-column
+        // chunks that reach past k are touched (the test is uniform).
+        if constexpr (!FULL) {
+#pragma unroll
+          for (int cc = 0; cc < KM / 32; ++cc) {
+            if (cc * 32 + 32 > k) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (cc * 32 + i >= k) sr[cc][i] = __float_as_uint(-INFINITY);
+            }
+          }
+        }
         // Stable softmax over the prototype axis (thread-local): four
         // independent max chains (three-input max) and four packed sums.
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -411,9 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int ja = j + 2 * u, jb = ja + 1;
-            const float va = (FULL || ja < k) ? __uint_as_float(sr[ja >> 5][ja & 31]) : -INFINITY;
-            const float vb = (FULL || jb < k) ? __uint_as_float(sr[jb >> 5][jb & 31]) : -INFINITY;
-            mx4[u] = max3f(mx4[u], va, vb);
+            mx4[u] = max3f(mx4[u], __uint_as_float(sr[ja >> 5][ja & 31]),
+                           __uint_as_float(sr[jb >> 5][jb & 31]));
           }
         }
         const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
@@ -426,8 +484,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    __uint_as_float(sr[(j + 1) >> 5][(j + 1) & 31])),
                            neg_m),
                     x0, x1);
-          const float e0 = (FULL || j < k) ? ex2_approx(x0) : 0.f;
-          const float e1 = (FULL || j + 1 < k) ? ex2_approx(x1) : 0.f;
+          const float e0 = ex2_approx(x0);
+          const float e1 = ex2_approx(x1);
           sr[j >> 5][j & 31] = __float_as_uint(e0);
           sr[(j + 1) >> 5][(j + 1) & 31] = __float_as_uint(e1);
           z2[(j >> 1) & 3] = f2_add(z2[(j >> 1) & 3], f2_pack(e0, e1));
@@ -435,7 +493,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         float za, zb, zc, zd;
         f2_unpack(f2_add(z2[0], z2[1]), za, zb);
         f2_unpack(f2_add(z2[2], z2[3]), zc, zd);
-        const float inv = valid ? 1.0f / ((za + zb) + (zc + zd)) : 0.f;
+        const float zl = (za + zb) + (zc + zd);
+        float inv;
+        if constexpr (CLU) {
+          // Send (m_h, z_h) of this row to every other CTA (slot [grp][h]
+          // of theirs, arriving on their stats_full[grp][q]) once they have
+          // all read what this group sent for its previous tile; then wait
+          // for theirs, which arrive in our slots [grp][p].
+          const uint32_t u = t >> 1;
+          if (u > 0 && !warp_wait_cluster(&slot_free[grp], (u - 1) & 1u, abort_flag, sticky)) {
+            ok = false;
+            break;
+          }
+          uint64_t* sfull = &stats_full[grp * 4 + q];
+          if (lane == 0) mbar_arrive_expect_tx(sfull, (ncl - 1) * 32 * 8);
+          const uint32_t sfull_a = smem_u32(sfull);
+          const uint32_t mine = xch_a + ((grp * 8 + h) * 128 + row) * 8;
+          for (uint32_t p = 0; p < ncl; ++p)
+            if (p != h) st_async_v2f(map_to_cta(mine, p), mx, zl, map_to_cta(sfull_a, p));
+          if (!warp_wait_cluster(sfull, u & 1u, abort_flag, sticky)) {
+            ok = false;
+            break;
+          }
+          float mv[kMaxCluster], zv[kMaxCluster];
+#pragma unroll
+          for (int p = 0; p < kMaxCluster; ++p) {
+            mv[p] = -INFINITY;
+            zv[p] = 0.f;
+            if (p < static_cast<int>(ncl)) {
+              if (p == static_cast<int>(h)) {
+                mv[p] = mx;
+                zv[p] = zl;
+              } else {
+                ld_shared_v2f(xch_a + ((grp * 8 + p) * 128 + row) * 8, mv[p], zv[p]);
+              }
+            }
+          }
+          float Mx = mv[0];
+#pragma unroll
+          for (int p = 1; p < kMaxCluster; ++p) Mx = fmaxf(Mx, mv[p]);
+          float Z = 0.f;
+#pragma unroll
+          for (int p = 0; p < kMaxCluster; ++p)
+            if (p < static_cast<int>(ncl)) Z += zv[p] * ex2_approx(mv[p] - Mx);
+          // Every lane's loads have returned (Mx and Z are pinned as
+          // computed before the warp barrier): the senders may write
+          // these slots again.
+          asm volatile("" : "+f"(Mx), "+f"(Z));
+          __syncwarp();
+          if (lane == 0)
+            for (uint32_t p = 0; p < ncl; ++p)
+              if (p != h) mbar_arrive_remote_relaxed(map_to_cta(smem_u32(&slot_free[grp]), p));
+          inv = valid ? ex2_approx(mx - Mx) / Z : 0.f;
+        } else {
+          inv = valid ? 1.0f / zl : 0.f;
+        }
         const uint64_t inv2 = f2_pack(inv, inv);
 
         // This warp's slice of the probability buffer is free once the
@@ -485,14 +597,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!warp_wait(&acc_full[seg & 1u], (seg >> 1) & 1u, abort_flag, sticky)) { ok = false; break; }
           tc_fence_after();
           const int64_t slotp = segment_slot(c, lo, hi, R0, R1);
-          float* dm = slotp < 0 ? a.out_m + user * k : a.part_m + slotp * k;
-          float* dxo = slotp < 0 ? a.out_x + user * k * D : a.part_x + slotp * k * D;
+          // This CTA's prototype rows start at h * KM of the user's k.
+          const int64_t krow = static_cast<int64_t>(h) * KM;
+          float* dm = (slotp < 0 ? a.out_m + user * a.k : a.part_m + slotp * a.k) + krow;
+          float* dxo = (slotp < 0 ? a.out_x + user * a.k * D : a.part_x + slotp * a.k * D) + krow * D;
           // M=128: prototype j sits in TMEM lane j.  M=64: prototypes
           // 16q..16q+15 sit in lanes 32q..32q+15.
           const int j0 = KM == 128 ? q * 32 : q * 16;
           const int j = j0 + lane;
           const bool has = (KM == 128 ? true : lane < 16) && j < k;
-          if (seg > 0 && !warp_wait(&stage_free[q], (seg - 1) & 1u, abort_flag, sticky)) {
+          if (!CLU && seg > 0 && !warp_wait(&stage_free[q], (seg - 1) & 1u, abort_flag, sticky)) {
             ok = false;
             break;
           }
@@ -524,31 +638,48 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_fence_before();
               warp_arrive(acc_empty, lane);
             }
-            // 32-column chunks: each lane stages its row (128 bytes, the
-            // 16-byte unit index XOR-ed with row mod 8), then the warp
-            // writes four whole rows per store.
+            if constexpr (CLU) {
+              // Straight from registers: lane j writes its row's columns.
+              if (has) {
 #pragma unroll
-            for (int cc = 0; cc < kDrainCols / 32; ++cc, ++chunk) {
-              if (chunk > 0) __syncwarp();  // the previous chunk's reads are done
-              if (lane < Pl::kDrainRows) {
+                for (int cc = 0; cc < kDrainCols / 32; ++cc) {
+                  float4* dst = reinterpret_cast<float4*>(dxo + static_cast<int64_t>(j) * D +
+                                                          bt * kDrainCols + cc * 32);
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                  st_shared_v4(stage + lane * 128 + ((u ^ (lane & 7)) << 4), v[cc][4 * u],
-                               v[cc][4 * u + 1], v[cc][4 * u + 2], v[cc][4 * u + 3]);
+                  for (int w4 = 0; w4 < 8; ++w4)
+                    dst[w4] = make_float4(__uint_as_float(v[cc][4 * w4]),
+                                          __uint_as_float(v[cc][4 * w4 + 1]),
+                                          __uint_as_float(v[cc][4 * w4 + 2]),
+                                          __uint_as_float(v[cc][4 * w4 + 3]));
+                }
               }
-              __syncwarp();
+            } else {
+              // 32-column chunks: each lane stages its row (128 bytes, the
+              // 16-byte unit index XOR-ed with row mod 8), then the warp
+              // writes four whole rows per store.
 #pragma unroll
-              for (int i = 0; i < Pl::kDrainRows / 4; ++i) {
-                const int rr = 4 * i + (lane >> 3), uu = lane & 7;
-                const float4 w = ld_shared_v4f(stage + rr * 128 + ((uu ^ (rr & 7)) << 4));
-                if (j0 + rr < k)
-                  *reinterpret_cast<float4*>(dxo + static_cast<int64_t>(j0 + rr) * D +
-                                             bt * kDrainCols + cc * 32 + uu * 4) = w;
+              for (int cc = 0; cc < kDrainCols / 32; ++cc, ++chunk) {
+                if (chunk > 0) __syncwarp();  // the previous chunk's reads are done
+                if (lane < Pl::kDrainRows) {
+#pragma unroll
+                  for (int u = 0; u < 8; ++u)
+                    st_shared_v4(stage + lane * 128 + ((u ^ (lane & 7)) << 4), v[cc][4 * u],
+                                 v[cc][4 * u + 1], v[cc][4 * u + 2], v[cc][4 * u + 3]);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < Pl::kDrainRows / 4; ++i) {
+                  const int rr = 4 * i + (lane >> 3), uu = lane & 7;
+                  const float4 w = ld_shared_v4f(stage + rr * 128 + ((uu ^ (rr & 7)) << 4));
+                  if (j0 + rr < k)
+                    *reinterpret_cast<float4*>(dxo + static_cast<int64_t>(j0 + rr) * D +
+                                               bt * kDrainCols + cc * 32 + uu * 4) = w;
+                }
               }
             }
           }
           __syncwarp();
-          if (lane == 0) mbar_arrive(&stage_free[q]);
+          if (!CLU && lane == 0) mbar_arrive(&stage_free[q]);
           if (has) dm[j] = __uint_as_float(mv);
         }
       }
@@ -582,12 +713,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // No CTA of a cluster leaves while another may still read its published
+  // statistics or signal its barriers.
+  if (CLU) cluster_sync();
 }
 
 template <int D, int KM>
 cudaError_t launch_one(const CUtensorMap& tx, const CUtensorMap& tq, const PassArgs& a,
                        int grid, cudaStream_t stream) {
-  auto kern = a.k == KM ? fused_sa_kernel<D, KM, true> : fused_sa_kernel<D, KM, false>;
+  auto kern = a.k == KM ? fused_sa_kernel<D, KM, true, false> : fused_sa_kernel<D, KM, false, false>;
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Plan<D, KM>::kSmem);
   if (err != cudaSuccess) return err;
@@ -604,7 +738,71 @@ cudaError_t launch_one(const CUtensorMap& tx, const CUtensorMap& tq, const PassA
   return cudaLaunchKernelEx(&cfg, kern, tx, tq, a);
 }
 
+// Prototype-split clusters: `ranges` clusters of `ncl` CTAs (k_pad = 128 ncl).
+template <int D>
+cudaLaunchConfig_t cluster_config(int ranges, int ncl, cudaStream_t stream,
+                                  cudaLaunchAttribute (&attr)[2]) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ranges * ncl));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Plan<D, 128>::kSmem;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(ncl);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cfg;
+}
+
+template <int D>
+cudaError_t launch_cluster(const CUtensorMap& tx, const CUtensorMap& tq, const PassArgs& a,
+                           int ranges, int ncl, cudaStream_t stream) {
+  auto kern = a.k == 128 * ncl ? fused_sa_kernel<D, 128, true, true>
+                               : fused_sa_kernel<D, 128, false, true>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Plan<D, 128>::kSmem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = cluster_config<D>(ranges, ncl, stream, attr);
+  return cudaLaunchKernelEx(&cfg, kern, tx, tq, a);
+}
+
+template <int D>
+int cluster_capacity(int ncl) {
+  auto kern = fused_sa_kernel<D, 128, false, true>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Plan<D, 128>::kSmem) != cudaSuccess)
+    return 0;
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = cluster_config<D>(1, ncl, nullptr, attr);
+  cfg.numAttrs = 1;  // the cluster shape alone
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) return 0;
+  return n;
+}
+
 }  // namespace
+
+int fused_bf16_cluster_max_clusters(int d, int ncl) {
+  if (ncl < 2 || ncl > kMaxCluster) return 0;
+  if (d == 64) return cluster_capacity<64>(ncl);
+  if (d == 128) return cluster_capacity<128>(ncl);
+  return 0;
+}
+
+cudaError_t launch_fused_bf16_cluster(const CUtensorMap& tx, const CUtensorMap& tq,
+                                      const PassArgs& a, int ranges, int ncl,
+                                      cudaStream_t stream) {
+  if (ncl < 2 || ncl > kMaxCluster || a.k > 128 * ncl || a.k <= 128 * (ncl - 1))
+    return cudaErrorInvalidValue;
+  if (a.d == 64) return launch_cluster<64>(tx, tq, a, ranges, ncl, stream);
+  if (a.d == 128) return launch_cluster<128>(tx, tq, a, ranges, ncl, stream);
+  return cudaErrorInvalidValue;
+}
 
 bool fused_bf16_supported(int d, int k_pad) {
   return (d == 64 && (k_pad == 64 || k_pad == 128)) ||

@@ -211,6 +211,16 @@ cudaError_t launch_fused_bf16(const CUtensorMap& tmap_x, const CUtensorMap& tmap
                               int k_pad, const PassArgs& a, int grid, cudaStream_t stream);
 bool fused_bf16_supported(int d, int k_pad);
 
+// Tensor-core pass for d = 64 or 128 and 129..1024 prototypes: `ranges`
+// clusters of ncl = k_pad / 128 CTAs (2..8), each CTA a slice of 128
+// prototypes.  tmap_q reads 128-row boxes of the padded Q' (k_pad x d, or
+// batch * k_pad x d with per-user queries).
+cudaError_t launch_fused_bf16_cluster(const CUtensorMap& tmap_x, const CUtensorMap& tmap_q,
+                                      const PassArgs& a, int ranges, int ncl,
+                                      cudaStream_t stream);
+// How many such clusters fit on the GPU at once (0 if none or on error).
+int fused_bf16_cluster_max_clusters(int d, int ncl);
+
 // Tensor-core pass for d = 256 and 129..256 prototypes: clusters of two CTAs,
 // one per prototype half; `ranges` row ranges, 2 * ranges CTAs.  tmap_q_half
 // reads 128-row boxes of the padded Q' (256 x 256).

@@ -338,6 +338,21 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   return r;
 }
 
+// Number of CTAs in this CTA's cluster.
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+
+// Arrival on an mbarrier in another CTA's shared memory (address from
+// map_to_cta), with no memory ordering of its own (a signal that carries
+// no data; data travels with st.async).
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
+               : "memory");
+}
+
 // All threads of all CTAs of the cluster (every warp must execute it).
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\t"

@@ -47,11 +47,12 @@ class Workload:
     mix_sd: float = 0.0
 
 
-# The five workloads.  Their shapes are the ones the method is quoted on:
+# The workloads.  Their shapes are the ones the method is quoted on:
 # single users of ~1K rows for the exact fp32 check, batches of 10K- and
 # 100K-row histories at width 128 (the final SA width of section 3.2), a
-# ragged batch spanning the whole 1K-100K range, and a wide d=256/k=256 case
-# where the tensor cores rather than HBM bound the step.
+# ragged batch spanning the whole 1K-100K range, a wide d=256/k=256 case
+# where the tensor cores rather than HBM bound the step, and the 100K batch
+# with about a thousand prototypes.
 WORKLOADS: Dict[str, Workload] = {
     w.name: w
     for w in [
@@ -67,6 +68,11 @@ WORKLOADS: Dict[str, Workload] = {
                  lo=1_000, hi=100_000),
         Workload("batch8_n100k_d256_k256_bf16", batch=8, n=100_000, d=256,
                  k=256, dtype="bf16", seed=1004),
+        # The 16 x 100K mixture batch at the prototype count of the final
+        # refinement layers (about a thousand; section 2.2).
+        Workload("batch16_n100k_d128_k1000_mixture_bf16", batch=16, n=100_000,
+                 d=128, k=1000, dtype="bf16", seed=1005, x_kind="mixture",
+                 mix_components=512, mix_sd=0.3),
     ]
 }
 

@@ -60,7 +60,7 @@ def test_null_and_range_arguments_rejected_on_host(lib):
                               ctypes.byref(out))
     assert st == binding.SA_ERR_INVALID_ARG and out.value is None
     dummy = ctypes.c_void_p(256)
-    for k, d in [(0, 64), (257, 64), (16, 96), (16, 512)]:
+    for k, d in [(0, 64), (1025, 64), (16, 96), (16, 512)]:
         st = lib.sa_prepare_query(dummy, dummy, dummy, k, d, 0.1, binding.SA_BF16, None,
                                   ctypes.byref(out))
         assert st == binding.SA_ERR_INVALID_ARG

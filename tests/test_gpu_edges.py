@@ -192,13 +192,15 @@ def test_partials_then_finalize_equals_forward():
     assert torch.equal(Xt, Xt2) and torch.equal(m, m2)
 
 
-@pytest.mark.parametrize("d", [64, 128])
-def test_more_than_128_prototypes_needs_d256(d):
-    """bf16 with k > 128 has a kernel only for d = 256 (pairs of CTAs split
-    the prototypes); other widths report SA_ERR_UNSUPPORTED on the host."""
+@pytest.mark.parametrize("d,k,dtype,status", [(256, 257, "bf16", "unsupported"),
+                                               (128, 257, "fp32", "unsupported"),
+                                               (128, 1025, "bf16", "invalid")])
+def test_prototype_limits(d, k, dtype, status):
+    """bf16 takes k <= 1024 at d = 64 and 128 (clusters) and k <= 256 at
+    d = 256 (pairs); fp32 takes k <= 256.  Beyond: an error on the host."""
     from sketch_attention_compression_b200 import SAError, SketchQuery
-    from sketch_attention_compression_b200.binding import SA_ERR_UNSUPPORTED
-    dev = to_device(make_inputs([10], d=d, k=129, dtype="bf16", seed=24))
+    from sketch_attention_compression_b200.binding import SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED
+    dev = to_device(make_inputs([10], d=d, k=k, dtype=dtype, seed=24))
     with pytest.raises(SAError) as e:
         SketchQuery(dev["P"], dev["W_Q"], dev["W_K"], 0.1)
-    assert e.value.status == SA_ERR_UNSUPPORTED
+    assert e.value.status == (SA_ERR_UNSUPPORTED if status == "unsupported" else SA_ERR_INVALID_ARG)

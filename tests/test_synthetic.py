@@ -45,7 +45,7 @@ def test_ragged_lengths_in_range():
 
 
 def test_workload_table():
-    assert len(WORKLOADS) == 5
+    assert len(WORKLOADS) == 6
     w = WORKLOADS["batch16_n100k_d128_k128_mixture_bf16"]
     assert (w.batch, w.n, w.d, w.k, w.x_kind) == (16, 100_000, 128, 128, "mixture")
 
