@@ -51,7 +51,12 @@ KERNEL_SOURCES = ["sketch_attention_compression_b200/csrc/sa_fused.cu",
                   "sketch_attention_compression_b200/csrc/sa_plan.h",
                   "sketch_attention_compression_b200/csrc/sa_ptx.cuh",
                   "sketch_attention_compression_b200/csrc/sa_internal.h"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fused_sa_batch16_n100k_d128_k128.md")
+# ncu summaries that carry the DRAM traffic of the dominant kernel, per workload
+TRAFFIC_FILES = {
+    DEFAULT_WORKLOAD: os.path.join(ROOT, "profiles", "fused_sa_batch16_n100k_d128_k128.md"),
+    "batch16_n100k_d128_k1000_mixture_bf16":
+        os.path.join(ROOT, "profiles", "fused_sa_cluster_batch16_n100k_d128_k1000.md"),
+}
 
 
 def kernel_source_hash() -> str:
@@ -71,12 +76,14 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def load_traffic():
-    """DRAM bytes per launch of the fused kernel from the committed ncu
-    summary, if it was taken on the current kernel source (else None)."""
-    if not os.path.exists(TRAFFIC_FILE):
+def load_traffic(workload: str):
+    """DRAM bytes per launch of the fused kernel on `workload` from the
+    committed ncu summary, if there is one and it was taken on the current
+    kernel source (else None)."""
+    path = TRAFFIC_FILES.get(workload)
+    if path is None or not os.path.exists(path):
         return None
-    text = open(TRAFFIC_FILE).read()
+    text = open(path).read()
     m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
     m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     if not m_hash or not m_tr or m_hash.group(1) != kernel_source_hash():
@@ -498,7 +505,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
         achieved, peak, unit = bytes_x / fused_s / 1e9, peaks["hbm_gbs"], "GB/s"
     else:
         achieved, peak, unit = flops / fused_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-    traffic = None if uq else load_traffic()  # the capture covers the shared-query pass
+    traffic = None if uq else load_traffic(args.workload)  # captures cover shared queries
     rows_total = ranks.sum(N)  # rows of all ranks' batches
     value = rows_total / (step_ms * 1e-3)
     cpu = None

@@ -53,16 +53,18 @@
 // accumulator; every CTA reads every X tile of the range (HBM once, L2 for
 // the others).  The softmax over all k prototypes of a row combines the
 // slices: each CTA computes its slice's maximum m_h and sum
-// z_h = sum_j exp2(s_j - m_h), publishes (m_h, z_h) in its own shared
-// memory and signals the other CTAs; each then reads all C pairs (in rank
-// order, so every CTA gets the same M and Z bit for bit) and scales its
-// exponentials by exp2(m_h - M) / Z, with M = max_h m_h and
-// Z = sum_h z_h exp2(m_h - M).  Each CTA sends its (m_h, z_h) of every row
-// to the others with st.async (the data and its arrival on the receiver's
-// barrier in one hop) into slots that take the place of the drain staging
-// (cluster CTAs drain straight from registers: they hold few segments); a
-// sender writes a group's slots again only after every receiver has
-// signalled that it read them (slot_free).
+// z_h = sum_j exp2(s_j - m_h), i.e. the slice's total in log2 form
+// L_h = m_h + log2 z_h, and sends L_h of every row to the other CTAs with
+// st.async (the value and its arrival on the receiver's barrier in one
+// hop).  Each CTA then takes M = max_h L_h and Z = sum_h exp2(L_h - M) over
+// all C values (in rank order, so every CTA gets the same M and Z bit for
+// bit) and scales its exponentials by exp2(m_h - M) / Z.  The values land
+// in slots that take the place of the drain staging (cluster CTAs drain
+// straight from registers: they hold few segments), double-buffered by
+// tile: a CTA sends tile u + 2 of a softmax group only after it has
+// received every CTA's tile u + 1, which each CTA sends only after it has
+// read its tile u slots, so no slot or barrier phase is overwritten early
+// and no acknowledgement has to travel back.
 //
 // Per-user queries (the SA step of a refinement layer, section 2.2 "Stacked
 // Refinement" of the notes): the one Q' buffer is reloaded per segment.
@@ -182,11 +184,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // buffers (phase s), so the drain of segment s + 1 may refill them.
   uint64_t* stage_free = drain + 2;
   uint64_t* q_empty = stage_free + 4;  // per-user queries: MMA1 is done with this segment's Q'
-  // Clusters: [group][lane quarter] the other CTAs' row statistics of this
-  // tile have arrived; [group] the other CTAs have read the ones we sent.
+  // Clusters: [group][tile parity] the other CTAs' row statistics of the
+  // tile have arrived.
   uint64_t* stats_full = q_empty + 1;
-  uint64_t* slot_free = stats_full + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(slot_free + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stats_full + 4);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   int64_t* b0_slot = reinterpret_cast<int64_t*>(tmem_slot + 2);
   volatile uint32_t* mma2_issued = tmem_slot + 4;  // tiles whose MMA2 has been issued
@@ -225,10 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&stage_free[i], 1);
-    if (CLU) {
-      for (int i = 0; i < 8; ++i) mbar_init(&stats_full[i], 1);
-      for (int i = 0; i < 2; ++i) mbar_init(&slot_free[i], 4 * (ncl - 1));
-    }
+    if (CLU)
+      for (int i = 0; i < 4; ++i) mbar_init(&stats_full[i], 1);
     *abort_flag = 0u;
     *mma2_issued = 0u;
     fence_mbar_init();
@@ -423,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int grp = (warp - 4) >> 2;       // 0: even tiles, 1: odd tiles
     const int q = warp & 3;                // TMEM lane quarter of this warp
     const int row = q * 32 + lane;         // tile row = TMEM lane of S^T
-    const uint32_t xch_a = sbase + Pl::kXch;  // clusters: received row statistics [group][src][row]
+    const uint32_t xch_a = sbase + Pl::kXch;  // clusters: [group][parity] 4 KB of row totals
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int k = k_loc;
     SegmentWalker w{a.offsets, a.batch, R0, R1, b0, off_cache, b0, n_cached};
@@ -496,54 +495,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float zl = (za + zb) + (zc + zd);
         float inv;
         if constexpr (CLU) {
-          // Send (m_h, z_h) of this row to every other CTA (slot [grp][h]
-          // of theirs, arriving on their stats_full[grp][q]) once they have
-          // all read what this group sent for its previous tile; then wait
-          // for theirs, which arrive in our slots [grp][p].
-          const uint32_t u = t >> 1;
-          if (u > 0 && !warp_wait_cluster(&slot_free[grp], (u - 1) & 1u, abort_flag, sticky)) {
-            ok = false;
-            break;
-          }
-          uint64_t* sfull = &stats_full[grp * 4 + q];
-          if (lane == 0) mbar_arrive_expect_tx(sfull, (ncl - 1) * 32 * 8);
+          // Send L_h of this row to every other CTA and wait for theirs.
+          // Each [group][parity] region holds 128 rows x 8 sources; up to
+          // 4 CTAs it is row-major (16 bytes per row: one 16-byte load
+          // gets a row's values), beyond that source-major (a warp's 32
+          // sends to one CTA then cover 128 contiguous bytes, where 32
+          // scattered sectors per send would cost more than the loads).
+          const uint32_t u = t >> 1, par = u & 1u;
+          uint64_t* sfull = &stats_full[grp * 2 + par];
+          if (q == 0 && lane == 0) mbar_arrive_expect_tx(sfull, (ncl - 1) * 128 * 4);
+          const float Lh = mx + lg2_approx(zl);
           const uint32_t sfull_a = smem_u32(sfull);
-          const uint32_t mine = xch_a + ((grp * 8 + h) * 128 + row) * 8;
+          const bool wide = ncl > 4;
+          const uint32_t region = xch_a + (grp * 2 + par) * 4096;
+          const uint32_t mine = wide ? region + h * 512 + row * 4 : region + row * 16 + h * 4;
           for (uint32_t p = 0; p < ncl; ++p)
-            if (p != h) st_async_v2f(map_to_cta(mine, p), mx, zl, map_to_cta(sfull_a, p));
-          if (!warp_wait_cluster(sfull, u & 1u, abort_flag, sticky)) {
+            if (p != h) st_async_f32(map_to_cta(mine, p), Lh, map_to_cta(sfull_a, p));
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(mine), "f"(Lh) : "memory");
+          if (!warp_wait_cluster(sfull, (u >> 1) & 1u, abort_flag, sticky)) {
             ok = false;
             break;
           }
-          float mv[kMaxCluster], zv[kMaxCluster];
+          float Lv[kMaxCluster];
+          if (wide) {
 #pragma unroll
-          for (int p = 0; p < kMaxCluster; ++p) {
-            mv[p] = -INFINITY;
-            zv[p] = 0.f;
-            if (p < static_cast<int>(ncl)) {
-              if (p == static_cast<int>(h)) {
-                mv[p] = mx;
-                zv[p] = zl;
-              } else {
-                ld_shared_v2f(xch_a + ((grp * 8 + p) * 128 + row) * 8, mv[p], zv[p]);
-              }
-            }
+            for (int p = 0; p < kMaxCluster; ++p)
+              Lv[p] = p < static_cast<int>(ncl) ? ld_shared_f32(region + p * 512 + row * 4)
+                                                : -INFINITY;
+          } else {
+            const float4 v = ld_shared_v4f(region + row * 16);
+            Lv[0] = v.x; Lv[1] = v.y; Lv[2] = v.z; Lv[3] = v.w;
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+              if (p >= static_cast<int>(ncl)) Lv[p] = -INFINITY;
+#pragma unroll
+            for (int p = 4; p < kMaxCluster; ++p) Lv[p] = -INFINITY;
           }
-          float Mx = mv[0];
+          float Mx = Lv[0];
 #pragma unroll
-          for (int p = 1; p < kMaxCluster; ++p) Mx = fmaxf(Mx, mv[p]);
+          for (int p = 1; p < kMaxCluster; ++p) Mx = fmaxf(Mx, Lv[p]);
           float Z = 0.f;
 #pragma unroll
           for (int p = 0; p < kMaxCluster; ++p)
-            if (p < static_cast<int>(ncl)) Z += zv[p] * ex2_approx(mv[p] - Mx);
-          // Every lane's loads have returned (Mx and Z are pinned as
-          // computed before the warp barrier): the senders may write
-          // these slots again.
-          asm volatile("" : "+f"(Mx), "+f"(Z));
-          __syncwarp();
-          if (lane == 0)
-            for (uint32_t p = 0; p < ncl; ++p)
-              if (p != h) mbar_arrive_remote_relaxed(map_to_cta(smem_u32(&slot_free[grp]), p));
+            if (p < static_cast<int>(ncl)) Z += ex2_approx(Lv[p] - Mx);
           inv = valid ? ex2_approx(mx - Mx) / Z : 0.f;
         } else {
           inv = valid ? 1.0f / zl : 0.f;

@@ -50,9 +50,10 @@ struct Plan {
   static_assert(kSmem <= kPlanMaxSmem, "shared memory budget");
   // Prototype-split clusters (KM = 128 per CTA) reuse the drain staging
   // (their drain stores straight from registers) for the softmax row
-  // statistics the other CTAs send: [group][source CTA (8)][row] float2.
+  // statistics the other CTAs send: [group][tile parity] regions of 128
+  // rows x 8 source CTAs, float.
   static constexpr int kXch = kDrain;
-  static_assert(2 * 8 * 128 * 8 <= 4 * kDrainBuf, "cluster exchange slots");
+  static_assert(2 * 2 * 8 * 128 * 4 <= 4 * kDrainBuf, "cluster exchange slots");
   // TMEM columns: two S^T buffers (one per softmax group), then the
   // accumulator [X~ | m] with D + 16 columns; the masses are column D.
   static constexpr uint32_t kColS = 0;

@@ -326,6 +326,12 @@ __device__ __forceinline__ float4 ld_shared_v4f(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+  float a;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(a) : "r"(addr) : "memory");
+  return a;
+}
+
 __device__ __forceinline__ void ld_shared_v2f(uint32_t addr, float& a, float& b) {
   asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(a), "=f"(b) : "r"(addr) : "memory");
 }
@@ -343,14 +349,6 @@ __device__ __forceinline__ uint32_t cluster_size() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
   return r;
-}
-
-// Arrival on an mbarrier in another CTA's shared memory (address from
-// map_to_cta), with no memory ordering of its own (a signal that carries
-// no data; data travels with st.async).
-__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar) {
-  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
-               : "memory");
 }
 
 // All threads of all CTAs of the cluster (every warp must execute it).
@@ -377,6 +375,21 @@ __device__ __forceinline__ void st_async_v2f(uint32_t remote, float a, float b,
           remote),
       "f"(a), "f"(b), "r"(remote_bar)
       : "memory");
+}
+
+// One float into another CTA's shared memory, signalled as 4 transaction
+// bytes on that CTA's mbarrier (both addresses from map_to_cta).
+__device__ __forceinline__ void st_async_f32(uint32_t remote, float a, uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(remote),
+      "f"(a), "r"(remote_bar)
+      : "memory");
+}
+
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // try_wait with cluster-scope acquire: for data that other CTAs of the

@@ -39,11 +39,11 @@ static int check() {
       bad |= take(P::box(s, b), "X" + std::to_string(s) + "." + std::to_string(b));
   // Barrier area (x_full/x_empty per stage; s_full, s_empty, acc_full,
   // drain per group; p_full, p_empty per group and slice; acc_empty,
-  // q_full; stage_free per lane quarter; q_empty) and the scheduler words
-  // (TMEM base, abort, first user, MMA2 count, pad, two range rows: ten
-  // 32-bit words) must fit the 512 bytes before the drain staging
-  // (128-byte rows).
-  const int bar_bytes = (2 * P::S + 4 * 2 + 2 * 8 + 2 + 4 + 1) * 8 + 10 * 4;
+  // q_full; stage_free per lane quarter; q_empty; the clusters'
+  // stats_full per group and tile parity) and the scheduler words (TMEM
+  // base, abort, first user, MMA2 count, pad, two range rows: ten 32-bit
+  // words) must fit the 512 bytes before the drain staging (128-byte rows).
+  const int bar_bytes = (2 * P::S + 4 * 2 + 2 * 8 + 2 + 4 + 1 + 4) * 8 + 10 * 4;
   if (bar_bytes > P::kDrain - P::kBars || P::kDrain % 128 != 0 ||
       P::kDrainRows * 128 > P::kDrainBuf) {
     std::printf("FAIL D=%d KM=%d: barrier area or drain staging\n", D, KM);
