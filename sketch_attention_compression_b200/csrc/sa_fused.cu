@@ -147,14 +147,18 @@ __device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity
 constexpr int kMaxCluster = 8;
 
 // FULL: no prototype column needs masking (k == KM, or k == KM * C for a
-// cluster).  CLU: prototype-split cluster of C CTAs (KM == 128 each).
-template <int D, int KM, bool FULL, bool CLU>
+// cluster).  CLU: prototype-split cluster of C CTAs (KM == 128 each); 0 none,
+// 1 for C <= 4 (row-major exchange slots), 2 for C > 4 (source-major).  The
+// slot layout is a template choice: a runtime branch between the two cost
+// the C = 2 pass 13 % in code generation.
+template <int D, int KM, bool FULL, int CLU>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_sa_kernel(const __grid_constant__ CUtensorMap tm_x,
                     const __grid_constant__ CUtensorMap tm_q, const PassArgs a) {
   using Pl = Plan<D, KM>;
   constexpr int S = Pl::S;
-  static_assert(!CLU || KM == 128, "clusters split the prototypes in slices of 128");
+  static_assert(CLU == 0 || KM == 128, "clusters split the prototypes in slices of 128");
+  constexpr bool kClu = CLU != 0;
 
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0u) {  // the 128-byte swizzle needs 1024-byte alignment
@@ -197,12 +201,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   // Row ranges: one per CTA, or one per cluster (whose CTAs are
   // consecutive blocks; CTA h = rank h holds prototype slice h).
-  const uint32_t ncl = CLU ? cluster_size() : 1u;
-  const uint32_t h = CLU ? cluster_rank() : 0u;
+  const uint32_t ncl = kClu ? cluster_size() : 1u;
+  const uint32_t h = kClu ? cluster_rank() : 0u;
   const int64_t G = gridDim.x / ncl;
   const int64_t c = blockIdx.x / ncl;
   const int64_t N = a.total_rows;
-  const int k_loc = CLU ? min(KM, a.k - static_cast<int>(h) * KM) : a.k;  // this CTA's prototypes
+  const int k_loc = kClu ? min(KM, a.k - static_cast<int>(h) * KM) : a.k;  // this CTA's prototypes
   uint32_t* sticky = &a.header->timeout_flags;
 
   int64_t* off_cache = reinterpret_cast<int64_t*>(smem + Pl::kOffs);
@@ -226,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&stage_free[i], 1);
-    if (CLU)
+    if (kClu)
       for (int i = 0; i < 4; ++i) mbar_init(&stats_full[i], 1);
     *abort_flag = 0u;
     *mma2_issued = 0u;
@@ -265,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   // With a cluster, the other CTAs' barriers must be initialised before
   // this CTA signals them: the cluster barrier also covers the CTA's own.
-  if (CLU) cluster_sync(); else __syncthreads();
+  if (kClu) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int64_t b0 = *b0_slot;
@@ -494,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         f2_unpack(f2_add(z2[2], z2[3]), zc, zd);
         const float zl = (za + zb) + (zc + zd);
         float inv;
-        if constexpr (CLU) {
+        if constexpr (kClu) {
           // Send L_h of this row to every other CTA and wait for theirs.
           // Each [group][parity] region holds 128 rows x 8 sources; up to
           // 4 CTAs it is row-major (16 bytes per row: one 16-byte load
@@ -506,9 +510,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (q == 0 && lane == 0) mbar_arrive_expect_tx(sfull, (ncl - 1) * 128 * 4);
           const float Lh = mx + lg2_approx(zl);
           const uint32_t sfull_a = smem_u32(sfull);
-          const bool wide = ncl > 4;
+          constexpr bool kWide = CLU == 2;
           const uint32_t region = xch_a + (grp * 2 + par) * 4096;
-          const uint32_t mine = wide ? region + h * 512 + row * 4 : region + row * 16 + h * 4;
+          const uint32_t mine = kWide ? region + h * 512 + row * 4 : region + row * 16 + h * 4;
           for (uint32_t p = 0; p < ncl; ++p)
             if (p != h) st_async_f32(map_to_cta(mine, p), Lh, map_to_cta(sfull_a, p));
           asm volatile("st.shared.f32 [%0], %1;" ::"r"(mine), "f"(Lh) : "memory");
@@ -517,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           float Lv[kMaxCluster];
-          if (wide) {
+          if constexpr (kWide) {
 #pragma unroll
             for (int p = 0; p < kMaxCluster; ++p)
               Lv[p] = p < static_cast<int>(ncl) ? ld_shared_f32(region + p * 512 + row * 4)
@@ -600,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int j0 = KM == 128 ? q * 32 : q * 16;
           const int j = j0 + lane;
           const bool has = (KM == 128 ? true : lane < 16) && j < k;
-          if (!CLU && seg > 0 && !warp_wait(&stage_free[q], (seg - 1) & 1u, abort_flag, sticky)) {
+          if (!kClu && seg > 0 && !warp_wait(&stage_free[q], (seg - 1) & 1u, abort_flag, sticky)) {
             ok = false;
             break;
           }
@@ -632,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_fence_before();
               warp_arrive(acc_empty, lane);
             }
-            if constexpr (CLU) {
+            if constexpr (kClu) {
               // Straight from registers: lane j writes its row's columns.
               if (has) {
 #pragma unroll
@@ -673,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           __syncwarp();
-          if (!CLU && lane == 0) mbar_arrive(&stage_free[q]);
+          if (!kClu && lane == 0) mbar_arrive(&stage_free[q]);
           if (has) dm[j] = __uint_as_float(mv);
         }
       }
@@ -709,13 +713,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // No CTA of a cluster leaves while another may still read its published
   // statistics or signal its barriers.
-  if (CLU) cluster_sync();
+  if (kClu) cluster_sync();
 }
 
 template <int D, int KM>
 cudaError_t launch_one(const CUtensorMap& tx, const CUtensorMap& tq, const PassArgs& a,
                        int grid, cudaStream_t stream) {
-  auto kern = a.k == KM ? fused_sa_kernel<D, KM, true, false> : fused_sa_kernel<D, KM, false, false>;
+  auto kern = a.k == KM ? fused_sa_kernel<D, KM, true, 0> : fused_sa_kernel<D, KM, false, 0>;
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Plan<D, KM>::kSmem);
   if (err != cudaSuccess) return err;
@@ -755,8 +759,9 @@ cudaLaunchConfig_t cluster_config(int ranges, int ncl, cudaStream_t stream,
 template <int D>
 cudaError_t launch_cluster(const CUtensorMap& tx, const CUtensorMap& tq, const PassArgs& a,
                            int ranges, int ncl, cudaStream_t stream) {
-  auto kern = a.k == 128 * ncl ? fused_sa_kernel<D, 128, true, true>
-                               : fused_sa_kernel<D, 128, false, true>;
+  const bool full = a.k == 128 * ncl;
+  auto kern = ncl > 4 ? (full ? fused_sa_kernel<D, 128, true, 2> : fused_sa_kernel<D, 128, false, 2>)
+                      : (full ? fused_sa_kernel<D, 128, true, 1> : fused_sa_kernel<D, 128, false, 1>);
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Plan<D, 128>::kSmem);
   if (err != cudaSuccess) return err;
@@ -767,7 +772,7 @@ cudaError_t launch_cluster(const CUtensorMap& tx, const CUtensorMap& tq, const P
 
 template <int D>
 int cluster_capacity(int ncl) {
-  auto kern = fused_sa_kernel<D, 128, false, true>;
+  auto kern = ncl > 4 ? fused_sa_kernel<D, 128, false, 2> : fused_sa_kernel<D, 128, false, 1>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Plan<D, 128>::kSmem) != cudaSuccess)
     return 0;

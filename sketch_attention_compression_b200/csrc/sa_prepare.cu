@@ -78,62 +78,76 @@ __global__ void prepare_query_kernel(const void* __restrict__ P, const void* __r
 // fp32 multiply-adds in f order.  Rows j in [k, k_rows) are zero (the
 // padded prototypes of the bf16 copy).  A CTA of 256 threads computes 32
 // rows x 64 columns: thread (ty, tx) owns rows 2ty, 2ty+1 and columns
-// 4tx..4tx+3; Q and M pass through shared memory in 32-wide slices of f.
-constexpr int kUqRows = 32, kUqCols = 64, kUqF = 32;
+// 4tx..4tx+3.  Its 32 rows of Q and 64 columns of M (all d of f) are
+// staged in shared memory in one step, so the CTA waits for global memory
+// once.
+constexpr int kUqRows = 32, kUqCols = 64;
+
+size_t user_query_smem(int d) {
+  return (static_cast<size_t>(kUqRows) * (d + 1) + static_cast<size_t>(d) * kUqCols) *
+         sizeof(float);
+}
 
 __global__ void __launch_bounds__(256)
     user_query_kernel(const float* __restrict__ Q, const float* __restrict__ M, int64_t B, int k,
                       int k_rows, int d, float* __restrict__ out_f32,
                       uint16_t* __restrict__ out_bf16) {
-  __shared__ float qs[kUqRows][kUqF + 1];
-  __shared__ float ms[kUqF][kUqCols];
+  extern __shared__ float uq_sh[];
+  float* qs = uq_sh;                            // [32][d + 1]
+  float* ms = uq_sh + kUqRows * (d + 1);        // [d][64]
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kUqRows;
   const int col0 = blockIdx.y * kUqCols;
   const int64_t total = B * k_rows;
-  // The pass that reads Q' may start its set-up now (it waits for this
-  // grid's completion before reading anything).
+  // Launched as a programmatic dependent of the stream's previous kernel
+  // (for back-to-back calls, the previous call's finalize, which already
+  // waited for the fused pass that read the old Q'_b): nothing is read or
+  // written before that kernel has completed.  The pass that reads Q'_b may
+  // then start its own set-up (it waits for this grid before reading).
+  grid_dependency_wait();
   grid_dependency_launch();
+  for (int i = tid; i < kUqRows * d; i += 256) {
+    const int rr = i / d, ff = i - rr * d;
+    const int64_t R = row0 + rr;
+    float v = 0.f;
+    if (R < total) {
+      const int64_t b = R / k_rows;
+      const int j = static_cast<int>(R - b * k_rows);
+      if (j < k) v = Q[(b * k + j) * d + ff];
+    }
+    qs[rr * (d + 1) + ff] = v;
+  }
+  for (int i = tid; i < d * kUqCols; i += 256) {
+    const int ff = i / kUqCols, cc = i % kUqCols;
+    ms[i] = M[static_cast<int64_t>(ff) * d + col0 + cc];
+  }
+  __syncthreads();
   float acc[2][4] = {};
-  for (int f0 = 0; f0 < d; f0 += kUqF) {
-    for (int i = tid; i < kUqRows * kUqF; i += 256) {
-      const int rr = i / kUqF, ff = i % kUqF;
-      const int64_t R = row0 + rr;
-      float v = 0.f;
-      if (R < total) {
-        const int64_t b = R / k_rows;
-        const int j = static_cast<int>(R - b * k_rows);
-        if (j < k) v = Q[(b * k + j) * d + f0 + ff];
-      }
-      qs[rr][ff] = v;
-    }
-    for (int i = tid; i < kUqF * kUqCols; i += 256) {
-      const int ff = i / kUqCols, cc = i % kUqCols;
-      ms[ff][cc] = M[static_cast<int64_t>(f0 + ff) * d + col0 + cc];
-    }
-    __syncthreads();
+  const float* q0p = qs + (2 * ty) * (d + 1);
+  const float* q1p = q0p + (d + 1);
 #pragma unroll 8
-    for (int ff = 0; ff < kUqF; ++ff) {
-      const float q0 = qs[2 * ty][ff], q1 = qs[2 * ty + 1][ff];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float mv = ms[ff][4 * tx + u];
-        acc[0][u] = fmaf(q0, mv, acc[0][u]);
-        acc[1][u] = fmaf(q1, mv, acc[1][u]);
-      }
-    }
-    __syncthreads();
+  for (int ff = 0; ff < d; ++ff) {
+    const float q0 = q0p[ff], q1 = q1p[ff];
+    const float4 mv = *reinterpret_cast<const float4*>(ms + ff * kUqCols + 4 * tx);
+    acc[0][0] = fmaf(q0, mv.x, acc[0][0]);
+    acc[0][1] = fmaf(q0, mv.y, acc[0][1]);
+    acc[0][2] = fmaf(q0, mv.z, acc[0][2]);
+    acc[0][3] = fmaf(q0, mv.w, acc[0][3]);
+    acc[1][0] = fmaf(q1, mv.x, acc[1][0]);
+    acc[1][1] = fmaf(q1, mv.y, acc[1][1]);
+    acc[1][2] = fmaf(q1, mv.z, acc[1][2]);
+    acc[1][3] = fmaf(q1, mv.w, acc[1][3]);
   }
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int64_t R = row0 + 2 * ty + h;
+  for (int hh = 0; hh < 2; ++hh) {
+    const int64_t R = row0 + 2 * ty + hh;
     if (R >= total) continue;
     const int64_t o = R * d + col0 + 4 * tx;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      if (out_f32 != nullptr) out_f32[o + u] = acc[h][u];
-      if (out_bf16 != nullptr) out_bf16[o + u] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[h][u]));
+      if (out_f32 != nullptr) out_f32[o + u] = acc[hh][u];
+      if (out_bf16 != nullptr) out_bf16[o + u] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[hh][u]));
     }
   }
 }
@@ -147,8 +161,23 @@ cudaError_t launch_user_query(const float* queries, const float* M, int64_t batc
   if (rows <= 0) return cudaSuccess;
   const dim3 grid(static_cast<unsigned>((rows + kUqRows - 1) / kUqRows),
                   static_cast<unsigned>(d / kUqCols));
-  user_query_kernel<<<grid, 256, 0, stream>>>(queries, M, batch, k, k_rows, d, out_f32, out_bf16);
-  return cudaGetLastError();
+  const size_t smem = user_query_smem(d);
+  cudaError_t err = cudaFuncSetAttribute(user_query_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, user_query_kernel, queries, M, batch, k, k_rows, d, out_f32,
+                            out_bf16);
 }
 
 cudaError_t launch_prepare_projection(const void* W_Q, const void* W_K, int d, double scale,
