@@ -255,6 +255,24 @@ sa_status sa_sketch_forward_noalloc(sa_query q, const void* X, const int64_t* of
                                     int64_t batch, int64_t total_rows, float* X_tilde,
                                     float* mass, uint32_t* device_flags_out, void* stream);
 
+/*
+ * sa_mass_normalise -- the mass-normalised sketch X~_bj / m_bj (0 where
+ * m_bj == 0), the weighted mean of user b's rows under prototype j (section
+ * 2.1: the sketch is a weighted aggregation; its masses make it a mean),
+ * e.g. as the query of the next refinement layer (section 2.2).
+ *
+ *   X_tilde  device, batch x k x d fp32 (16-byte aligned), as written by
+ *            sa_sketch_forward
+ *   mass     device, batch x k fp32
+ *   batch    B >= 0;  k >= 1;  d >= 4, a multiple of 4
+ *   out      device, batch x k x d fp32 (16-byte aligned); may be X_tilde
+ *   stream   the kernel is enqueued here
+ *
+ * Returns SA_ERR_INVALID_ARG for bad sizes, null pointers or misalignment.
+ */
+sa_status sa_mass_normalise(const float* X_tilde, const float* mass, int64_t batch, int k, int d,
+                            float* out, void* stream);
+
 /* Static description of a status code. */
 const char* sa_status_string(sa_status s);
 

@@ -12,5 +12,6 @@ from .binding import (  # noqa: F401
     SAError,
     SketchQuery,
     load_library,
+    mass_normalise,
     read_device_status,
 )

@@ -41,6 +41,7 @@ SIGNATURES = {
     "sa_sketch_forward_host": (_i32, _FWD_ARGS),
     "sa_sketch_forward_noalloc": (_i32, [_vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp]),
     "sa_read_device_status": (_i32, [_vp, _sz, _vp, ctypes.POINTER(ctypes.c_uint32)]),
+    "sa_mass_normalise": (_i32, [_vp, _vp, _i64, _i32, _i32, _vp, _vp]),
     "sa_status_string": (ctypes.c_char_p, [_i32]),
     "sa_query_info": (_i32, [_vp, ctypes.POINTER(_i32), ctypes.POINTER(_i32),
                              ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
@@ -304,6 +305,25 @@ class SketchQuery:
             self.close()
         except Exception:
             pass
+
+
+def mass_normalise(X_tilde, mass, out=None, stream=None):
+    """X~_bj / m_bj (0 where m_bj == 0) for fp32 CUDA tensors X~ (B, k, d)
+    and m (B, k); ``out`` may be X_tilde (in place)."""
+    torch = _torch()
+    lib = load_library()
+    if X_tilde.dtype != torch.float32 or mass.dtype != torch.float32 or X_tilde.dim() != 3:
+        raise TypeError("X_tilde (B, k, d) and mass (B, k) must be float32")
+    B, k, d = (int(x) for x in X_tilde.shape)
+    if tuple(mass.shape) != (B, k):
+        raise ValueError("mass must be (B, k)")
+    if out is None:
+        out = torch.empty_like(X_tilde)
+    if B > 0:
+        _check(lib.sa_mass_normalise(_dev_ptr(X_tilde, "X_tilde"), _dev_ptr(mass, "mass"), B, k, d,
+                                     _dev_ptr(out, "out"), ctypes.c_void_p(_stream_handle(stream))),
+               "sa_mass_normalise")
+    return out
 
 
 def read_device_status(workspace, stream=None) -> int:

@@ -104,15 +104,14 @@ def test_two_stacked_layers(dtype):
     # sketch normalised by its masses (X~_j / m_j); each side runs its own
     # chain and the final sketches are compared.
     import torch
-    from sketch_attention_compression_b200 import SketchQuery
+    from sketch_attention_compression_b200 import SketchQuery, mass_normalise
     lens = [3000, 129, 0, 5000, 64]
     d, k = 128, 64
     inp = make_inputs(lens, d=d, k=k, dtype=dtype, seed=34)
     dev = to_device(inp)
     q = SketchQuery(dev["P"], dev["W_Q"], dev["W_K"], inp["scale"])
     Xt1, m1 = q.forward(dev["X"], dev["offsets"])
-    Q2 = torch.where(m1[..., None] > 0, Xt1 / m1[..., None].clamp_min(1e-30),
-                     torch.zeros_like(Xt1)).contiguous()
+    Q2 = mass_normalise(Xt1, m1)
     Xt2, m2 = q.forward_user_queries(Q2, dev["X"], dev["offsets"])
     torch.cuda.synchronize()
     Xt_g, m_g = Xt2.double().cpu().numpy(), m2.double().cpu().numpy()
@@ -158,4 +157,31 @@ def test_errors():
         ctypes.c_void_p(m.data_ptr()), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
         ctypes.c_void_p(0))
     assert st == binding.SA_ERR_INVALID_ARG
+    q.close()
+
+
+def test_mass_normalise():
+    # X~_j / m_j against the oracle's mass_normalised, 0 for the empty
+    # user's rows; in place gives the same bits.
+    import torch
+    from sketch_attention_compression_b200 import SketchQuery, mass_normalise
+    lens = [700, 0, 1, 2500]
+    inp = make_inputs(lens, d=128, k=100, dtype="bf16", seed=37)
+    dev = to_device(inp)
+    q = SketchQuery(dev["P"], dev["W_Q"], dev["W_K"], inp["scale"])
+    Xt, m = q.forward(dev["X"], dev["offsets"])
+    out = mass_normalise(Xt, m)
+    torch.cuda.synchronize()
+    Xn = out.double().cpu().numpy()
+    Xt_o, m_o = sa_batch(inp["X"], inp["offsets"], inp["P"], inp["W_Q"], inp["W_K"], inp["scale"])
+    for b in range(len(lens)):
+        ref = mass_normalised(Xt_o[b], m_o[b])
+        assert np.max(np.abs(Xn[b] - ref)) <= 2e-2 * max(np.max(np.abs(ref)), 1e-30), f"user {b}"
+    assert np.all(Xn[1] == 0)
+    # the kernel divides the library's own X~ by its own m: compare with fp32 division
+    want = torch.where(m[..., None] > 0, Xt / m[..., None], torch.zeros_like(Xt))
+    assert torch.equal(out, want)
+    Xt2 = Xt.clone()
+    mass_normalise(Xt2, m, out=Xt2)
+    assert torch.equal(Xt2, out)
     q.close()
