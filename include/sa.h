@@ -156,8 +156,8 @@ sa_status sa_sketch_forward(sa_query q, const void* X, const int64_t* offsets, i
  *   workspace   device, >= sa_workspace_bytes_user_queries(q, B, N) bytes,
  *               256-byte aligned; one call at a time
  *
- * Returns SA_ERR_UNSUPPORTED for queries run on pairs of CTAs (bf16, d = 256,
- * k > 64; the clusters of d = 64 and 128 take per-user queries), SA_ERR_INVALID_ARG if queries is NULL with B > 0 or if B * k_pad
+ * Every query shape that sa_sketch_forward runs takes per-user queries.
+ * Returns SA_ERR_INVALID_ARG if queries is NULL with B > 0 or if B * k_pad
  * reaches 2^31 (k_pad as sa_query_info reports), otherwise as
  * sa_sketch_forward.  An empty user gets X~ = 0 and m = 0 whatever its Q_b.
  */

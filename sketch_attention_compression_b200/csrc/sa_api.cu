@@ -126,9 +126,7 @@ sa_status run(sa_query q, const float* queries, const void* X, const int64_t* of
   if (!same_device(q)) return SA_ERR_INVALID_ARG;
   const bool user_q = queries != nullptr;
   if (user_q) {
-    // The two-CTA pass (d = 256, k > 64) keeps its one Q' per CTA half; and
-    // the tensor map's row coordinate b * k_pad is a 32-bit integer.
-    if (q->dtype == SA_BF16 && q->d == 256 && q->k_pad == 256) return SA_ERR_UNSUPPORTED;
+    // The tensor map's row coordinate b * k_pad is a 32-bit integer.
     if (batch > (int64_t{1} << 31) / (q->k_pad > 0 ? q->k_pad : 1) - 1) return SA_ERR_INVALID_ARG;
   }
   const WsLayout l = ws_layout(q, total_rows);
@@ -164,7 +162,7 @@ sa_status run(sa_query q, const float* queries, const void* X, const int64_t* of
       CUtensorMap tmq;
       if (user_q && !make_tmap_bf16(&tmq, uq, static_cast<uint64_t>(batch) * q->k_pad,
                                     static_cast<uint64_t>(q->d),
-                                    static_cast<uint32_t>(q->ncl > 1 ? 128 : q->k_pad)))
+                                    static_cast<uint32_t>(q->k_pad > 128 ? 128 : q->k_pad)))
         return SA_ERR_CUDA;
       CUtensorMap tmx;
       // A zero-row tensor map is not encodable; with N == 0 the kernel
@@ -177,7 +175,8 @@ sa_status run(sa_query q, const float* queries, const void* X, const int64_t* of
       if (!ok) return SA_ERR_CUDA;
       const CUtensorMap& tq = user_q ? tmq : q->tmap_q;
       err = q->ncl > 1 ? sa::launch_fused_bf16_cluster(tmx, tq, a, G, q->ncl, st)
-            : q->k_pad == 256 ? sa::launch_fused_bf16_pair(tmx, q->tmap_q_half, a, G, st)
+            : q->k_pad == 256 ? sa::launch_fused_bf16_pair(tmx, user_q ? tmq : q->tmap_q_half, a,
+                                                           G, st)
                               : sa::launch_fused_bf16(tmx, tq, q->k_pad, a, G, st);
     } else {
       err = sa::launch_simt_fp32(user_q ? static_cast<const float*>(uq) : q->q_f32,

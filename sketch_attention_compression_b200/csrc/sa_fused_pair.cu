@@ -85,7 +85,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   uint64_t* q_full = acc_empty + 1;
   uint64_t* drain = q_full + 1;          // [2 issuers]
   uint64_t* xch = drain + 2;             // [2 tile parities]: the other half's (m, z) arrived
-  float2* xslot = reinterpret_cast<float2*>(xch + 2);  // [2 tile parities][128 rows]
+  uint64_t* q_empty = xch + 2;           // per-user queries: MMA1 is done with this segment's Q'
+  float2* xslot = reinterpret_cast<float2*>(q_empty + 2);  // [2 tile parities][128 rows]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xslot + 256);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   int64_t* b0_slot = reinterpret_cast<int64_t*>(tmem_slot + 2);
@@ -113,6 +114,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
     mbar_init(acc_empty, 4);
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     *abort_flag = 0u;
     int64_t b0u;
     const int64_t r0 = range_begin(a.offsets, a.batch, N, c, G, &b0u);
@@ -142,6 +144,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   tc_fence_after();
 
   uint32_t tiles_issued = 0;  // producer thread: X tiles whose TMA copy was issued
+  uint32_t q_loads = 0;       // Q' loader thread (per-user queries): Q'_b copies issued
+  const bool user_q = a.user_queries != 0;
   if (aligned) {
     const uint32_t tmem = *tmem_slot;
     const int64_t b0 = *b0_slot;
@@ -151,10 +155,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       if (lane == 0) {
         // Both CTAs of the pair read every tile; the default L2 policy keeps
         // a tile for the second reader.
-        mbar_arrive_expect_tx(q_full, 128 * D * 2);
+        if (!user_q) {
+          mbar_arrive_expect_tx(q_full, 128 * D * 2);
 #pragma unroll
-        for (int cb = 0; cb < D / 64; ++cb)
-          tma_load_2d(smem + cb * kB, &tm_qh, q_full, cb * 64, static_cast<int32_t>(128 * h));
+          for (int cb = 0; cb < D / 64; ++cb)
+            tma_load_2d(smem + cb * kB, &tm_qh, q_full, cb * 64, static_cast<int32_t>(128 * h));
+        }
         TileCursor cur{SegmentWalker{a.offsets, a.batch, R0, R1, b0}};
         int64_t r;
         uint32_t t = 0;
@@ -170,6 +176,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
         tiles_issued = t;
       }
+    } else if (warp == 2) {
+      // ---------------------------------------------------------- Q'_b loader
+      // Per-user queries: segment g's half of Q'_b (rows (2 user + h) 128..
+      // of the per-call array, 256 padded prototypes per user) once MMA1 has
+      // finished segment g - 1 with the previous one.
+      if (lane == 0 && user_q) {
+        SegmentWalker w{a.offsets, a.batch, R0, R1, b0};
+        int64_t user, s, e, lo, hi;
+        uint32_t g = 0;
+        while (w.next(user, s, e, lo, hi)) {
+          if (g > 0 && !mbar_wait(q_empty, (g - 1) & 1u, abort_flag, sticky)) break;
+          mbar_arrive_expect_tx(q_full, 128 * D * 2);
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb)
+            tma_load_2d(smem + cb * kB, &tm_qh, q_full, cb * 64,
+                        static_cast<int32_t>((2 * user + h) * 128));
+          ++g;
+        }
+        q_loads = g;
+      }
     } else if (warp == 1 || warp == 3) {
       // ---------------------------------------------------------- MMA issuers
       if (lane == 0) {
@@ -179,7 +205,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         constexpr uint32_t idesc_s = idesc_bf16_f32(kTileRows, 128, 0, 0);
         constexpr uint32_t idesc_x0 = idesc_bf16_f32(128, 128, 1, 1);
         constexpr uint32_t idesc_x1 = idesc_bf16_f32(128, 144, 1, 1);
-        bool ok = role == 1 || mbar_wait(q_full, 0, abort_flag, sticky);
+        bool ok = true;
         SegmentWalker w{a.offsets, a.batch, R0, R1, b0};
         int64_t user, s, e, lo, hi;
         uint32_t t = 0, seg = 0;
@@ -187,7 +213,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           for (int64_t r = s; r < e; r += kTileRows, ++t) {
             const int st = t % S;
             if (role == 0) {
-              if (!mbar_wait(&x_full[st], (t / S) & 1u, abort_flag, sticky) ||
+              // Q' of this segment: loaded once (phase 0) for shared
+              // queries, phase seg of the per-user reloads otherwise.
+              if ((r == s && !mbar_wait(q_full, user_q ? (seg & 1u) : 0u, abort_flag, sticky)) ||
+                  !mbar_wait(&x_full[st], (t / S) & 1u, abort_flag, sticky) ||
                   !mbar_wait(s_empty, (t & 1u) ^ 1u, abort_flag, sticky)) {
                 ok = false;
                 break;
@@ -200,6 +229,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                             base_k + (((ks >> 2) * kB + (ks & 3) * 32) >> 4), idesc_s,
                             ks > 0 ? 1u : 0u);
               mma_commit(s_full);
+              if (user_q && r + kTileRows >= e) mma_commit(q_empty);
             } else {
               const bool first = (r == s);
               const bool last = (r + kTileRows >= e);
@@ -408,8 +438,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const uint32_t t = tiles_issued;
       for (uint32_t u = (t > static_cast<uint32_t>(S) ? t - S : 0u); u < t; ++u)
         mbar_wait_bounded(&x_full[u % S], (u / S) & 1u);
-      mbar_wait_bounded(q_full, 0);
+      if (!user_q) mbar_wait_bounded(q_full, 0);
     }
+    if (warp == 2 && lane == 0 && q_loads > 0) mbar_wait_bounded(q_full, (q_loads - 1) & 1u);
     if ((warp == 1 || warp == 3) && lane == 0) {
       const int role = warp == 1 ? 0 : 1;
       mma_commit(&drain[role]);
