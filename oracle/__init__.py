@@ -19,3 +19,4 @@ from .sa_oracle import (  # noqa: F401
     sa_user,
 )
 from .brute import sa_user_bruteforce  # noqa: F401
+from .sa_backward import sa_batch_backward, sa_user_backward  # noqa: F401
