@@ -154,3 +154,25 @@ def test_a_planted_mistake_trips_a_pin(kind):
         except AssertionError:
             tripped += 1
     assert tripped >= 1
+
+
+def test_q_prime_form_of_the_gradients():
+    # The form a fused backward pass computes (S = X Q'^T with
+    # Q' = P W_Q W_K^T scale, and the per-user accumulator R = dS X):
+    #   dX = A^T G + dS^T Q',  dP = scale R W_K W_Q^T,
+    #   dW_Q = scale P^T R W_K,  dW_K = scale R^T P W_Q
+    # equals the oracle's chain rule through K = X W_K and Q = P W_Q.
+    c = _case(11, n=9, k=5, d=6)
+    X, P, WQ, WK, sc, G, g = (c[key] for key in ("Xb", "P", "W_Q", "W_K", "scale", "G", "g"))
+    Qp = P @ WQ @ WK.T * sc
+    S = Qp @ X.T
+    E = np.exp(S - S.max(axis=0, keepdims=True))
+    A = E / E.sum(axis=0, keepdims=True)
+    dA = G @ X.T + g[:, None]
+    dS = A * (dA - (A * dA).sum(axis=0, keepdims=True))
+    R = dS @ X
+    r = sa_user_backward(X, P, WQ, WK, sc, G, g)
+    np.testing.assert_allclose(A.T @ G + dS.T @ Qp, r["dX"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sc * R @ WK @ WQ.T, r["dP"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sc * P.T @ R @ WK, r["dW_Q"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sc * R.T @ P @ WQ, r["dW_K"], rtol=1e-12, atol=1e-12)
