@@ -1,0 +1,154 @@
+"""Model check of the clusters' softmax exchange (host-side simulation).
+
+The prototype-split cluster pass (more than 128 prototypes; section 2.2 of
+the SequenceO1 reading notes puts the final layers at about a thousand)
+combines each row's softmax over C CTAs.  Every CTA sends its slice total of
+tile u to every other CTA with st.async: the value lands in the receiver's
+slot [group][u & 1][sender] and adds its bytes to the receiver's barrier
+[group][u & 1]; the receiver arms that barrier once per tile (one arrival
+plus the expected bytes), waits for the phase to complete, then reads the
+slots.  No acknowledgement travels back: the argument is that a CTA can only
+send tile u + 2 of a group after it received every CTA's tile u + 1, which
+each CTA sends only after reading its own tile u slots.
+
+This test runs that protocol on a model of the mbarrier (pending arrivals,
+transaction bytes that may arrive before or after the arming, phase parity)
+with arbitrary interleavings and arbitrary delivery delays, and checks that
+  * every read sees the values of its own tile from every sender;
+  * no value lands in a slot that still holds an unread value;
+  * no barrier phase completes on bytes of another tile;
+  * no wait finds its barrier two phases ahead (the hardware waits on the
+    phase parity);
+  * nothing deadlocks (every CTA finishes every tile).
+A variant with one buffer per group in place of two (single-buffered slots)
+must fail, which shows the check can catch the hazard the double buffering
+avoids."""
+
+import random
+
+import pytest
+
+
+class Barrier:
+    """mbarrier: a phase completes when its pending arrivals reach 0 and its
+    transaction count is back to 0."""
+
+    def __init__(self, count):
+        self.count = count
+        self.pending = count
+        self.tx = 0
+        self.phase = 0          # completed phases
+        self.tiles = set()      # tiles whose bytes were counted in this phase
+
+    def _maybe_complete(self):
+        if self.pending == 0 and self.tx == 0:
+            self.phase += 1
+            self.pending = self.count
+            done = self.tiles
+            self.tiles = set()
+            return done
+        return None
+
+    def arrive_expect(self, nbytes, tile):
+        self.tx += nbytes
+        self.pending -= 1
+        self.tiles.add(tile)
+        return self._maybe_complete()
+
+    def complete_tx(self, nbytes, tile):
+        self.tx -= nbytes
+        self.tiles.add(tile)
+        return self._maybe_complete()
+
+
+def simulate(C, tiles, seed, buffers=2, warps=4):
+    """C CTAs x 2 softmax groups x `warps` warps.  Every warp sends its rows
+    of each tile to the other CTAs (one unit per warp and receiver); warp 0
+    of a group arms the group's barrier for the tile with the units of all
+    warps of all senders; every warp waits on the barrier, then reads the
+    slots of its own rows."""
+    rng = random.Random(seed)
+    groups = 2
+    bars = [[[Barrier(1) for _ in range(buffers)] for _ in range(groups)] for _ in range(C)]
+    # slots[CTA][group][buf][sender][warp] = (tile, read?)
+    slots = [[[[[None] * warps for _ in range(C)] for _ in range(buffers)] for _ in range(groups)]
+             for _ in range(C)]
+    # each (CTA, group, warp) walks its tiles u = g, g + 2, ... (local v = u // 2)
+    step = {(h, g, w): ("send", g) for h in range(C) for g in range(groups) for w in range(warps)}
+    in_flight = []  # (receiver, group, buf, sender, warp, tile)
+    errors = []
+
+    def on_complete(done, h, g, b, u_expected):
+        if done is not None and done != {u_expected}:
+            errors.append(f"CTA {h} group {g} buf {b}: phase completed on tiles {done}")
+
+    guard = 0
+    while True:
+        guard += 1
+        if guard > 400000:
+            errors.append("no progress (deadlock)")
+            break
+        actors = [key for key, (st, u) in step.items() if u < tiles]
+        if not actors and not in_flight:
+            break
+        choices = [("cta", a) for a in actors] + [("deliver", i) for i in range(len(in_flight))]
+        kind, what = rng.choice(choices)
+        if kind == "deliver":
+            recv, g, b, sender, w, tile = in_flight.pop(what)
+            cell = slots[recv][g][b][sender][w]
+            if cell is not None and not cell[1]:
+                errors.append(f"CTA {recv}: slot [{g}][{b}][{sender}][{w}] overwritten by tile "
+                              f"{tile} before tile {cell[0]} was read")
+            slots[recv][g][b][sender][w] = (tile, False)
+            on_complete(bars[recv][g][b].complete_tx(1, tile), recv, g, b, tile)
+            continue
+        h, g, w = what
+        st, u = step[what]
+        v = u // 2
+        par = v % buffers
+        if st == "send":
+            if w == 0:
+                on_complete(bars[h][g][par].arrive_expect((C - 1) * warps, u), h, g, par, u)
+            for p in range(C):
+                if p != h:
+                    in_flight.append((p, g, par, h, w, u))
+            step[what] = ("wait", u)
+        elif st == "wait":
+            # the phase for local tile v is phase number v // buffers of the
+            # barrier; the hardware waits on its parity, so the barrier must
+            # never be two phases past it when the wait runs
+            want = v // buffers
+            if bars[h][g][par].phase > want + 1:
+                errors.append(f"CTA {h} group {g} warp {w} tile {u}: barrier two phases ahead")
+            if bars[h][g][par].phase > want:
+                for p in range(C):
+                    if p == h:
+                        continue
+                    cell = slots[h][g][par][p][w]
+                    if cell is None or cell[0] != u:
+                        errors.append(f"CTA {h} group {g} warp {w} tile {u}: slot from {p} "
+                                      f"holds {cell}")
+                    else:
+                        slots[h][g][par][p][w] = (u, True)
+                step[what] = ("send", u + 2)
+        if errors:
+            break
+    return errors
+
+
+@pytest.mark.parametrize("C", [2, 3, 4, 8])
+def test_double_buffered_exchange_is_safe(C):
+    for seed in range(40 if C < 8 else 15):
+        errs = simulate(C, tiles=14, seed=seed)
+        assert not errs, f"C={C} seed={seed}: {errs[:3]}"
+
+
+def test_single_buffered_exchange_is_caught():
+    # With one slot set and one barrier per group, a fast CTA's next tile
+    # can land before a slow CTA has read the current one.
+    found = False
+    for seed in range(200):
+        if simulate(4, tiles=12, seed=seed, buffers=1):
+            found = True
+            break
+    assert found
