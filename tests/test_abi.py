@@ -82,3 +82,62 @@ def test_host_path_rejects_bad_offsets_before_any_copy(lib):
     offs = (ctypes.c_int64 * 3)(0, 5, 3)
     assert lib.sa_sketch_forward_host(None, None, offs, 2, 3, None, None, None, 0, None) == \
         binding.SA_ERR_INVALID_ARG
+
+
+def declared_signatures():
+    """name -> (return type, [parameter types]) parsed from include/sa.h."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"#[^\n]*", "", text)
+    out = {}
+    for m in re.finditer(r"([A-Za-z_][\w \*]*?)\b(sa_[a-z_]+)\s*\(([^;{]*?)\)\s*;", text):
+        ret, name, params = m.group(1).strip(), m.group(2), m.group(3).strip()
+        plist = [] if params in ("", "void") else [p.strip() for p in params.split(",")]
+        out[name] = (ret, plist)
+    return out
+
+
+def _kind(ctype_decl):
+    """Coarse class of a C parameter or return type: pointer, 64-bit integer,
+    32-bit integer/enum, float, size_t or void."""
+    t = " ".join(ctype_decl.replace("*", " * ").split())
+    if "*" in t or t.startswith("sa_query"):
+        return "ptr"
+    if "int64_t" in t:
+        return "i64"
+    if "size_t" in t:
+        return "size"
+    if "float" in t:
+        return "f32"
+    if t == "void":
+        return "void"
+    return "i32"  # int, sa_dtype, sa_status
+
+
+def _ctypes_kind(ct):
+    if ct is None:
+        return "void"
+    if ct in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(ct, "_type_") and ct.__name__.startswith("LP_"):
+        return "ptr"
+    if ct is ctypes.c_int64:
+        return "i64"
+    if ct is ctypes.c_size_t:
+        return "size"
+    if ct is ctypes.c_float:
+        return "f32"
+    return "i32"
+
+
+def test_binding_signatures_match_header():
+    """Every ctypes declaration has the header's parameter count and, class
+    by class (pointer, int64, size_t, float, 32-bit int), its types."""
+    decl = declared_signatures()
+    assert sorted(decl) == declared_functions()
+    for name, (ret, params) in decl.items():
+        res, args = binding.SIGNATURES[name]
+        # names of parameters are stripped: keep the type part of "type name"
+        ptypes = [p.rsplit(" ", 1)[0] if not p.endswith("*") else p for p in params]
+        got = [_ctypes_kind(a) for a in args]
+        want = [_kind(p) for p in ptypes]
+        assert got == want, f"{name}: binding {got} vs header {want}"
+        assert _ctypes_kind(res) == _kind(ret), f"{name}: return {res} vs {ret}"
