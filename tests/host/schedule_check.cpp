@@ -137,9 +137,12 @@ static int check(const std::vector<int64_t>& off, int64_t sms) {
 int main() {
   std::mt19937_64 rng(12345);
   long long cases = 0;
-  const int64_t sms_list[] = {1, 2, 3, 7, 148};
-  for (int iter = 0; iter < 3000; ++iter) {
-    const int64_t sms = sms_list[iter % 5];
+  // Range counts: tiny grids, one per SM (148), and the cluster passes' counts on a
+  // B200 (74 pairs, 45 clusters of 3, 33 of 4, 15 of 8).
+  const int64_t sms_list[] = {1, 2, 3, 7, 15, 33, 45, 74, 148};
+  const int n_sms = static_cast<int>(sizeof(sms_list) / sizeof(sms_list[0]));
+  for (int iter = 0; iter < 4500; ++iter) {
+    const int64_t sms = sms_list[iter % n_sms];
     const int B = 1 + static_cast<int>(rng() % 40);
     std::vector<int64_t> off{0};
     const int mode = iter % 4;
@@ -164,7 +167,7 @@ int main() {
     const int B = 1000 + static_cast<int>(rng() % 40000);
     std::vector<int64_t> off{0};
     for (int b = 0; b < B; ++b) off.push_back(off.back() + ((rng() % 3 == 0) ? 0 : 1 + rng() % 900));
-    if (check(off, 148)) {
+    if (check(off, iter % 2 ? 148 : 15)) {
       std::printf("case large iter=%d B=%d\n", iter, B);
       return 1;
     }
@@ -173,7 +176,7 @@ int main() {
   // the benchmark shapes
   std::vector<int64_t> u16{0};
   for (int b = 0; b < 16; ++b) u16.push_back(u16.back() + 100000);
-  if (check(u16, 148)) return 1;
+  if (check(u16, 148) || check(u16, 15)) return 1;  // one CTA per SM; clusters of 8
   std::vector<int64_t> zero{0, 0, 0};
   if (check(zero, 148)) return 1;
   std::printf("OK %lld cases\n", cases + 2);
