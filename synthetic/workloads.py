@@ -206,3 +206,10 @@ def user_queries(batch: int, k: int, d: int, seed: int) -> np.ndarray:
     sketch's own type) and not rounded to bf16."""
     rng = np.random.default_rng(seed)
     return rng.standard_normal((batch, k, d), dtype=np.float32)
+
+
+def upstream_gradients(batch: int, k: int, d: int, seed: int):
+    """Seeded upstream gradients for an SA layer's backward: G = dL/dX~
+    (batch, k, d) and g = dL/dm (batch, k), float64 ~ N(0, 1)."""
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((batch, k, d)), rng.standard_normal((batch, k))
