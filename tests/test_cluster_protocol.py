@@ -22,7 +22,7 @@ with arbitrary interleavings and arbitrary delivery delays, and checks that
   * nothing deadlocks (every CTA finishes every tile).
 A variant with one buffer per group in place of two (single-buffered slots)
 must fail, which shows the check can catch the hazard the double buffering
-avoids."""
+avoids.  `simulate_abort` checks the drain planned for the abort path."""
 
 import random
 
@@ -152,3 +152,109 @@ def test_single_buffered_exchange_is_caught():
             found = True
             break
     assert found
+
+
+def simulate_abort(C, tiles, seed, warps=4, settle=True):
+    """The same exchange, but one CTA stops at a random moment (a wait ran
+    out), and every other CTA stops when it would wait for data that the
+    stopped CTA never sends (its own bounded wait runs out).  Then the drain
+    planned for the abort path: every warp's count of tiles sent to each
+    other CTA is published (the exit cluster barrier has every CTA stopped);
+    each CTA arms every phase up to the largest count it was sent, settles
+    the shares that were never sent with a local complete_tx, and waits for
+    those phases.  Checks that when a CTA's phases have all completed no
+    value to it is still in flight (so it may leave), and that the phases do
+    complete once the values in flight have landed (no stuck wait)."""
+    rng = random.Random(seed)
+    groups = 2
+    bars = [[[Barrier(1) for _ in range(2)] for _ in range(groups)] for _ in range(C)]
+    armed = [[0] * groups for _ in range(C)]          # local tiles armed per group
+    sent = {}                                         # (sender, group, warp) -> local tiles sent
+    step = {(h, g, w): ("send", g) for h in range(C) for g in range(groups) for w in range(warps)}
+    stopped = [False] * C
+    in_flight = []
+    victim = rng.randrange(C)
+    stop_after = rng.randrange(1, 40)
+    moves = 0
+    errors = []
+    # run until every actor is done or stuck
+    while True:
+        moves += 1
+        if moves == stop_after:
+            stopped[victim] = True
+        live = [key for key, (st, u) in step.items() if u < tiles and not stopped[key[0]]]
+        runnable = []
+        for key in live:
+            h, g, w = key
+            st, u = step[key]
+            v = u // 2
+            if st == "send" or bars[h][g][v % 2].phase > v // 2:
+                runnable.append(("cta", key))
+        choices = runnable + [("deliver", i) for i in range(len(in_flight))]
+        if not choices:
+            break  # every remaining actor waits for something that never comes
+        kind, what = rng.choice(choices)
+        if kind == "deliver":
+            recv, g, b, sender, w, tile = in_flight.pop(what)
+            bars[recv][g][b].complete_tx(1, tile)
+            continue
+        h, g, w = what
+        st, u = step[what]
+        v = u // 2
+        if st == "send":
+            if w == 0:
+                bars[h][g][v % 2].arrive_expect((C - 1) * warps, u)
+                armed[h][g] = v + 1
+            for p in range(C):
+                if p != h:
+                    in_flight.append((p, g, v % 2, h, w, u))
+            sent[(h, g, w)] = v + 1
+            step[what] = ("wait", u)
+        else:
+            step[what] = ("send", u + 2)
+    # every CTA has stopped: the drain
+    for h in range(C):
+        for g in range(groups):
+            top = max([sent.get((p, g, w), 0) for p in range(C) if p != h for w in range(warps)]
+                      + [armed[h][g]])
+            for v in range(armed[h][g], top):
+                bars[h][g][v % 2].arrive_expect((C - 1) * warps, 2 * v + g)
+            for v in range(top):
+                for p in range(C):
+                    if p == h:
+                        continue
+                    for w in range(warps):
+                        if sent.get((p, g, w), 0) <= v and settle:
+                            bars[h][g][v % 2].complete_tx(1, 2 * v + g)
+            armed[h][g] = top
+
+    def drained(h):
+        return all(bars[h][g][b].phase >= (armed[h][g] + 1 - b) // 2
+                   for g in range(groups) for b in range(2))
+
+    while True:
+        for h in range(C):
+            if drained(h) and any(m[0] == h for m in in_flight):
+                errors.append(f"CTA {h} drained with values still in flight")
+        if errors or not in_flight:
+            break
+        recv, g, b, sender, w, tile = in_flight.pop(rng.randrange(len(in_flight)))
+        bars[recv][g][b].complete_tx(1, tile)
+    for h in range(C):
+        if not drained(h):
+            errors.append(f"CTA {h}: a drain phase never completes")
+    return errors
+
+
+@pytest.mark.parametrize("C", [2, 4, 8])
+def test_abort_drain_plan(C):
+    for seed in range(40):
+        errs = simulate_abort(C, tiles=10, seed=seed)
+        assert not errs, f"C={C} seed={seed}: {errs[:3]}"
+
+
+def test_abort_without_settling_gets_stuck():
+    # Without settling the shares that were never sent, some drain phase
+    # never completes (the bounded wait would run out): the settle step is
+    # what makes the drain finish.
+    assert any(simulate_abort(4, tiles=10, seed=s, settle=False) for s in range(40))
