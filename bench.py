@@ -518,7 +518,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
         "metric": METRIC,
         "value": value,
         "unit": "rows/s",
-        "n_gpus": world,
+        "n_gpus": args.gpus,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": step_ms,
@@ -588,6 +588,14 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if world != args.gpus:
+        # One process per GPU: N GPUs need N ranks (torchrun --nproc-per-node
+        # N).  A mismatch would time a different number of GPUs than the line
+        # reports.
+        ap.error(f"--gpus {args.gpus} but {world} rank(s) were launched "
+                 "(use torchrun --nproc-per-node N for N > 1)")
     if args.impl == "reference":
         run_reference(args, rank)
         return

@@ -228,8 +228,11 @@ sa_status sa_read_device_status(void* workspace, size_t workspace_bytes, void* s
  * pre-registered buffers.  This call takes the same inputs and outputs as
  * sa_sketch_forward, but in place of a caller-provided workspace it uses a
  * fixed 32 MiB scratch array inside the library's device image.  Every GPU
- * that loads the library holds that array until the process exits.  The
- * call itself allocates nothing.
+ * that loads the library's module holds that array until the process exits.
+ * Under CUDA's default lazy module loading the module, and with it the
+ * array, is loaded on a device by the first call there; a call with
+ * batch = 0 does only that set-up, so a caller can make it while allocating
+ * is still allowed.  Later calls allocate nothing.
  *
  *   q, X, offsets, batch, total_rows, X_tilde, mass, stream
  *                     as for sa_sketch_forward
@@ -246,10 +249,13 @@ sa_status sa_read_device_status(void* workspace, size_t workspace_bytes, void* s
  * returns.
  *
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture on the device.  All calls share the
- * one array, so calls whose work overlaps on the GPU (other streams, other
- * host threads) race on it and give wrong results: serialise them.
+ * (cudaGetSymbolAddress, with that device current) and caches it with the
+ * ID of the device's context; make that first call before any stream
+ * capture on the device.  After a device reset the next call runs in a new
+ * context and looks the address up again (the module is reloaded then).
+ * All calls share the one array, so calls whose work overlaps on the GPU
+ * (other streams, other host threads) race on it and give wrong results:
+ * serialise them.
  */
 sa_status sa_sketch_forward_noalloc(sa_query q, const void* X, const int64_t* offsets,
                                     int64_t batch, int64_t total_rows, float* X_tilde,

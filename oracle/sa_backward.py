@@ -21,7 +21,7 @@ Given the upstream gradients G = dL/dX~ (k x d) and g = dL/dm (k):
     dP  = dQ W_Q^T,          dW_Q = P^T dQ
     dX  = A^T G + dK W_K^T,  dW_K = X^T dK
 
-Readings (also listed in the design doc):
+Readings (the page prints no backward pass):
   B1  the loss may depend on both outputs, X~ and m (m is returned beside X~,
       reading R4), so both upstream gradients are inputs; g = 0 gives the
       gradient of a loss on X~ alone.

@@ -22,7 +22,7 @@ remains fixes the computation:
 * The sketch is a weighted aggregation, not a selection; prototypes are not
   forced to receive equal mass (section 2.1, closing paragraph).
 
-Readings where the page is silent (each also listed in the design doc):
+Readings where the page is silent:
   R1  S = (P W_Q)(X W_K)^T * scale, i.e. S_ji = scale * (p_j W_Q).(x_i W_K).
   R2  scale is an input (1/sqrt(d) in every workload); no learnable
       temperature, no projection bias.

@@ -163,7 +163,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0u) {  // the 128-byte swizzle needs 1024-byte alignment
     grid_dependency_wait();
-    if (threadIdx.x == 0) atomicOr(&a.header->timeout_flags, DEVFLAG_SMEM_ALIGN);
+    // Every CTA of the launch has the same layout and takes this path, so
+    // block 0 alone reports it (clearing the previous call's offset bits).
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      a.header->flags = 0u;
+      a.header->timeout_flags = DEVFLAG_SMEM_ALIGN;
+    }
     return;
   }
   const uint32_t sbase = smem_u32(smem);
@@ -247,6 +252,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   grid_dependency_wait();
+  // The device flags of this call start clear.  This is block 0's first
+  // global access: the preceding kernel's writes are visible, and any other
+  // CTA can set a flag only after a bounded wait has run out (seconds).
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    a.header->flags = 0u;
+    a.header->timeout_flags = 0u;
+  }
   if (warp == 0) {
     // This CTA's row range and its first user (the work split of
     // sa_internal.h, searched by the whole warp).
@@ -258,7 +270,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       range_slot[0] = r0;
       range_slot[1] = r1;
       *b0_slot = b0v;
-      if (c == 0) { a.header->flags = 0u; a.header->timeout_flags = 0u; }
     }
     // Offsets from the CTA's first user on, in shared memory: every role
     // walks them at each segment change, and a global load there (a

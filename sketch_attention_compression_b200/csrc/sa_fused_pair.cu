@@ -99,6 +99,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const int64_t N = a.total_rows;
   uint32_t* sticky = &a.header->timeout_flags;
 
+  // The device flags of this call start clear (block 0's first global
+  // access; another CTA can set a flag only after a bounded wait has run
+  // out).  Every CTA has the same shared-memory layout, so on misalignment
+  // all of them stop here and block 0 alone reports it.
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    a.header->flags = 0u;
+    a.header->timeout_flags = aligned ? 0u : DEVFLAG_SMEM_ALIGN;
+  }
   if (aligned && threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
     mbar_init(s_full, 1);
@@ -122,10 +130,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     range_slot[0] = r0;
     range_slot[1] = r1;
     *b0_slot = r0 < r1 ? b0u : a.batch;
-    if (c == 0 && h == 0) { a.header->flags = 0u; a.header->timeout_flags = 0u; }
     fence_mbar_init();
   }
-  if (!aligned && threadIdx.x == 0) atomicOr(&a.header->timeout_flags, DEVFLAG_SMEM_ALIGN);
   if (aligned) {  // the block of bf16 ones read as MMA2's extra 16 columns
     const uint32_t ones = sbase + kOnesBlk * kB;
     for (int i = threadIdx.x; i < kB / 16; i += kPairThreads)

@@ -38,9 +38,12 @@ constexpr int kTileRows = 128;
 struct WsHeader {
   uint32_t flags;          // offset validation bits (set by the finalize pass)
   uint32_t timeout_flags;  // bounded-wait timeouts (set by the partial pass)
-  // Both words are zeroed by CTA 0 of the partial pass at the start of every
-  // call; all CTAs of that pass are resident together, so this precedes any
-  // timeout report (which takes seconds to arise).
+  // Both words are zeroed by block 0 of the partial pass as its first global
+  // write of every call.  Another CTA of that pass reports a timeout only
+  // after one of its bounded waits has run out (seconds), and the finalize
+  // pass sets the offset bits after the partial pass has completed, so the
+  // clearing precedes every report of the call.  On misaligned shared memory
+  // every CTA stops at once and block 0 alone writes both words.
   uint32_t pad[62];
 };
 constexpr size_t kWsHeaderBytes = 256;

@@ -7,14 +7,23 @@
 // hand the library only fixed, pre-registered buffers.  This entry point
 // takes the same inputs and outputs as sa_sketch_forward.  In place of a
 // caller-provided workspace it uses a fixed scratch array that lives in this
-// library's device image.  The array is reserved when the library's module
-// is loaded on a device, and it stays reserved on every device that loads
-// the library until the process exits.
+// library's device image.
+//
+// When the array is reserved.  The array sits in the module built from this
+// file.  With CUDA's default lazy module loading, that module is loaded on a
+// device, and the array reserved there, at the first call that needs it:
+// the address lookup of the first call on the device.  A call with batch = 0
+// does that set-up and nothing else, so a caller can make it at start-up,
+// while allocating is still allowed.  From then on the array stays reserved
+// on that device until the process exits (or the device is reset), and no
+// call allocates.
 //
 // The array's name is a host-side stand-in, not a device address.  Host code
-// must look the address up with cudaGetSymbolAddress, once per device, with
-// that device current.  That lookup is the per-device set-up below.
+// must look the address up with cudaGetSymbolAddress, with the device
+// current, once per device and context.  That lookup is the set-up below.
 #include <mutex>
+
+#include <cuda.h>
 
 #include "sa.h"
 
@@ -29,10 +38,44 @@ static __device__ __align__(256) unsigned char sa_noalloc_scratch[kNoAllocScratc
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
+// Per device: the scratch address and the context it was looked up in.  A
+// device reset (cudaDeviceReset) destroys the context and unloads the
+// module; the next call on that device runs in a new context, which has a
+// new ID, and looks the address up again.
 void* g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
 
-// Address of the scratch array on the current device (looked up once per
-// device), or nullptr with *err set if the lookup failed.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique ID of the context current on this thread (0 if none, or if the
+// driver does not offer the query).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    looked_up = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS ||
+      ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Address of the scratch array on the current device, looked up once per
+// device and context, or nullptr with *err set if the lookup failed.
 void* scratch_on_current_device(cudaError_t* err) {
   int dev = -1;
   *err = cudaGetDevice(&dev);
@@ -42,11 +85,14 @@ void* scratch_on_current_device(cudaError_t* err) {
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_scratch_ptr[dev] == nullptr || ctx == 0 || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     *err = cudaGetSymbolAddress(&p, sa_noalloc_scratch);
     if (*err != cudaSuccess) return nullptr;
     g_scratch_ptr[dev] = p;
+    // The lookup makes the runtime's context current if none was.
+    g_scratch_ctx[dev] = ctx != 0 ? ctx : current_context_id();
   }
   return g_scratch_ptr[dev];
 }

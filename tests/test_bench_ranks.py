@@ -76,3 +76,20 @@ def test_reference_arm_runs_on_rank0_only(rank):
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+@pytest.mark.parametrize("impl", ["ours", "reference"])
+def test_gpus_must_match_the_launched_ranks(impl):
+    """--gpus 2 in a single process (no torchrun) is an error, not a silent
+    one-GPU run reported as two; so is --gpus 1 among two ranks."""
+    for gpus, world in ((2, None), (1, 2)):
+        env = _cpu_env()
+        for key in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+            env.pop(key, None)
+        if world is not None:
+            env.update({"RANK": "0", "WORLD_SIZE": str(world), "LOCAL_RANK": "0"})
+        r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", impl,
+                            "--gpus", str(gpus), "--steps", "1", "--warmup", "3",
+                            "--workload", "batch32_n10k_d128_k64_bf16"],
+                           capture_output=True, text=True, timeout=240, env=env, cwd=ROOT)
+        assert r.returncode != 0 and "rank(s) were launched" in r.stderr, r.stderr[-1000:]
