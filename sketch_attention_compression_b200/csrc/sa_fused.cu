@@ -291,6 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool user_q = a.user_queries != 0;
   uint32_t tiles_issued = 0;  // producer thread: X tiles whose TMA copy was issued
   uint32_t q_loads = 0;       // Q' loader thread (per-user queries): Q'_b copies issued
+  // Clusters, per softmax warp: the group's tiles (local index u) whose row
+  // totals this warp sent, whose exchange phase it saw complete, and (warp
+  // q = 0, which arms the group's barrier) whose phase it armed.  The abort
+  // drain at exit reads them.
+  uint32_t xch_sent = 0, xch_waited = 0, xch_armed = 0;
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -519,6 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t u = t >> 1, par = u & 1u;
           uint64_t* sfull = &stats_full[grp * 2 + par];
           if (q == 0 && lane == 0) mbar_arrive_expect_tx(sfull, (ncl - 1) * 128 * 4);
+          if (q == 0) xch_armed = u + 1;
           const float Lh = mx + lg2_approx(zl);
           const uint32_t sfull_a = smem_u32(sfull);
           constexpr bool kWide = CLU == 2;
@@ -526,11 +532,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t mine = kWide ? region + h * 512 + row * 4 : region + row * 16 + h * 4;
           for (uint32_t p = 0; p < ncl; ++p)
             if (p != h) st_async_f32(map_to_cta(mine, p), Lh, map_to_cta(sfull_a, p));
+          xch_sent = u + 1;
           asm volatile("st.shared.f32 [%0], %1;" ::"r"(mine), "f"(Lh) : "memory");
           if (!warp_wait_cluster(sfull, (u >> 1) & 1u, abort_flag, sticky)) {
             ok = false;
             break;
           }
+          xch_waited = u + 1;
           float Lv[kMaxCluster];
           if constexpr (kWide) {
 #pragma unroll
@@ -722,9 +730,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  // No CTA of a cluster leaves while another may still read its published
-  // statistics or signal its barriers.
-  if (kClu) cluster_sync();
+  if constexpr (kClu) {
+    // Row totals travel between the CTAs with st.async, which the cluster
+    // barrier does not order.  On the normal path every value a CTA was
+    // sent has been waited for.  If any CTA of the cluster gave up, a value
+    // may still be in flight to a CTA that stopped waiting, so before the
+    // final barrier each CTA waits until everything sent to it has landed:
+    //   1. every CTA publishes its abort flag and, per softmax warp, its
+    //      exchange counts (in the offset cache, unused from here on), then
+    //      all pass one cluster barrier, on every path;
+    //   2. if any CTA aborted, one thread per group re-arms the at most one
+    //      phase that was sent to but not armed, settles with complete_tx
+    //      the shares of every phase that a stopped warp never sent, and
+    //      waits (bounded) until those phases complete, i.e. until the
+    //      values in flight have landed.
+    // A sender can only send tile u + 1 of a group after it received the
+    // receiver's tile u, which the receiver sends after arming it, and a
+    // warp arms tile u + 1 only after it saw tile u complete; so the
+    // phases left open are the group's tiles waited and waited + 1, on the
+    // two different barriers of its double buffer.
+    uint32_t* pub = reinterpret_cast<uint32_t*>(off_cache);  // [0] abort, [1 + 12 g + 3 q + i]
+    if (warp >= 4 && lane == 0) {
+      const int g = (warp - 4) >> 2, q = warp & 3;
+      pub[1 + 12 * g + 3 * q + 0] = xch_sent;
+      pub[1 + 12 * g + 3 * q + 1] = xch_waited;
+      pub[1 + 12 * g + 3 * q + 2] = xch_armed;
+    }
+    if (threadIdx.x == 0) pub[0] = *abort_flag;
+    cluster_sync();
+    if ((warp == 4 || warp == 8) && lane == 0) {
+      const int g = (warp - 4) >> 2;
+      const uint32_t pub_a = smem_u32(pub);
+      uint32_t any = 0;
+      for (uint32_t p = 0; p < ncl; ++p) any |= ld_shared_cluster_u32(map_to_cta(pub_a, p));
+      if (any) {
+        uint32_t waited = 0;
+        for (int q = 0; q < 4; ++q) waited = max(waited, pub[1 + 12 * g + 3 * q + 1]);
+        const uint32_t armed = pub[1 + 12 * g + 2];
+        uint32_t sent[kMaxCluster][4];
+        uint32_t top = armed;
+        for (uint32_t p = 0; p < ncl; ++p)
+          for (int q = 0; q < 4; ++q) {
+            sent[p][q] = p == h ? 0u : ld_shared_cluster_u32(map_to_cta(pub_a + 4 * (1 + 12 * g + 3 * q), p));
+            top = max(top, sent[p][q]);
+          }
+        for (uint32_t v = waited; v < top && v < waited + 2; ++v) {
+          uint64_t* bar = &stats_full[g * 2 + (v & 1u)];
+          if (v >= armed) mbar_arrive_expect_tx(bar, (ncl - 1) * 128 * 4);
+          for (uint32_t p = 0; p < ncl; ++p)
+            for (int q = 0; q < 4; ++q)
+              if (p != h && sent[p][q] <= v) mbar_complete_tx(bar, 32 * 4);
+        }
+        for (uint32_t v = waited; v < top && v < waited + 2; ++v)
+          mbar_wait_bounded(&stats_full[g * 2 + (v & 1u)], (v >> 1) & 1u);
+      }
+    }
+    // No CTA of a cluster leaves while another may still read its published
+    // counts or signal its barriers.
+    cluster_sync();
+  }
 }
 
 template <int D, int KM>

@@ -91,6 +91,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   volatile uint32_t* abort_flag = tmem_slot + 1;
   int64_t* b0_slot = reinterpret_cast<int64_t*>(tmem_slot + 2);
   int64_t* range_slot = reinterpret_cast<int64_t*>(tmem_slot + 4);  // R0, R1
+  // Published at exit for the abort drain: [0] abort flag, then per softmax
+  // warp q the tiles it sent, saw complete and (q = 0) armed: [1 + 3q + i].
+  uint32_t* pub = reinterpret_cast<uint32_t*>(range_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -151,6 +154,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
   uint32_t tiles_issued = 0;  // producer thread: X tiles whose TMA copy was issued
   uint32_t q_loads = 0;       // Q' loader thread (per-user queries): Q'_b copies issued
+  // Per softmax thread: tiles whose (m, z) it sent, whose exchange phase it
+  // saw complete, and (row 0, which arms the barrier) whose phase it armed.
+  uint32_t xch_sent = 0, xch_waited = 0, xch_armed = 0;
   const bool user_q = a.user_queries != 0;
   if (aligned) {
     const uint32_t tmem = *tmem_slot;
@@ -349,9 +355,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           // which are sent after this CTA read tile t's slot, so neither a
           // slot nor a barrier phase is reused early.
           if (row == 0) mbar_arrive_expect_tx(&xch[par], 128 * 8);
+          xch_armed = t + 1;
           st_async_v2f(map_to_cta(xslot_a + (par * 128 + row) * 8, peer), m_h, z_h,
                        map_to_cta(xch_a + par * 8, peer));
+          xch_sent = t + 1;
           if (!mbar_wait_cluster(&xch[par], (t >> 1) & 1u, abort_flag, sticky)) { ok = false; break; }
+          xch_waited = t + 1;
           const float2 other = xslot[par * 128 + row];
           const float m_row = fmaxf(m_h, other.x);
           const float f_h = ex2_approx(m_h - m_row);  // 0 when this half is fully masked
@@ -459,7 +468,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     tc_fence_after();
     tmem_dealloc(*tmem_slot, 512);
   }
-  // No CTA leaves while the other may still store into its shared memory.
+  // The (m, z) values travel with st.async, which the cluster barrier does
+  // not order.  On the normal path every value a CTA was sent has been
+  // waited for.  If either CTA gave up, a value may still be in flight to a
+  // CTA that stopped waiting, so before the final barrier each CTA waits
+  // until everything sent to it has landed: both publish their abort flag
+  // and exchange counts and pass a cluster barrier (on every path); then, if
+  // either aborted, thread 0 of the softmax warps arms the at most one phase
+  // the peer sent to but this CTA did not arm, settles with complete_tx the
+  // shares the peer's stopped warps never sent, and waits (bounded) for
+  // those phases.  The peer sends tile t + 1 only after receiving this CTA's
+  // tile t, which row 0 sends after arming it, and row 0 arms tile t + 1
+  // only after tile t completed; so only tiles `waited` and `waited` + 1
+  // can be open, one on each barrier of the double buffer.  (The row-0
+  // thread's counts stand for its warp; another lane's later success only
+  // means a phase is complete, which the drain then finds at once.)
+  if (aligned) {
+    if (warp >= 4 && lane == 0) {
+      const int q = warp & 3;
+      pub[1 + 3 * q] = xch_sent;
+      pub[2 + 3 * q] = xch_waited;
+      pub[3 + 3 * q] = xch_armed;
+    }
+    if (threadIdx.x == 0) pub[0] = *abort_flag;
+  }
+  cluster_sync();
+  if (aligned && warp == 4 && lane == 0) {
+    const uint32_t peer_pub = map_to_cta(smem_u32(pub), peer);
+    if (pub[0] | ld_shared_cluster_u32(peer_pub)) {
+      uint32_t waited = 0;
+      for (int q = 0; q < 4; ++q) waited = max(waited, pub[2 + 3 * q]);
+      const uint32_t armed = pub[3];
+      uint32_t sent[4];
+      uint32_t top = armed;
+      for (int q = 0; q < 4; ++q) {
+        sent[q] = ld_shared_cluster_u32(peer_pub + 4 * (1 + 3 * q));
+        top = max(top, sent[q]);
+      }
+      for (uint32_t v = waited; v < top && v < waited + 2; ++v) {
+        if (v >= armed) mbar_arrive_expect_tx(&xch[v & 1u], 128 * 8);
+        for (int q = 0; q < 4; ++q)
+          if (sent[q] <= v) mbar_complete_tx(&xch[v & 1u], 32 * 8);
+      }
+      for (uint32_t v = waited; v < top && v < waited + 2; ++v)
+        mbar_wait_bounded(&xch[v & 1u], (v >> 1) & 1u);
+    }
+  }
+  // No CTA leaves while the other may still read its published counts or
+  // store into its shared memory.
   cluster_sync();
 }
 

@@ -386,6 +386,23 @@ __device__ __forceinline__ void st_async_f32(uint32_t remote, float a, uint32_t 
       : "memory");
 }
 
+// Completes `bytes` transaction bytes on this CTA's own mbarrier without a
+// transfer (the abort drain of the cluster passes settles the shares of an
+// exchange phase that a stopped CTA never sent).
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// A 32-bit word of another CTA's shared memory (address from map_to_cta);
+// ordered after the cluster barrier that published it.
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t remote) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ float lg2_approx(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

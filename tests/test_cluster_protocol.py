@@ -22,7 +22,8 @@ with arbitrary interleavings and arbitrary delivery delays, and checks that
   * nothing deadlocks (every CTA finishes every tile).
 A variant with one buffer per group in place of two (single-buffered slots)
 must fail, which shows the check can catch the hazard the double buffering
-avoids.  `simulate_abort` checks the drain planned for the abort path."""
+avoids.  `simulate_abort` checks the drain the kernels run on the abort
+path."""
 
 import random
 
@@ -158,18 +159,29 @@ def simulate_abort(C, tiles, seed, warps=4, settle=True):
     """The same exchange, but one CTA stops at a random moment (a wait ran
     out), and every other CTA stops when it would wait for data that the
     stopped CTA never sends (its own bounded wait runs out).  Then the drain
-    planned for the abort path: every warp's count of tiles sent to each
-    other CTA is published (the exit cluster barrier has every CTA stopped);
-    each CTA arms every phase up to the largest count it was sent, settles
-    the shares that were never sent with a local complete_tx, and waits for
-    those phases.  Checks that when a CTA's phases have all completed no
-    value to it is still in flight (so it may leave), and that the phases do
-    complete once the values in flight have landed (no stuck wait)."""
+    at the end of the cluster passes (sa_fused.cu with CLU, and
+    sa_fused_pair.cu with C = 2 and one group), step for step:
+      * every softmax warp has counted the tiles of its group it sent
+        (xch_sent), saw complete (xch_waited) and, warp 0, armed
+        (xch_armed); the counts are published and all pass a cluster
+        barrier;
+      * per group, waited = the largest xch_waited of its warps, armed =
+        warp 0's xch_armed, top = the largest count any other CTA's warp
+        sent; for the local tiles v in [waited, min(top, waited + 2)) the
+        drain arms the phase if v >= armed and settles with complete_tx the
+        share of every (sender, warp) whose count is <= v; then it waits
+        for those phases.
+    Checks that top never exceeds waited + 2 (so the cap drops nothing and
+    the open tiles sit on the two barriers of the double buffer), that when
+    a CTA's phases have all completed no value to it is still in flight (so
+    it may pass the final barrier), and that the phases do complete once the
+    values in flight have landed (no stuck wait)."""
     rng = random.Random(seed)
     groups = 2
     bars = [[[Barrier(1) for _ in range(2)] for _ in range(groups)] for _ in range(C)]
-    armed = [[0] * groups for _ in range(C)]          # local tiles armed per group
-    sent = {}                                         # (sender, group, warp) -> local tiles sent
+    armed = [[0] * groups for _ in range(C)]          # xch_armed of warp 0, per group
+    sent = {}                                         # xch_sent, (CTA, group, warp)
+    waited = {}                                       # xch_waited, (CTA, group, warp)
     step = {(h, g, w): ("send", g) for h in range(C) for g in range(groups) for w in range(warps)}
     stopped = [False] * C
     in_flight = []
@@ -211,26 +223,33 @@ def simulate_abort(C, tiles, seed, warps=4, settle=True):
             sent[(h, g, w)] = v + 1
             step[what] = ("wait", u)
         else:
+            waited[(h, g, w)] = v + 1
             step[what] = ("send", u + 2)
     # every CTA has stopped: the drain
+    open_tiles = {}
     for h in range(C):
         for g in range(groups):
+            wt = max(waited.get((h, g, w), 0) for w in range(warps))
             top = max([sent.get((p, g, w), 0) for p in range(C) if p != h for w in range(warps)]
                       + [armed[h][g]])
-            for v in range(armed[h][g], top):
-                bars[h][g][v % 2].arrive_expect((C - 1) * warps, 2 * v + g)
-            for v in range(top):
+            if top > wt + 2:
+                errors.append(f"CTA {h} group {g}: top {top} > waited {wt} + 2")
+            hi = min(top, wt + 2)
+            for v in range(wt, hi):
+                if v >= armed[h][g]:
+                    bars[h][g][v % 2].arrive_expect((C - 1) * warps, 2 * v + g)
                 for p in range(C):
                     if p == h:
                         continue
                     for w in range(warps):
                         if sent.get((p, g, w), 0) <= v and settle:
                             bars[h][g][v % 2].complete_tx(1, 2 * v + g)
-            armed[h][g] = top
+            open_tiles[(h, g)] = (wt, hi)
 
     def drained(h):
-        return all(bars[h][g][b].phase >= (armed[h][g] + 1 - b) // 2
-                   for g in range(groups) for b in range(2))
+        # the drain's bounded waits: phase v // 2 of barrier v % 2 complete
+        return all(bars[h][g][v % 2].phase > v // 2
+                   for g in range(groups) for v in range(*open_tiles[(h, g)]))
 
     while True:
         for h in range(C):
@@ -247,7 +266,7 @@ def simulate_abort(C, tiles, seed, warps=4, settle=True):
 
 
 @pytest.mark.parametrize("C", [2, 4, 8])
-def test_abort_drain_plan(C):
+def test_abort_drain(C):
     for seed in range(40):
         errs = simulate_abort(C, tiles=10, seed=seed)
         assert not errs, f"C={C} seed={seed}: {errs[:3]}"
