@@ -20,3 +20,11 @@ from .sa_oracle import (  # noqa: F401
 )
 from .brute import sa_user_bruteforce  # noqa: F401
 from .sa_backward import sa_batch_backward, sa_user_backward  # noqa: F401
+from .sa_refine import (  # noqa: F401
+    layer_norm,
+    refine_layer,
+    refine_stack,
+    refine_update,
+    silu,
+    swiglu_ffn,
+)
