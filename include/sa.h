@@ -279,6 +279,113 @@ sa_status sa_sketch_forward_noalloc(sa_query q, const void* X, const int64_t* of
 sa_status sa_mass_normalise(const float* X_tilde, const float* mass, int64_t batch, int k, int d,
                             float* out, void* stream);
 
+/*
+ * Stacked refinement layers (section 2.2 "Stacked Refinement" of the same
+ * notes).  Layer l queries the ORIGINAL history X with the previous layer's
+ * sketches (layer 1 with the shared prototypes: X~^(0) = P^(0)) and then
+ * updates every (user, prototype) row of width d:
+ *
+ *     z   = LN1(prev_bj + X~_bj / m_bj)          (X~/m is 0 where m_bj = 0)
+ *     out = LN2(z + (SiLU(z W1) * (z W3)) W2)
+ *
+ * where X~, m are that layer's SA outputs, LN normalises over the d features
+ * (biased variance, eps 1e-5) with gain gamma and shift beta, and the FFN is
+ * SwiGLU-gated with hidden width h and no biases.  The page lost the layer's
+ * formulas; this is the reading its text supports (the aggregation added to
+ * the previous state and normalised, then a residual feed-forward network):
+ * the aggregation enters mass-normalised, a weighted mean of the user's
+ * rows, whose scale does not grow with the history length.  Every layer has
+ * its own sa_query (W_Q, W_K, scale) and sa_refine (LN and FFN parameters).
+ */
+typedef struct sa_refine_s* sa_refine;
+
+/*
+ * sa_prepare_refine -- the LN and FFN parameters of one refinement layer.
+ *
+ *   W1, W3   device, d x h fp32, row-major (z W1, z W3)
+ *   W2       device, h x d fp32, row-major
+ *   gamma1, beta1, gamma2, beta2   device, d fp32 each (LN1, LN2)
+ *   d        64 or 128 (256: SA_ERR_UNSUPPORTED)
+ *   h        hidden width, a multiple of 128, 128 <= h <= 4096
+ *   stream   the copies (bf16, transposed) are made by kernels on it
+ *   out      host; receives the handle
+ *
+ * Allocates device memory for the parameters; the inputs may be freed once
+ * `stream` has passed this call.  Errors: SA_ERR_INVALID_ARG (null,
+ * misaligned, bad d or h), SA_ERR_UNSUPPORTED (d = 256, or not sm_100),
+ * SA_ERR_CUDA.
+ */
+sa_status sa_prepare_refine(const float* W1, const float* W3, const float* W2,
+                            const float* gamma1, const float* beta1, const float* gamma2,
+                            const float* beta2, int d, int h, void* stream, sa_refine* out);
+
+/* Releases a refinement handle and its device memory.  NULL is a no-op. */
+void sa_refine_free(sa_refine r);
+
+/*
+ * sa_refine_update -- the update after a layer's SA step, for batch * k rows
+ * (one tcgen05 kernel: LN1, the FFN on the tensor cores in bf16 with fp32
+ * accumulation, LN2; the norms in fp32).
+ *
+ *   prev         device fp32, 16-byte aligned: batch x k x d, or k x d
+ *                shared by every user when prev_shared != 0 (layer 1: P)
+ *   X_tilde      device, batch x k x d fp32 (16-byte aligned): the layer's
+ *                SA sketches
+ *   mass         device, batch x k fp32: the layer's masses
+ *   batch, k     batch >= 0, k >= 1
+ *   out          device, batch x k x d fp32 (16-byte aligned); must not
+ *                overlap the inputs
+ *   device_flags device uint32 (or NULL): SA_DEVFLAG_TIMEOUT is OR-ed in if
+ *                a bounded wait in the kernel gave up
+ *   stream       the kernel is enqueued here
+ */
+sa_status sa_refine_update(sa_refine r, const float* prev, int prev_shared, const float* X_tilde,
+                           const float* mass, int64_t batch, int k, float* out,
+                           uint32_t* device_flags, void* stream);
+
+/*
+ * sa_refine_layer_forward -- one refinement layer over a ragged batch: the
+ * SA step (section 2.1 with the layer's query; per-user queries for l >= 2)
+ * followed by sa_refine_update.
+ *
+ *   q          the layer's SA query (its W_Q, W_K, scale; its P for layer 1)
+ *   r          the layer's LN and FFN parameters (same d as q; q bf16)
+ *   prev       device fp32: NULL for layer 1 (the query and the residual are
+ *              the shared prototypes, given as P_f32), else the previous
+ *              layer's sketches, batch x k x d
+ *   P_f32      device, k x d fp32: the prototypes q was prepared with, as
+ *              fp32 (read only when prev is NULL)
+ *   X, offsets, batch, total_rows   as for sa_sketch_forward
+ *   out        device, batch x k x d fp32: X~^(l); must not overlap prev
+ *   workspace  device, >= sa_workspace_bytes_refine_layer(q, batch,
+ *              total_rows), 256-byte aligned; one call at a time
+ *
+ * Device flags (bad offsets, timeouts) are read with sa_read_device_status
+ * on the workspace, as for sa_sketch_forward.
+ */
+size_t sa_workspace_bytes_refine_layer(sa_query q, int64_t batch, int64_t total_rows);
+sa_status sa_refine_layer_forward(sa_query q, sa_refine r, const float* prev, const float* P_f32,
+                                  const void* X, const int64_t* offsets, int64_t batch,
+                                  int64_t total_rows, float* out, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/*
+ * sa_refine_stack_forward -- `layers` refinement layers in sequence (the
+ * final configuration of section 2.2 has two): layer 1 from P_f32, each
+ * later layer queried by the previous layer's output; every layer reads the
+ * original X.  qs[l], rs[l] are layer l's handles (all with the same k, d).
+ *
+ *   out        device, batch x k x d fp32: X~^(layers)
+ *   workspace  device, >= sa_workspace_bytes_refine_stack(qs[0], batch,
+ *              total_rows) (which also holds the layers' intermediate
+ *              sketches), 256-byte aligned
+ */
+size_t sa_workspace_bytes_refine_stack(sa_query q, int64_t batch, int64_t total_rows);
+sa_status sa_refine_stack_forward(int layers, const sa_query* qs, const sa_refine* rs,
+                                  const float* P_f32, const void* X, const int64_t* offsets,
+                                  int64_t batch, int64_t total_rows, float* out, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
 /* Static description of a status code. */
 const char* sa_status_string(sa_status s);
 

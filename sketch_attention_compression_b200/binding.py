@@ -45,6 +45,16 @@ SIGNATURES = {
     "sa_status_string": (ctypes.c_char_p, [_i32]),
     "sa_query_info": (_i32, [_vp, ctypes.POINTER(_i32), ctypes.POINTER(_i32),
                              ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
+    "sa_prepare_refine": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp,
+                                 ctypes.POINTER(_vp)]),
+    "sa_refine_free": (None, [_vp]),
+    "sa_refine_update": (_i32, [_vp, _vp, _i32, _vp, _vp, _i64, _i32, _vp, _vp, _vp]),
+    "sa_workspace_bytes_refine_layer": (_sz, [_vp, _i64, _i64]),
+    "sa_refine_layer_forward": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _sz,
+                                       _vp]),
+    "sa_workspace_bytes_refine_stack": (_sz, [_vp, _i64, _i64]),
+    "sa_refine_stack_forward": (_i32, [_i32, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _sz,
+                                       _vp]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -305,6 +315,107 @@ class SketchQuery:
             self.close()
         except Exception:
             pass
+
+
+class RefineParams:
+    """The LN and FFN parameters of one refinement layer (sa_prepare_refine):
+    W1, W3 (d, h), W2 (h, d), gamma1, beta1, gamma2, beta2 (d,), fp32 CUDA
+    tensors."""
+
+    def __init__(self, W1, W3, W2, gamma1, beta1, gamma2, beta2, stream=None):
+        torch = _torch()
+        lib = load_library()
+        for name, t in (("W1", W1), ("W3", W3), ("W2", W2), ("gamma1", gamma1), ("beta1", beta1),
+                        ("gamma2", gamma2), ("beta2", beta2)):
+            if t.dtype != torch.float32:
+                raise TypeError(f"{name} must be float32")
+        self.d, self.h = int(W1.shape[0]), int(W1.shape[1])
+        if tuple(W3.shape) != (self.d, self.h) or tuple(W2.shape) != (self.h, self.d):
+            raise ValueError("W1, W3 must be (d, h) and W2 (h, d)")
+        handle = ctypes.c_void_p()
+        st = lib.sa_prepare_refine(*(_dev_ptr(t, n) for n, t in (
+            ("W1", W1), ("W3", W3), ("W2", W2), ("gamma1", gamma1), ("beta1", beta1),
+            ("gamma2", gamma2), ("beta2", beta2))), self.d, self.h,
+            ctypes.c_void_p(_stream_handle(stream)), ctypes.byref(handle))
+        _check(st, "sa_prepare_refine")
+        self._h = handle
+        self._lib = lib
+
+    def update(self, prev, X_tilde, mass, out=None, prev_shared: bool = False,
+               device_flags=None, stream=None):
+        """out = LN2(z + FFN(z)), z = LN1(prev + X~ / m) for (B, k, d) fp32
+        tensors; prev is (k, d) and shared by every user with prev_shared."""
+        torch = _torch()
+        B, k, d = (int(x) for x in X_tilde.shape)
+        if out is None:
+            out = torch.empty_like(X_tilde)
+        fp = _dev_ptr(device_flags, "device_flags") if device_flags is not None else ctypes.c_void_p(0)
+        _check(self._lib.sa_refine_update(self._h, _dev_ptr(prev, "prev"), int(prev_shared),
+                                          _dev_ptr(X_tilde, "X_tilde"), _dev_ptr(mass, "mass"), B, k,
+                                          _dev_ptr(out, "out"), fp,
+                                          ctypes.c_void_p(_stream_handle(stream))),
+               "sa_refine_update")
+        return out
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self._lib.sa_refine_free(self._h)
+            self._h = None
+
+    def __del__(self):  # pragma: no cover
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def refine_layer_forward(query: "SketchQuery", params: RefineParams, X, offsets, prev=None,
+                         P_f32=None, out=None, workspace=None, stream=None):
+    """One refinement layer (sa_refine_layer_forward): prev None means layer 1
+    (queried by, and residual on, the prototypes P_f32 (k, d) fp32)."""
+    torch = _torch()
+    lib = load_library()
+    B, N = int(offsets.shape[0]) - 1, int(X.shape[0])
+    if out is None:
+        out = torch.empty((B, query.k, query.d), dtype=torch.float32, device=X.device)
+    if workspace is None:
+        workspace = torch.empty(int(lib.sa_workspace_bytes_refine_layer(query._h, B, N)),
+                                dtype=torch.uint8, device=X.device)
+    _check(lib.sa_refine_layer_forward(
+        query._h, params._h, _dev_ptr(prev, "prev") if prev is not None else ctypes.c_void_p(0),
+        _dev_ptr(P_f32, "P_f32") if P_f32 is not None else ctypes.c_void_p(0),
+        ctypes.c_void_p(X.data_ptr() if N > 0 else 0), _dev_ptr(offsets, "offsets"), B, N,
+        _dev_ptr(out, "out"), _dev_ptr(workspace, "workspace"),
+        int(workspace.numel() * workspace.element_size()),
+        ctypes.c_void_p(_stream_handle(stream))), "sa_refine_layer_forward")
+    return out, workspace
+
+
+def refine_stack_forward(queries, params, P_f32, X, offsets, out=None, workspace=None,
+                         stream=None):
+    """len(queries) refinement layers (sa_refine_stack_forward); queries[l]
+    and params[l] are layer l's handles.  Returns (out, workspace)."""
+    torch = _torch()
+    lib = load_library()
+    L = len(queries)
+    if L != len(params) or L < 1:
+        raise ValueError("one query and one parameter set per layer")
+    B, N = int(offsets.shape[0]) - 1, int(X.shape[0])
+    q0 = queries[0]
+    if out is None:
+        out = torch.empty((B, q0.k, q0.d), dtype=torch.float32, device=X.device)
+    if workspace is None:
+        workspace = torch.empty(int(lib.sa_workspace_bytes_refine_stack(q0._h, B, N)),
+                                dtype=torch.uint8, device=X.device)
+    qs = (ctypes.c_void_p * L)(*[q._h.value for q in queries])
+    rs = (ctypes.c_void_p * L)(*[r._h.value for r in params])
+    _check(lib.sa_refine_stack_forward(
+        L, ctypes.cast(qs, ctypes.c_void_p), ctypes.cast(rs, ctypes.c_void_p),
+        _dev_ptr(P_f32, "P_f32"), ctypes.c_void_p(X.data_ptr() if N > 0 else 0),
+        _dev_ptr(offsets, "offsets"), B, N, _dev_ptr(out, "out"),
+        _dev_ptr(workspace, "workspace"), int(workspace.numel() * workspace.element_size()),
+        ctypes.c_void_p(_stream_handle(stream))), "sa_refine_stack_forward")
+    return out, workspace
 
 
 def mass_normalise(X_tilde, mass, out=None, stream=None):

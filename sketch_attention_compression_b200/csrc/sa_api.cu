@@ -25,16 +25,14 @@ struct sa_query_s {
   CUtensorMap tmap_q_half;  // boxes of 128 rows (k_pad == 256: one half per CTA of a pair)
 };
 
-namespace {
-
-using sa::PassArgs;
+namespace sa {
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_fn() {
+static EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   if (fn == nullptr) {
     void* p = nullptr;
@@ -47,8 +45,6 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor map over a row-major [rows][cols] array, boxes of
-// 64 columns (128 bytes) x box_rows rows, 128-byte swizzle, zero fill.
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
@@ -62,6 +58,13 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+}  // namespace sa
+
+namespace {
+
+using sa::PassArgs;
+using sa::make_tmap_bf16;
 
 constexpr int64_t kMaxRows = (int64_t{1} << 31) - 256;
 
@@ -113,7 +116,7 @@ enum class Phase { kBoth, kPartials, kFinalize };
 // queries every user with the prepared Q'.
 sa_status run(sa_query q, const float* queries, const void* X, const int64_t* offsets,
               int64_t batch, int64_t total_rows, float* X_tilde, float* mass, void* workspace,
-              size_t workspace_bytes, void* stream, Phase phase) {
+              size_t workspace_bytes, void* stream, Phase phase, bool keep_flags = false) {
   if (q == nullptr) return SA_ERR_INVALID_ARG;
   if (batch < 0 || total_rows < 0 || total_rows > kMaxRows) return SA_ERR_INVALID_ARG;
   if (batch == 0) return total_rows == 0 ? SA_OK : SA_ERR_INVALID_ARG;
@@ -147,6 +150,7 @@ sa_status run(sa_query q, const float* queries, const void* X, const int64_t* of
   a.part_m = reinterpret_cast<float*>(ws + l.part_m_off);
   a.header = reinterpret_cast<sa::WsHeader*>(ws);
   a.user_queries = user_q ? 1 : 0;
+  a.keep_flags = keep_flags ? 1 : 0;
   const int G = static_cast<int>(grid_for(q, total_rows));
 
   if (phase != Phase::kFinalize) {
@@ -416,6 +420,94 @@ sa_status sa_sketch_forward_host(sa_query q, const void* X_host, const int64_t* 
       cudaMemcpyAsync(mass_host, m_dev, m_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return SA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return SA_ERR_CUDA;
+  return SA_OK;
+}
+
+size_t sa_workspace_bytes_refine_layer(sa_query q, int64_t batch, int64_t total_rows) {
+  if (q == nullptr || batch < 0 || total_rows < 0) return 0;
+  const size_t kd = static_cast<size_t>(q->k) * q->d;
+  return round_up(ws_layout(q, total_rows).total + uq_bytes(q, batch), 256) +
+         round_up(static_cast<size_t>(batch) * kd * sizeof(float), 256) +
+         round_up(static_cast<size_t>(batch) * q->k * sizeof(float), 256);
+}
+
+namespace {
+
+// One refinement layer: the SA step (shared query when prev is null, else
+// per-user queries prev) into the workspace, then the update into out.
+sa_status refine_layer(sa_query q, sa_refine r, const float* prev, const float* P_f32,
+                       const void* X, const int64_t* offsets, int64_t batch, int64_t total_rows,
+                       float* out, void* workspace, size_t workspace_bytes, void* stream,
+                       bool keep_flags) {
+  if (q == nullptr || r == nullptr || out == nullptr) return SA_ERR_INVALID_ARG;
+  if (q->dtype != SA_BF16) return SA_ERR_UNSUPPORTED;
+  if (sa::refine_width(r) != q->d) return SA_ERR_INVALID_ARG;
+  if (prev == nullptr && P_f32 == nullptr) return SA_ERR_INVALID_ARG;
+  if (batch < 0 || total_rows < 0) return SA_ERR_INVALID_ARG;
+  if (batch == 0) return total_rows == 0 ? SA_OK : SA_ERR_INVALID_ARG;
+  if (!aligned(out, 16) || !aligned(prev, 16) || !aligned(P_f32, 16) || !aligned(workspace, 256))
+    return SA_ERR_INVALID_ARG;
+  if (workspace == nullptr) return SA_ERR_INVALID_ARG;
+  if (workspace_bytes < sa_workspace_bytes_refine_layer(q, batch, total_rows))
+    return SA_ERR_WORKSPACE;
+  const size_t kd = static_cast<size_t>(q->k) * q->d;
+  const size_t sa_bytes = round_up(ws_layout(q, total_rows).total + uq_bytes(q, batch), 256);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* xt = reinterpret_cast<float*>(ws + sa_bytes);
+  float* m = reinterpret_cast<float*>(ws + sa_bytes +
+                                      round_up(static_cast<size_t>(batch) * kd * sizeof(float), 256));
+  sa_status s = run(q, prev, X, offsets, batch, total_rows, xt, m, workspace, sa_bytes, stream,
+                    Phase::kBoth, keep_flags);
+  if (s != SA_OK) return s;
+  sa::WsHeader* hdr = reinterpret_cast<sa::WsHeader*>(ws);
+  return sa::launch_refine_update(r, prev != nullptr ? prev : P_f32, prev == nullptr, xt, m,
+                                  batch, q->k, out, &hdr->timeout_flags,
+                                  static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SA_OK
+             : SA_ERR_CUDA;
+}
+
+}  // namespace
+
+sa_status sa_refine_layer_forward(sa_query q, sa_refine r, const float* prev, const float* P_f32,
+                                  const void* X, const int64_t* offsets, int64_t batch,
+                                  int64_t total_rows, float* out, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  return refine_layer(q, r, prev, P_f32, X, offsets, batch, total_rows, out, workspace,
+                      workspace_bytes, stream, false);
+}
+
+size_t sa_workspace_bytes_refine_stack(sa_query q, int64_t batch, int64_t total_rows) {
+  if (q == nullptr || batch < 0 || total_rows < 0) return 0;
+  return sa_workspace_bytes_refine_layer(q, batch, total_rows) +
+         round_up(static_cast<size_t>(batch) * q->k * q->d * sizeof(float), 256);
+}
+
+sa_status sa_refine_stack_forward(int layers, const sa_query* qs, const sa_refine* rs,
+                                  const float* P_f32, const void* X, const int64_t* offsets,
+                                  int64_t batch, int64_t total_rows, float* out, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (layers < 1 || qs == nullptr || rs == nullptr || P_f32 == nullptr) return SA_ERR_INVALID_ARG;
+  for (int l = 0; l < layers; ++l) {
+    if (qs[l] == nullptr || rs[l] == nullptr) return SA_ERR_INVALID_ARG;
+    if (qs[l]->k != qs[0]->k || qs[l]->d != qs[0]->d) return SA_ERR_INVALID_ARG;
+  }
+  if (batch == 0) return total_rows == 0 ? SA_OK : SA_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < sa_workspace_bytes_refine_stack(qs[0], batch, total_rows))
+    return SA_ERR_WORKSPACE;
+  // Layer outputs alternate between `out` and a buffer after the layer
+  // workspace, so that the last layer writes `out` and no layer writes the
+  // sketches it is queried with.
+  const size_t layer_bytes = sa_workspace_bytes_refine_layer(qs[0], batch, total_rows);
+  float* tmp = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + layer_bytes);
+  const float* prev = nullptr;
+  for (int l = 0; l < layers; ++l) {
+    float* dst = ((layers - 1 - l) % 2 == 0) ? out : tmp;
+    const sa_status s = refine_layer(qs[l], rs[l], prev, P_f32, X, offsets, batch, total_rows, dst,
+                                     workspace, layer_bytes, stream, l > 0);
+    if (s != SA_OK) return s;
+    prev = dst;
+  }
   return SA_OK;
 }
 

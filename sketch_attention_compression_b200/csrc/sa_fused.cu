@@ -166,8 +166,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Every CTA of the launch has the same layout and takes this path, so
     // block 0 alone reports it (clearing the previous call's offset bits).
     if (blockIdx.x == 0 && threadIdx.x == 0) {
-      a.header->flags = 0u;
-      a.header->timeout_flags = DEVFLAG_SMEM_ALIGN;
+      if (a.keep_flags) {
+        atomicOr(&a.header->timeout_flags, DEVFLAG_SMEM_ALIGN);
+      } else {
+        a.header->flags = 0u;
+        a.header->timeout_flags = DEVFLAG_SMEM_ALIGN;
+      }
     }
     return;
   }
@@ -255,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The device flags of this call start clear.  This is block 0's first
   // global access: the preceding kernel's writes are visible, and any other
   // CTA can set a flag only after a bounded wait has run out (seconds).
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
+  if (blockIdx.x == 0 && threadIdx.x == 0 && !a.keep_flags) {
     a.header->flags = 0u;
     a.header->timeout_flags = 0u;
   }

@@ -107,8 +107,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   // out).  Every CTA has the same shared-memory layout, so on misalignment
   // all of them stop here and block 0 alone reports it.
   if (blockIdx.x == 0 && threadIdx.x == 0) {
-    a.header->flags = 0u;
-    a.header->timeout_flags = aligned ? 0u : DEVFLAG_SMEM_ALIGN;
+    if (!a.keep_flags) {
+      a.header->flags = 0u;
+      a.header->timeout_flags = aligned ? 0u : DEVFLAG_SMEM_ALIGN;
+    } else if (!aligned) {
+      atomicOr(&a.header->timeout_flags, DEVFLAG_SMEM_ALIGN);
+    }
   }
   if (aligned && threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }

@@ -187,7 +187,16 @@ struct PassArgs {
   // (the tensor-core pass reads rows b * k_pad.. of its Q' tensor map, the
   // fp32 pass the k x d block at b * k * d).
   int user_queries;
+  // 1: leave the header's flag words as they are (a later layer of a stacked
+  // call, which adds its flags to the earlier layers'); 0: clear them.
+  int keep_flags;
 };
+
+// 2-D bf16 tensor map over a row-major [rows][cols] array: boxes of 64
+// columns (128 bytes) x box_rows rows, 128-byte swizzle, zero fill.  False if
+// the driver's encoder is unavailable or rejects the shape.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows);
 
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error.
@@ -239,5 +248,21 @@ cudaError_t launch_simt_fp32(const float* q_f32, const float* X, const PassArgs&
 // Fixed-order reduction of split users, zero-fill of empty users, offset
 // validation.  Launched with programmatic stream serialization.
 cudaError_t launch_finalize(const PassArgs& a, int grid_ctas, cudaStream_t stream);
+
+}  // namespace sa
+
+struct sa_refine_s;
+
+namespace sa {
+
+// The update of a refinement layer after its SA step (sa_refine.cu):
+// out = LN2(z + FFN(z)), z = LN1(prev + x_tilde / mass), for batch * k rows;
+// prev is k x d shared by every user when prev_shared.  Timeouts are OR-ed
+// into *flags (may be null).
+cudaError_t launch_refine_update(const sa_refine_s* r, const float* prev, bool prev_shared,
+                                 const float* x_tilde, const float* mass, int64_t batch, int k,
+                                 float* out, uint32_t* flags, cudaStream_t st);
+// Feature width d of a refinement handle.
+int refine_width(const sa_refine_s* r);
 
 }  // namespace sa

@@ -46,7 +46,10 @@ __global__ void __launch_bounds__(kThreadsSimt)
   const int64_t N = a.total_rows;
   // The device flags of this call start clear (block 0's first global
   // access; this pass sets no flag itself).
-  if (c == 0 && blockIdx.y == 0 && tid == 0) { a.header->flags = 0u; a.header->timeout_flags = 0u; }
+  if (c == 0 && blockIdx.y == 0 && tid == 0 && !a.keep_flags) {
+    a.header->flags = 0u;
+    a.header->timeout_flags = 0u;
+  }
   const int64_t R0 = range_begin(a.offsets, a.batch, N, c, G);
   const int64_t R1 = range_begin(a.offsets, a.batch, N, c + 1, G);
   if (a.batch == 0 || R0 >= R1) return;

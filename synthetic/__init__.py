@@ -29,6 +29,7 @@ from .workloads import (  # noqa: F401
     generate,
     round_to_bf16,
     ragged_lengths,
+    refine_params,
     upstream_gradients,
     user_queries,
     workload_lengths,

@@ -213,3 +213,24 @@ def upstream_gradients(batch: int, k: int, d: int, seed: int):
     (batch, k, d) and g = dL/dm (batch, k), float64 ~ N(0, 1)."""
     rng = np.random.default_rng(seed)
     return rng.standard_normal((batch, k, d)), rng.standard_normal((batch, k))
+
+
+def refine_params(d: int, h: int, seed: int, dtype: str = "bf16") -> dict:
+    """Seeded parameters of one refinement layer: W_Q, W_K (d, d) ~ N(0, 1/d)
+    (rounded to bf16 for dtype "bf16", like every SA input), and the LN and
+    FFN parameters in float32: gamma ~ 1 + 0.1 N(0, 1), beta ~ 0.1 N(0, 1),
+    W1, W3 (d, h) ~ N(0, 1/d), W2 (h, d) ~ N(0, 1/h)."""
+    rng = np.random.default_rng(seed)
+    w_sd = np.float32(1.0 / math.sqrt(d))
+    W_Q = rng.standard_normal((d, d), dtype=np.float32) * w_sd
+    W_K = rng.standard_normal((d, d), dtype=np.float32) * w_sd
+    if dtype == "bf16":
+        W_Q, W_K = round_to_bf16(W_Q), round_to_bf16(W_K)
+    out = dict(W_Q=W_Q, W_K=W_K, scale=float(1.0 / math.sqrt(d)))
+    for g, b in (("gamma1", "beta1"), ("gamma2", "beta2")):
+        out[g] = (1.0 + 0.1 * rng.standard_normal(d)).astype(np.float32)
+        out[b] = (0.1 * rng.standard_normal(d)).astype(np.float32)
+    out["W1"] = (rng.standard_normal((d, h)) / math.sqrt(d)).astype(np.float32)
+    out["W3"] = (rng.standard_normal((d, h)) / math.sqrt(d)).astype(np.float32)
+    out["W2"] = (rng.standard_normal((h, d)) / math.sqrt(h)).astype(np.float32)
+    return out

@@ -101,7 +101,7 @@ def _kind(ctype_decl):
     """Coarse class of a C parameter or return type: pointer, 64-bit integer,
     32-bit integer/enum, float, size_t or void."""
     t = " ".join(ctype_decl.replace("*", " * ").split())
-    if "*" in t or t.startswith("sa_query"):
+    if "*" in t or t.startswith("sa_query") or t.startswith("sa_refine"):
         return "ptr"
     if "int64_t" in t:
         return "i64"
@@ -141,3 +141,27 @@ def test_binding_signatures_match_header():
         want = [_kind(p) for p in ptypes]
         assert got == want, f"{name}: binding {got} vs header {want}"
         assert _ctypes_kind(res) == _kind(ret), f"{name}: return {res} vs {ret}"
+
+
+def test_refine_entry_points_reject_bad_arguments_on_the_host(lib):
+    """The refinement entry points check their arguments before touching the
+    device (null handles and pointers, unsupported widths)."""
+    out = ctypes.c_void_p()
+    dummy = ctypes.c_void_p(256)
+    args7 = [dummy] * 7
+    assert lib.sa_prepare_refine(*args7, 128, 512, None, None) == binding.SA_ERR_INVALID_ARG
+    assert lib.sa_prepare_refine(None, *args7[1:], 128, 512, None, ctypes.byref(out)) == \
+        binding.SA_ERR_INVALID_ARG
+    for d, h, want in [(128, 100, binding.SA_ERR_INVALID_ARG), (128, 64, binding.SA_ERR_INVALID_ARG),
+                       (96, 128, binding.SA_ERR_INVALID_ARG), (256, 128, binding.SA_ERR_UNSUPPORTED)]:
+        assert lib.sa_prepare_refine(*args7, d, h, None, ctypes.byref(out)) == want
+        assert out.value is None
+    lib.sa_refine_free(None)  # NULL-safe
+    assert lib.sa_refine_update(None, dummy, 0, dummy, dummy, 1, 4, dummy, None, None) == \
+        binding.SA_ERR_INVALID_ARG
+    assert lib.sa_refine_layer_forward(None, None, None, None, None, None, 1, 1, None, None, 0,
+                                       None) == binding.SA_ERR_INVALID_ARG
+    assert lib.sa_refine_stack_forward(0, None, None, None, None, None, 1, 1, None, None, 0,
+                                       None) == binding.SA_ERR_INVALID_ARG
+    assert lib.sa_workspace_bytes_refine_layer(None, 1, 1) == 0
+    assert lib.sa_workspace_bytes_refine_stack(None, 1, 1) == 0
