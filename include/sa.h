@@ -280,6 +280,48 @@ sa_status sa_mass_normalise(const float* X_tilde, const float* mass, int64_t bat
                             float* out, void* stream);
 
 /*
+ * sa_sketch_backward -- gradients of one SA layer (section 2.2 of the notes:
+ * the compression module is trained end to end by the ranking loss; the
+ * page prints no backward, so these follow from section 2.1's forward by
+ * the chain rule).  For upstream gradients G_b = dL/dX~_b and g_b = dL/dm_b:
+ *
+ *     dA  = G X^T + g 1^T,   dS = A * (dA - 1 c^T),  c_i = sum_j A_ji dA_ji
+ *     dX  = A^T G + dS^T Q'              (Q' = P W_Q W_K^T * scale)
+ *     R   = dS X,   dP = scale R W_K W_Q^T,
+ *     dW_Q = scale P^T R W_K,   dW_K = scale R^T P W_Q
+ *
+ * One tcgen05 pass over X recomputes the softmax per 128-row tile (no saved
+ * activations), writes dX and accumulates R per user; small GEMMs turn R
+ * into the parameter gradients.
+ *
+ *   q           prepared bf16 query with d in {64, 128} and k <= 128
+ *               (others: SA_ERR_UNSUPPORTED)
+ *   queries     device B x k x d fp32 (per-user queries, as for
+ *               sa_sketch_forward_user_queries) or NULL (the shared P)
+ *   P_f32       device k x d fp32: the prototypes q was prepared with (read
+ *               only when queries is NULL)
+ *   W_Q_f32, W_K_f32   device d x d fp32: the projections q was prepared with
+ *   X, offsets, batch, total_rows   as for sa_sketch_forward
+ *   G           device B x k x d fp32: dL/dX~
+ *   g           device B x k fp32: dL/dm, or NULL (zero)
+ *   dX          device out, total_rows x d bf16 (16-byte aligned)
+ *   dP          device out, k x d fp32 summed over users (shared P), or
+ *               B x k x d fp32 per user (with queries: dL/dQ_b)
+ *   dW_Q, dW_K  device out, d x d fp32, summed over users
+ *   workspace   device, >= sa_workspace_bytes_backward(q, B, N) bytes,
+ *               256-byte aligned; one call at a time
+ *
+ * Device flags (bad offsets, timeouts) are read with sa_read_device_status
+ * on the workspace.  Rows of empty users contribute nothing.
+ */
+size_t sa_workspace_bytes_backward(sa_query q, int64_t batch, int64_t total_rows);
+sa_status sa_sketch_backward(sa_query q, const float* queries, const float* P_f32,
+                             const float* W_Q_f32, const float* W_K_f32, const void* X,
+                             const int64_t* offsets, int64_t batch, int64_t total_rows,
+                             const float* G, const float* g, void* dX, float* dP, float* dW_Q,
+                             float* dW_K, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Stacked refinement layers (section 2.2 "Stacked Refinement" of the same
  * notes).  Layer l queries the ORIGINAL history X with the previous layer's
  * sketches (layer 1 with the shared prototypes: X~^(0) = P^(0)) and then

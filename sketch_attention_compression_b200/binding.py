@@ -45,6 +45,9 @@ SIGNATURES = {
     "sa_status_string": (ctypes.c_char_p, [_i32]),
     "sa_query_info": (_i32, [_vp, ctypes.POINTER(_i32), ctypes.POINTER(_i32),
                              ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
+    "sa_workspace_bytes_backward": (_sz, [_vp, _i64, _i64]),
+    "sa_sketch_backward": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp,
+                                  _vp, _vp, _vp, _vp, _sz, _vp]),
     "sa_prepare_refine": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp,
                                  ctypes.POINTER(_vp)]),
     "sa_refine_free": (None, [_vp]),
@@ -304,6 +307,36 @@ class SketchQuery:
             int(device_buffer.numel()), ctypes.c_void_p(_stream_handle(stream)))
         _check(st, "sa_sketch_forward_host")
         return out_x, out_m
+
+    def backward(self, X, offsets, G, g=None, P_f32=None, W_Q_f32=None, W_K_f32=None,
+                 queries=None, workspace=None, stream=None):
+        """Gradients of the layer (sa_sketch_backward) for upstream G = dL/dX~
+        (B, k, d) and g = dL/dm (B, k) or None.  P_f32 (shared queries) or
+        queries (B, k, d), and W_Q_f32, W_K_f32 are the fp32 values the query
+        was prepared with.  Returns dict(dX (N, d) bf16, dP (k, d) or
+        dQueries (B, k, d), dW_Q, dW_K (d, d)) and the workspace."""
+        torch = _torch()
+        B, N = int(offsets.shape[0]) - 1, int(X.shape[0])
+        dX = torch.empty((N, self.d), dtype=torch.bfloat16, device=X.device)
+        dP = torch.empty((self.k, self.d) if queries is None else (B, self.k, self.d),
+                         dtype=torch.float32, device=X.device)
+        dWQ = torch.empty((self.d, self.d), dtype=torch.float32, device=X.device)
+        dWK = torch.empty_like(dWQ)
+        if workspace is None:
+            workspace = torch.empty(int(self._lib.sa_workspace_bytes_backward(self._h, B, N)),
+                                    dtype=torch.uint8, device=X.device)
+        opt = lambda t, n: _dev_ptr(t, n) if t is not None else ctypes.c_void_p(0)  # noqa: E731
+        _check(self._lib.sa_sketch_backward(
+            self._h, opt(queries, "queries"), opt(P_f32, "P_f32"), _dev_ptr(W_Q_f32, "W_Q_f32"),
+            _dev_ptr(W_K_f32, "W_K_f32"), ctypes.c_void_p(X.data_ptr() if N > 0 else 0),
+            _dev_ptr(offsets, "offsets"), B, N, _dev_ptr(G, "G"), opt(g, "g"),
+            ctypes.c_void_p(dX.data_ptr() if N > 0 else 0), _dev_ptr(dP, "dP"),
+            _dev_ptr(dWQ, "dW_Q"), _dev_ptr(dWK, "dW_K"), _dev_ptr(workspace, "workspace"),
+            int(workspace.numel() * workspace.element_size()),
+            ctypes.c_void_p(_stream_handle(stream))), "sa_sketch_backward")
+        out = dict(dX=dX, dW_Q=dWQ, dW_K=dWK)
+        out["dP" if queries is None else "dQueries"] = dP
+        return out, workspace
 
     def close(self) -> None:
         if getattr(self, "_h", None):

@@ -18,6 +18,7 @@ struct sa_query_s {
   int d;
   int k_pad;  // prototype rows of the bf16 Q' copy (multiple of 64), 0 for fp32
   sa_dtype dtype;
+  double scale;      // affinity scale the query was prepared with
   float* q_f32;      // [k][d]
   uint16_t* q_bf16;  // [k_pad][d], rows >= k zero
   float* m_f32;      // [d][d]: W_Q W_K^T * scale * log2(e), for per-user queries
@@ -270,6 +271,7 @@ sa_status sa_prepare_query(const void* P, const void* W_Q, const void* W_K, int 
   q->d = d;
   q->k_pad = k_pad;
   q->dtype = dtype;
+  q->scale = static_cast<double>(scale);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   bool ok = cudaMalloc(&q->q_f32, static_cast<size_t>(k) * d * sizeof(float)) == cudaSuccess;
   if (ok && dtype == SA_BF16) {
@@ -509,6 +511,138 @@ sa_status sa_refine_stack_forward(int layers, const sa_query* qs, const sa_refin
     prev = dst;
   }
   return SA_OK;
+}
+
+namespace {
+
+struct BwdLayout {
+  size_t gb, gp, r, m, rs, tmp, t, uq, total;
+};
+
+BwdLayout bwd_layout(const sa_query_s* q, int64_t batch, int64_t total_rows) {
+  const size_t B = static_cast<size_t>(batch), k = q->k, d = q->d, kp = q->k_pad;
+  BwdLayout l;
+  l.gb = round_up(ws_layout(q, total_rows).total, 256);
+  l.gp = l.gb + round_up(B * kp * d * 2, 256);
+  l.r = l.gp + round_up(B * kp * 4, 256);
+  l.m = l.r + round_up(B * k * d * 4, 256);
+  l.rs = l.m + round_up(B * k * 4, 256);
+  l.tmp = l.rs + round_up(k * d * 4, 256);
+  l.t = l.tmp + round_up(B * k * d * 4, 256);
+  l.uq = l.t + round_up(d * d * 4, 256);
+  l.total = l.uq + round_up(B * kp * d * 2, 256);
+  return l;
+}
+
+}  // namespace
+
+size_t sa_workspace_bytes_backward(sa_query q, int64_t batch, int64_t total_rows) {
+  if (q == nullptr || batch < 0 || total_rows < 0) return 0;
+  return bwd_layout(q, batch, total_rows).total;
+}
+
+sa_status sa_sketch_backward(sa_query q, const float* queries, const float* P_f32,
+                             const float* W_Q_f32, const float* W_K_f32, const void* X,
+                             const int64_t* offsets, int64_t batch, int64_t total_rows,
+                             const float* G, const float* g, void* dX, float* dP, float* dW_Q,
+                             float* dW_K, void* workspace, size_t workspace_bytes, void* stream) {
+  if (q == nullptr) return SA_ERR_INVALID_ARG;
+  if (q->dtype != SA_BF16 || q->ncl > 1 || !sa::backward_supported(q->d, q->k_pad))
+    return SA_ERR_UNSUPPORTED;
+  if (batch < 0 || total_rows < 0 || total_rows > kMaxRows) return SA_ERR_INVALID_ARG;
+  if (batch == 0) return total_rows == 0 ? SA_OK : SA_ERR_INVALID_ARG;
+  const bool user_q = queries != nullptr;
+  if (offsets == nullptr || G == nullptr || dP == nullptr || dW_Q == nullptr || dW_K == nullptr ||
+      W_Q_f32 == nullptr || W_K_f32 == nullptr || workspace == nullptr ||
+      (!user_q && P_f32 == nullptr) || (total_rows > 0 && (X == nullptr || dX == nullptr)))
+    return SA_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(dX, 16) || !aligned(offsets, 8) || !aligned(workspace, 256) ||
+      !aligned(G, 4) || !aligned(g, 4) || !aligned(queries, 4) || !aligned(P_f32, 4) ||
+      !aligned(W_Q_f32, 4) || !aligned(W_K_f32, 4) || !aligned(dP, 4) || !aligned(dW_Q, 4) ||
+      !aligned(dW_K, 4))
+    return SA_ERR_INVALID_ARG;
+  if (!same_device(q)) return SA_ERR_INVALID_ARG;
+  if (user_q && batch > (int64_t{1} << 31) / q->k_pad - 1) return SA_ERR_INVALID_ARG;
+  const BwdLayout l = bwd_layout(q, batch, total_rows);
+  if (workspace_bytes < l.total) return SA_ERR_WORKSPACE;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const WsLayout wl = ws_layout(q, total_rows);
+  uint16_t* gb = reinterpret_cast<uint16_t*>(ws + l.gb);
+  float* gp = reinterpret_cast<float*>(ws + l.gp);
+  float* R = reinterpret_cast<float*>(ws + l.r);
+  float* m = reinterpret_cast<float*>(ws + l.m);
+  float* Rs = reinterpret_cast<float*>(ws + l.rs);
+  float* tmp = reinterpret_cast<float*>(ws + l.tmp);
+  float* T = reinterpret_cast<float*>(ws + l.t);
+  uint16_t* uq = reinterpret_cast<uint16_t*>(ws + l.uq);
+  const int k = q->k, d = q->d, kp = q->k_pad;
+
+  PassArgs a;
+  a.offsets = offsets;
+  a.batch = batch;
+  a.total_rows = total_rows;
+  a.tiles = sa::tiles_of(total_rows);
+  a.k = k;
+  a.d = d;
+  a.out_x = R;
+  a.out_m = m;
+  a.part_x = reinterpret_cast<float*>(ws + wl.part_x_off);
+  a.part_m = reinterpret_cast<float*>(ws + wl.part_m_off);
+  a.header = reinterpret_cast<sa::WsHeader*>(ws);
+  a.user_queries = user_q ? 1 : 0;
+  a.keep_flags = 0;
+  const int Gr = static_cast<int>(grid_for(q, total_rows));
+
+  if (sa::launch_bwd_prep(G, g, batch, k, kp, d, gb, gp, st) != cudaSuccess) return SA_ERR_CUDA;
+  if (user_q && sa::launch_user_query(queries, q->m_f32, batch, k, kp, d, nullptr, uq, st) !=
+                    cudaSuccess)
+    return SA_ERR_CUDA;
+  CUtensorMap tmx, tmg, tmq;
+  const bool ok_maps =
+      (total_rows > 0 ? make_tmap_bf16(&tmx, X, static_cast<uint64_t>(total_rows),
+                                       static_cast<uint64_t>(d), sa::kTileRows)
+                      : make_tmap_bf16(&tmx, q->q_bf16, static_cast<uint64_t>(kp),
+                                       static_cast<uint64_t>(d), 64)) &&
+      make_tmap_bf16(&tmg, gb, static_cast<uint64_t>(batch) * kp, static_cast<uint64_t>(d),
+                     static_cast<uint32_t>(kp)) &&
+      (!user_q || make_tmap_bf16(&tmq, uq, static_cast<uint64_t>(batch) * kp,
+                                 static_cast<uint64_t>(d), static_cast<uint32_t>(kp)));
+  if (!ok_maps) return SA_ERR_CUDA;
+  if (sa::launch_backward(tmx, user_q ? tmq : q->tmap_q, tmg, kp, a, gp,
+                          static_cast<uint16_t*>(dX), Gr, st) != cudaSuccess ||
+      sa::launch_finalize(a, Gr, st) != cudaSuccess)
+    return SA_ERR_CUDA;
+
+  // Parameter gradients from R = ln 2 dL/dQ' (Q' = scale P W_Q W_K^T):
+  //   dP = c R W_K W_Q^T,  dW_Q = c P^T R W_K,  dW_K = c R^T P W_Q,  c = scale log2 e,
+  // summed over users for shared P, per user (dQ_b) with per-user queries.
+  const double cgrad = q->scale / 0.6931471805599453;
+  const int64_t kd = static_cast<int64_t>(k) * d;
+  bool ok = true;
+  if (!user_q) {
+    ok = sa::launch_sum_users(R, batch, kd, Rs, st) == cudaSuccess &&
+         sa::launch_bwd_gemm(Rs, 0, false, W_K_f32, 0, false, tmp, 0, k, d, d, 1.0, false, 1, st) ==
+             cudaSuccess &&
+         sa::launch_bwd_gemm(tmp, 0, false, W_Q_f32, 0, true, dP, 0, k, d, d, cgrad, false, 1, st) ==
+             cudaSuccess &&
+         sa::launch_bwd_gemm(P_f32, 0, true, Rs, 0, false, T, 0, d, d, k, 1.0, false, 1, st) ==
+             cudaSuccess;
+  } else {
+    ok = sa::launch_bwd_gemm(R, kd, false, W_K_f32, 0, false, tmp, kd, k, d, d, 1.0, false, batch,
+                             st) == cudaSuccess &&
+         sa::launch_bwd_gemm(tmp, kd, false, W_Q_f32, 0, true, dP, kd, k, d, d, cgrad, false, batch,
+                             st) == cudaSuccess &&
+         sa::launch_bwd_gemm(queries, 0, true, R, 0, false, T, 0, d, d,
+                             static_cast<int>(batch * k), 1.0, false, 1, st) == cudaSuccess;
+  }
+  ok = ok &&
+       sa::launch_bwd_gemm(T, 0, false, W_K_f32, 0, false, dW_Q, 0, d, d, d, cgrad, false, 1, st) ==
+           cudaSuccess &&
+       sa::launch_bwd_gemm(T, 0, true, W_Q_f32, 0, false, dW_K, 0, d, d, d, cgrad, false, 1, st) ==
+           cudaSuccess;
+  return ok ? SA_OK : SA_ERR_CUDA;
 }
 
 sa_status sa_read_device_status(void* workspace, size_t workspace_bytes, void* stream,

@@ -265,4 +265,27 @@ cudaError_t launch_refine_update(const sa_refine_s* r, const float* prev, bool p
 // Feature width d of a refinement handle.
 int refine_width(const sa_refine_s* r);
 
+// Backward pass (sa_backward.cu).  launch_backward runs the per-tile kernel:
+// dX (bf16) for every row, and R_b = ln 2 * dL/dQ' for every user into
+// p.out_x (users inside one CTA range) or p.part_x (split users; the finalize
+// pass sums them).  tmap_q reads k_pad-row boxes of Q'' (shared) or of the
+// per-call Q''_b array (p.user_queries); tmap_g reads k_pad-row boxes of
+// G_b (bf16, batch * k_pad x d); g_pad is batch x k_pad fp32.
+bool backward_supported(int d, int k_pad);
+cudaError_t launch_backward(const CUtensorMap& tx, const CUtensorMap& tq, const CUtensorMap& tg,
+                            int k_pad, const PassArgs& p, const float* g_pad, uint16_t* dX,
+                            int grid, cudaStream_t st);
+// G (batch x k x d) -> bf16 batch x k_pad x d (zero rows past k); g -> fp32
+// batch x k_pad (zeros past k, or everywhere when g is null).
+cudaError_t launch_bwd_prep(const float* G, const float* g, int64_t batch, int k, int km, int d,
+                            uint16_t* Gb, float* gp, cudaStream_t st);
+// out = sum over `batch` consecutive blocks of n floats of R.
+cudaError_t launch_sum_users(const float* R, int64_t batch, int64_t n, float* out,
+                             cudaStream_t st);
+// C[b] = alpha op(A[b]) op(B[b]) (+ C[b]), row-major, fp64 accumulation, for
+// b < batch (strides sa, sb, sc in floats).
+cudaError_t launch_bwd_gemm(const float* A, int64_t sa, bool ta, const float* B, int64_t sb,
+                            bool tb, float* C, int64_t sc, int m, int n, int l, double alpha,
+                            bool accumulate, int64_t batch, cudaStream_t st);
+
 }  // namespace sa

@@ -165,3 +165,11 @@ def test_refine_entry_points_reject_bad_arguments_on_the_host(lib):
                                        None) == binding.SA_ERR_INVALID_ARG
     assert lib.sa_workspace_bytes_refine_layer(None, 1, 1) == 0
     assert lib.sa_workspace_bytes_refine_stack(None, 1, 1) == 0
+
+
+def test_backward_rejects_bad_arguments_on_the_host(lib):
+    dummy = ctypes.c_void_p(256)
+    assert lib.sa_sketch_backward(None, None, dummy, dummy, dummy, dummy, dummy, 1, 1, dummy, None,
+                                  dummy, dummy, dummy, dummy, dummy, 1 << 20, None) == \
+        binding.SA_ERR_INVALID_ARG
+    assert lib.sa_workspace_bytes_backward(None, 1, 1) == 0
