@@ -567,6 +567,196 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
     print(json.dumps(line), flush=True)
 
 
+def _timed(fn, steps, dev, stream, ranks):
+    """Mean ms of `steps` back-to-back calls of fn between two CUDA events on
+    `stream`, bracketed by barrier + synchronize; max over ranks."""
+    import torch
+    ranks.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ranks.barrier()
+    return ranks.max(e0.elapsed_time(e1) / steps)
+
+
+def _roofline(bytes_per_launch, flops_per_launch, ms, peaks, peak_kind, kernel, note):
+    t_hbm = bytes_per_launch / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops_per_launch / (peaks["bf16_tflops"] * 1e12)
+    s = ms * 1e-3
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    if bound == "hbm":
+        achieved, peak, unit = bytes_per_launch / s / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved, peak, unit = flops_per_launch / s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": None, "kernel": kernel, "kernel_ms": ms,
+            "roofline_ms": 1e3 * max(t_hbm, t_tc),
+            "tensor_frac": (flops_per_launch / s / 1e12) / peaks["bf16_tflops"],
+            "hbm_frac": (bytes_per_launch / s / 1e9) / peaks["hbm_gbs"],
+            "peak_source": f"MEASURED_PEAKS.json ({peak_kind}, burst)", "algorithmic": note}
+
+
+def run_backward(args, rank, world, local_rank, ranks):
+    """One step = sa_sketch_backward over the batch (upstream gradients G, g
+    seeded), the SA backward of section 2.2's end-to-end training."""
+    import torch
+
+    from sketch_attention_compression_b200 import SketchQuery, load_library, read_device_status
+    from synthetic import upstream_gradients
+    load_library()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOADS[args.workload]
+    inp = workload_inputs(args, seed=rank_seed(args.workload, rank))
+    X = torch.from_numpy(inp["X"]).to(dev).to(torch.bfloat16)
+    P, W_Q, W_K = (torch.from_numpy(inp[k]).to(dev).to(torch.bfloat16) for k in ("P", "W_Q", "W_K"))
+    f32 = {k: torch.from_numpy(inp[k]).to(dev) for k in ("P", "W_Q", "W_K")}
+    offsets = torch.from_numpy(inp["offsets"]).to(dev)
+    B, N = len(inp["offsets"]) - 1, int(inp["offsets"][-1])
+    Gn, gn = upstream_gradients(B, w.k, w.d, seed=rank_seed(args.workload, rank) + 200)
+    G = torch.from_numpy(Gn.astype(np.float32)).to(dev)
+    g = torch.from_numpy(gn.astype(np.float32)).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    q = SketchQuery(P, W_Q, W_K, inp["scale"], stream=stream)
+    _, ws = q.backward(X, offsets, G, g, P_f32=f32["P"], W_Q_f32=f32["W_Q"], W_K_f32=f32["W_K"])
+
+    def step():
+        q.backward(X, offsets, G, g, P_f32=f32["P"], W_Q_f32=f32["W_Q"], W_K_f32=f32["W_K"],
+                   workspace=ws, stream=stream)
+    for _ in range(args.warmup):
+        step()
+    if read_device_status(ws, stream) != 0:
+        raise RuntimeError("device flags raised during warm-up")
+    sampler = None
+    if rank == 0:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        sampler.start()
+        time.sleep(0.05)
+    mark = sampler.mark() if sampler else 0
+    ms = _timed(step, args.steps, dev, stream, ranks)
+    clocks = sampler.summary(mark) if sampler else None
+    if sampler:
+        sampler.stop()
+    if read_device_status(ws, stream) != 0:
+        raise RuntimeError("device flags raised during the timed region")
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    rows_total = ranks.sum(N)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        from oracle import sa_user_backward
+        t0 = time.perf_counter()
+        rows, done = 0, 0
+        offs = inp["offsets"]
+        for b in range(B):
+            lo, hi = int(offs[b]), int(offs[b + 1])
+            sa_user_backward(inp["X"][lo:hi], inp["P"], inp["W_Q"], inp["W_K"], inp["scale"],
+                             Gn[b], gn[b])
+            rows += hi - lo
+            done = b
+            if time.perf_counter() - t0 >= args.cpu_budget:
+                break
+        dt = time.perf_counter() - t0
+        cpu = {"value": rows / dt, "unit": "rows/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"users 0..{done} ({rows} rows, {dt:.1f} s, numpy fp64 sa_user_backward)"}
+    line = {
+        "metric": "SA backward history rows/sec on 1 B200 (dX, dP, dW_Q, dW_K)",
+        "value": rows_total / (ms * 1e-3), "unit": "rows/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "mode": "backward", "users_per_gpu": B,
+                   "rows_per_gpu": N, "d": w.d, "k": w.k, "upstream": "G, g ~ N(0, 1)"},
+        "roofline": _roofline(4.0 * w.d * N, 10.0 * w.k * w.d * N, ms, peaks, peak_kind,
+                              "sa_sketch_backward (prep + backward pass + finalize + GEMMs)",
+                              f"{4 * w.d} B (X read, dX written) and {10 * w.k * w.d} flop "
+                              f"per row x {N} rows"),
+        "clocks": clocks, "cpu_baseline": cpu,
+        "gpu_launches": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_refine(args, rank, world, local_rank, ranks):
+    """One step = sa_refine_stack_forward with --refine-layers layers over the
+    batch (section 2.2's stacked refinement; each layer one SA pass over X
+    plus the LN / SwiGLU update of the B x k sketches)."""
+    import torch
+
+    from sketch_attention_compression_b200 import (RefineParams, SketchQuery, load_library,
+                                                   read_device_status, refine_stack_forward)
+    from synthetic import refine_params
+    load_library()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOADS[args.workload]
+    L, h = args.refine_layers, 4 * w.d
+    inp = workload_inputs(args, seed=rank_seed(args.workload, rank))
+    X = torch.from_numpy(inp["X"]).to(dev).to(torch.bfloat16)
+    offsets = torch.from_numpy(inp["offsets"]).to(dev)
+    B, N = len(inp["offsets"]) - 1, int(inp["offsets"][-1])
+    P = torch.from_numpy(inp["P"]).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    qs, rs = [], []
+    for layer in range(L):
+        p = refine_params(w.d, h, seed=rank_seed(args.workload, rank) + 300 + layer)
+        qs.append(SketchQuery(P.to(torch.bfloat16), torch.from_numpy(p["W_Q"]).to(dev).to(torch.bfloat16),
+                              torch.from_numpy(p["W_K"]).to(dev).to(torch.bfloat16), p["scale"],
+                              stream=stream))
+        t = {key: torch.from_numpy(p[key]).to(dev) for key in ("W1", "W3", "W2", "gamma1", "beta1",
+                                                                 "gamma2", "beta2")}
+        rs.append(RefineParams(t["W1"], t["W3"], t["W2"], t["gamma1"], t["beta1"], t["gamma2"],
+                               t["beta2"], stream=stream))
+    out, ws = refine_stack_forward(qs, rs, P, X, offsets, stream=stream)
+
+    def step():
+        refine_stack_forward(qs, rs, P, X, offsets, out=out, workspace=ws, stream=stream)
+    for _ in range(args.warmup):
+        step()
+    if read_device_status(ws, stream) != 0:
+        raise RuntimeError("device flags raised during warm-up")
+    sampler = None
+    if rank == 0:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        sampler.start()
+        time.sleep(0.05)
+    mark = sampler.mark() if sampler else 0
+    ms = _timed(step, args.steps, dev, stream, ranks)
+    clocks = sampler.summary(mark) if sampler else None
+    if sampler:
+        sampler.stop()
+    if read_device_status(ws, stream) != 0:
+        raise RuntimeError("device flags raised during the timed region")
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    rows_total = ranks.sum(N)
+    flops = L * (4.0 * w.k * w.d * N + 6.0 * h * w.d * B * w.k)
+    line = {
+        "metric": f"SA refinement stack ({L} layers) history rows/sec on 1 B200",
+        "value": rows_total / (ms * 1e-3), "unit": "rows/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "mode": f"refine_stack x{L}", "users_per_gpu": B,
+                   "rows_per_gpu": N, "d": w.d, "k": w.k, "ffn_hidden": h},
+        "roofline": _roofline(L * 2.0 * w.d * N, flops, ms, peaks, peak_kind,
+                              "sa_refine_stack_forward (per layer: SA pass + finalize + update)",
+                              f"per layer {2 * w.d} B and {4 * w.k * w.d} flop per row x {N} rows, "
+                              f"plus 6 h d flop per (user, prototype) row"),
+        "clocks": clocks, "cpu_baseline": None, "gpu_launches": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -579,6 +769,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--user-queries", action="store_true",
                     help="query every user with its own k x d matrix (refinement-layer SA step)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the SA backward pass (sa_sketch_backward) instead")
+    ap.add_argument("--refine-layers", type=int, default=0,
+                    help="time a stack of this many refinement layers instead")
     ap.add_argument("--users", type=int, default=0,
                     help="use only the first U users of the workload (smaller case)")
     args = ap.parse_args()
@@ -601,7 +795,12 @@ def main():
         return
     ranks = init_rank_group(world, local_rank, "nccl")
     try:
-        run_ours(args, rank, world, local_rank, ranks)
+        if args.backward:
+            run_backward(args, rank, world, local_rank, ranks)
+        elif args.refine_layers > 0:
+            run_refine(args, rank, world, local_rank, ranks)
+        else:
+            run_ours(args, rank, world, local_rank, ranks)
     finally:
         if world > 1:
             import torch.distributed as dist

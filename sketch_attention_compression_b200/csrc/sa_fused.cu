@@ -119,6 +119,10 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar, int lane) {
 #endif
 constexpr uint32_t kMma1Lead = SA_MMA1_LEAD;
 
+#ifndef SA_EARLY_TRIGGER
+#define SA_EARLY_TRIGGER 1
+#endif
+
 
 // Bounded wait until the counter `cnt` (a shared-memory word that only
 // grows) reaches `target`; same abort and timeout contract as mbar_wait.
@@ -256,6 +260,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   grid_dependency_wait();
+#if SA_EARLY_TRIGGER
+  // The next kernel in the stream (the finalize pass) may be scheduled as
+  // SMs free up; its own grid_dependency_wait still waits for this pass to
+  // complete, so only its launch overlaps this pass's tail.
+  grid_dependency_launch();
+#endif
   // The device flags of this call start clear.  This is block 0's first
   // global access: the preceding kernel's writes are visible, and any other
   // CTA can set a flag only after a bounded wait has run out (seconds).
