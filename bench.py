@@ -481,6 +481,27 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
     barrier()
     e2e_ms = max_over_ranks(h0.elapsed_time(h1) / e2e_steps)
 
+    # -- region D: sustained, back to back for about args.sustained seconds --
+    sustained = None
+    if args.sustained > 0:
+        mark_d = sampler.mark() if sampler else 0
+        n_sus = max(args.steps, int(args.sustained / max(step_ms * 1e-3, 1e-6)))
+        barrier()
+        torch.cuda.synchronize(dev)
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for i in range(n_sus):
+            step(Xs[i % n_copies])
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        sus_ms = max_over_ranks(s0.elapsed_time(s1) / n_sus)
+        sustained = {"ms_per_step": sus_ms, "steps": n_sus,
+                     "seconds": sus_ms * n_sus * 1e-3,
+                     "value": ranks.sum(N) / (sus_ms * 1e-3),
+                     "clocks": sampler.summary(mark_d) if sampler else None}
+
     if sampler is not None:
         sampler.stop()
         # the kernel-only regions A and B (region C is mostly host copies)
@@ -562,6 +583,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, ranks: RankGroup):
                 "ms_per_step": e2e_ms},
         "gpu_launches": launches,
         "clocks": clocks,
+        "sustained": sustained,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
@@ -769,6 +791,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--user-queries", action="store_true",
                     help="query every user with its own k x d matrix (refinement-layer SA step)")
+    ap.add_argument("--sustained", type=float, default=2.0,
+                    help="seconds of back-to-back whole steps after the timed regions, reported "
+                         "as 'sustained' with their own clocks (0: skip)")
     ap.add_argument("--backward", action="store_true",
                     help="time the SA backward pass (sa_sketch_backward) instead")
     ap.add_argument("--refine-layers", type=int, default=0,
