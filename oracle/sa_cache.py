@@ -22,8 +22,9 @@ Readings where the page is silent:
   C1  an entry is fresh while now - t_insert < ttl (strictly); an expired
       entry is a miss and is dropped when found;
   C2  a lookup that hits refreshes the entry's last-use time; capacity
-      eviction removes, first, expired entries, then the least recently used
-      one (ties: the smaller slot index, i.e. the older allocation);
+      eviction takes a free slot (the smallest index) if there is one, else
+      the expired entry inserted earliest, else the least recently used one
+      (ties: the smaller slot index);
   C3  inserting a key that is present replaces its sketch and resets its
       insertion time; within one batch, a key that appears twice keeps the
       later sketch;
@@ -82,7 +83,7 @@ class SketchCacheModel:
                 return s
         expired = [s for s in range(self.capacity) if not self._fresh(s, now)]
         if expired:
-            s = expired[0]
+            s = min(expired, key=lambda i: (self.t_insert[i], i))
         else:
             s = min(range(self.capacity), key=lambda i: (self.t_use[i], i))
         self._drop(s)

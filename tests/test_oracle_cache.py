@@ -73,6 +73,17 @@ def pin_replace_and_round_trip(model=SketchCacheModel):
     assert c.lookup([_key(1)], 51.0) == [-1]
 
 
+def pin_expired_oldest_first(model=SketchCacheModel):
+    c = model(2, 3, 3, ttl=10.0)
+    c.insert([_key(1)], 2.0, *_sk(1))             # slot 0, inserted at 2
+    c.insert([_key(2)], 0.0, *_sk(2))             # slot 1, inserted at 0
+    c.insert([_key(3)], 5.0, *_sk(3))             # slot 2
+    c.insert([_key(4)], 13.0, *_sk(4))            # keys 1 and 2 expired: key 2 (inserted first) goes
+    got = c.lookup([_key(1), _key(2)], 13.5)
+    assert got[1] == -1
+    assert c.evictions == 1
+
+
 def pin_key_fields(model=SketchCacheModel):
     c = model(2, 3, 8, ttl=50.0)
     c.insert([_key(1)], 0.0, *_sk(1))
@@ -95,7 +106,8 @@ def pin_adapter(adapter=width_adapter):
     assert np.max(np.abs(adapter(X, W) - np.array(want))) < 1e-13
 
 
-CACHE_PINS = [pin_ttl, pin_lru, pin_expired_first, pin_replace_and_round_trip, pin_key_fields]
+CACHE_PINS = [pin_ttl, pin_lru, pin_expired_first, pin_expired_oldest_first,
+              pin_replace_and_round_trip, pin_key_fields]
 
 
 @pytest.mark.parametrize("pin", CACHE_PINS + [pin_adapter], ids=lambda p: p.__name__)
