@@ -428,6 +428,125 @@ sa_status sa_refine_stack_forward(int layers, const sa_query* qs, const sa_refin
                                   int64_t batch, int64_t total_rows, float* out, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/*
+ * Sketch cache (section 2.4 "Local KVCache" of the same notes; section 2.3,
+ * Figure 2: hit -> the stored sketch, miss -> one compression).  Only the
+ * user-side sketch (X~_b and m_b, k x d and k fp32) is stored, keyed by the
+ * user, the model version, the history timestamp and the sketch
+ * configuration, for a time-to-live, in a device pool of `capacity` slots.
+ * Times are seconds on any clock the caller chooses (passed as `now`).
+ *
+ * Decisions (the page names the key, the TTL and capacity eviction and no
+ * more; this is the reading built):
+ *  - an entry is fresh while now - t_insert < ttl; a lookup that finds an
+ *    expired entry counts a miss and drops it;
+ *  - a hit refreshes the entry's last-use time;
+ *  - an insert of a new key takes the free slot with the smallest index,
+ *    else evicts the expired entry inserted earliest, else the least
+ *    recently used entry (ties: the smaller slot);
+ *  - inserting a key that is present replaces its sketch in place and
+ *    restarts its TTL; within one call, of two equal keys the later wins.
+ * The index is host memory guarded by a mutex; the sketches move only on
+ * the device.  Calls on one cache that move data (lookup, insert, forward)
+ * must be ordered with one another by the caller: the library reuses one
+ * device slot list, so use one stream per cache.
+ */
+typedef struct sa_cache_key {
+  int64_t user;
+  int64_t model_version;
+  int64_t history_ts;
+  int64_t config;
+} sa_cache_key;
+
+typedef struct sa_cache_s* sa_cache;
+
+/* A cache of `capacity` sketches of k x d (k >= 1, d >= 4 and a multiple of
+ * 4, capacity >= 1) with a time-to-live of ttl_seconds (> 0).  Allocates
+ * capacity * k * (d + 1) * 4 bytes on the current device.  Errors:
+ * SA_ERR_INVALID_ARG, SA_ERR_CUDA. */
+sa_status sa_cache_create(int k, int d, int64_t capacity, double ttl_seconds, sa_cache* out);
+
+/* Releases the cache and its device memory.  NULL is a no-op. */
+void sa_cache_free(sa_cache c);
+
+/*
+ * sa_cache_lookup -- for each of `batch` keys (host array): hit[b] (host
+ * out) = 1 if a fresh entry exists, else 0; for each hit a kernel on
+ * `stream` copies the entry into X_tilde[b] (device, batch x k x d fp32,
+ * 16-byte aligned) and mass[b] (device, batch x k fp32).  Rows of misses
+ * are left as they were.  The decisions are taken on the host before the
+ * call returns; the copies complete with the stream.
+ */
+sa_status sa_cache_lookup(sa_cache c, const sa_cache_key* keys, int64_t batch, double now,
+                          uint8_t* hit, float* X_tilde, float* mass, void* stream);
+
+/*
+ * sa_cache_insert -- stores X_tilde[b], mass[b] (device, layout as for
+ * lookup) under keys[b] (host) at time `now`, evicting as described above.
+ * The copies are kernels on `stream`; the sources must stay unchanged until
+ * they complete.
+ */
+sa_status sa_cache_insert(sa_cache c, const sa_cache_key* keys, int64_t batch, double now,
+                          const float* X_tilde, const float* mass, void* stream);
+
+/* Host-side counters: entries held, hits, misses (expired ones included),
+ * evictions.  Any pointer may be NULL. */
+sa_status sa_cache_stats(sa_cache c, int64_t* entries, int64_t* hits, int64_t* misses,
+                         int64_t* evictions);
+
+/*
+ * sa_cache_forward -- one SA layer served through the cache: look the keys
+ * up, copy the hits to the outputs, gather the missed users' history rows
+ * into a compact array on the device, run sa_sketch_forward on the misses
+ * only, scatter their sketches to the outputs and insert them.
+ *
+ *   c, q           a cache and a prepared query of the same k and d
+ *   keys           host, batch keys
+ *   offsets_host   host, batch + 1 int64 (validated on the host): the same
+ *                  ragged layout as sa_sketch_forward's device offsets
+ *   X              device, total_rows x d, q's dtype, 16-byte aligned
+ *   X_tilde, mass  device outputs as for sa_sketch_forward
+ *   hit            host out, batch bytes: 1 where the cache served the user
+ *   workspace      device, >= sa_cache_forward_workspace_bytes(q, batch,
+ *                  total_rows), 256-byte aligned; the SA pass's device
+ *                  flags are read with sa_read_device_status on it, as for
+ *                  sa_sketch_forward
+ *
+ * Returns once the host work is done and everything is enqueued on `stream`.
+ */
+size_t sa_cache_forward_workspace_bytes(sa_query q, int64_t batch, int64_t total_rows);
+sa_status sa_cache_forward(sa_cache c, sa_query q, const sa_cache_key* keys, double now,
+                           const void* X, const int64_t* offsets_host, int64_t batch,
+                           int64_t total_rows, float* X_tilde, float* mass, uint8_t* hit,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Width adapter (section 2.3): Y = X~ W_A with W_A in R^{d x D} and no bias,
+ * mapping every sketch row to the ranking model's width (D = 1024 in the
+ * final configuration).  The adapted sketch is shared by a request's targets
+ * but not cached (section 2.4).  One tcgen05 kernel: X~ rounded to bf16,
+ * W_A held as bf16, fp32 accumulation, Y written as bf16.
+ */
+typedef struct sa_adapter_s* sa_adapter;
+
+/* W_A: device, d x D fp32 (4-byte aligned); d 64 or 128; D a positive
+ * multiple of 256.  A kernel on `stream` makes the bf16 copy; W_A may be
+ * freed once the stream has passed this call.  Errors: SA_ERR_INVALID_ARG,
+ * SA_ERR_UNSUPPORTED (not sm_100), SA_ERR_CUDA. */
+sa_status sa_prepare_adapter(const float* W_A, int d, int D, void* stream, sa_adapter* out);
+
+/* Releases an adapter.  NULL is a no-op. */
+void sa_adapter_free(sa_adapter a);
+
+/*
+ * sa_adapter_forward -- Y (device out, rows x D bf16, 16-byte aligned) =
+ * X_tilde (device, rows x d fp32, 16-byte aligned) W_A, for rows = batch * k
+ * sketch rows.  device_flags (device uint32, or NULL): SA_DEVFLAG_TIMEOUT or
+ * SA_DEVFLAG_SMEM_ALIGN is OR-ed in if the kernel gave up.
+ */
+sa_status sa_adapter_forward(sa_adapter a, const float* X_tilde, int64_t rows, void* out,
+                             uint32_t* device_flags, void* stream);
+
 /* Static description of a status code. */
 const char* sa_status_string(sa_status s);
 

@@ -9,9 +9,12 @@ binding (binding.py).  Importing the package does not load the library;
 from .binding import (  # noqa: F401
     SA_BF16,
     SA_FP32,
+    CacheKey,
     RefineParams,
     SAError,
+    SketchCache,
     SketchQuery,
+    WidthAdapter,
     load_library,
     mass_normalise,
     read_device_status,

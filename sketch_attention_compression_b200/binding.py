@@ -23,8 +23,8 @@ DEVFLAG_OFFSET0_NONZERO, DEVFLAG_OFFSETS_DECREASE, DEVFLAG_OFFSET_LAST, DEVFLAG_
     DEVFLAG_SMEM_ALIGN = 1, 2, 4, 8, 16
 
 # name -> (restype, argtypes); mirrors include/sa.h
-_vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, \
-    ctypes.c_float
+_vp, _i32, _i64, _sz, _f32, _f64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, \
+    ctypes.c_size_t, ctypes.c_float, ctypes.c_double
 _FWD_ARGS = [_vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _sz, _vp]
 SIGNATURES = {
     "sa_prepare_query": (_i32, [_vp, _vp, _vp, _i32, _i32, _f32, _i32, _vp,
@@ -58,7 +58,33 @@ SIGNATURES = {
     "sa_workspace_bytes_refine_stack": (_sz, [_vp, _i64, _i64]),
     "sa_refine_stack_forward": (_i32, [_i32, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _sz,
                                        _vp]),
+    "sa_cache_create": (_i32, [_i32, _i32, _i64, _f64, ctypes.POINTER(_vp)]),
+    "sa_cache_free": (None, [_vp]),
+    "sa_cache_lookup": (_i32, [_vp, _vp, _i64, _f64, _vp, _vp, _vp, _vp]),
+    "sa_cache_insert": (_i32, [_vp, _vp, _i64, _f64, _vp, _vp, _vp]),
+    "sa_cache_stats": (_i32, [_vp, _vp, _vp, _vp, _vp]),
+    "sa_cache_forward_workspace_bytes": (_sz, [_vp, _i64, _i64]),
+    "sa_cache_forward": (_i32, [_vp, _vp, _vp, _f64, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _sz,
+                                _vp]),
+    "sa_prepare_adapter": (_i32, [_vp, _i32, _i32, _vp, ctypes.POINTER(_vp)]),
+    "sa_adapter_free": (None, [_vp]),
+    "sa_adapter_forward": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp]),
 }
+
+
+class CacheKey(ctypes.Structure):
+    """sa_cache_key: the cache key of section 2.4 (user, model version,
+    history timestamp, sketch configuration)."""
+    _fields_ = [("user", ctypes.c_int64), ("model_version", ctypes.c_int64),
+                ("history_ts", ctypes.c_int64), ("config", ctypes.c_int64)]
+
+
+def _keys_array(keys):
+    """A ctypes array of CacheKey from a sequence of 4-tuples."""
+    arr = (CacheKey * max(len(keys), 1))()
+    for i, key in enumerate(keys):
+        arr[i] = CacheKey(*(int(x) for x in key))
+    return arr
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -481,3 +507,122 @@ def read_device_status(workspace, stream=None) -> int:
     if st not in (SA_OK, SA_ERR_DEVICE_FLAG):
         _check(st, "sa_read_device_status")
     return int(flags.value)
+
+
+class SketchCache:
+    """A device pool of user sketches with a host index (sa_cache_create):
+    `capacity` entries of (k, d) fp32 sketches plus (k,) masses, a
+    time-to-live of `ttl` seconds.  Keys are 4-tuples (user, model_version,
+    history_ts, config); `now` is the caller's clock in seconds."""
+
+    def __init__(self, k: int, d: int, capacity: int, ttl: float):
+        lib = load_library()
+        handle = ctypes.c_void_p()
+        _check(lib.sa_cache_create(int(k), int(d), int(capacity), float(ttl), ctypes.byref(handle)),
+               "sa_cache_create")
+        self._h, self._lib = handle, lib
+        self.k, self.d, self.capacity, self.ttl = int(k), int(d), int(capacity), float(ttl)
+
+    def lookup(self, keys, now: float, X_tilde, mass, stream=None) -> np.ndarray:
+        """Copies the fresh entries into X_tilde[b], mass[b]; returns the hit
+        mask (bool, one per key)."""
+        B = len(keys)
+        hit = np.zeros(max(B, 1), dtype=np.uint8)
+        _check(self._lib.sa_cache_lookup(
+            self._h, ctypes.cast(_keys_array(keys), ctypes.c_void_p), B, float(now),
+            hit.ctypes.data_as(ctypes.c_void_p), _dev_ptr(X_tilde, "X_tilde"), _dev_ptr(mass, "mass"),
+            ctypes.c_void_p(_stream_handle(stream))), "sa_cache_lookup")
+        return hit[:B].astype(bool)
+
+    def insert(self, keys, now: float, X_tilde, mass, stream=None) -> None:
+        _check(self._lib.sa_cache_insert(
+            self._h, ctypes.cast(_keys_array(keys), ctypes.c_void_p), len(keys), float(now),
+            _dev_ptr(X_tilde, "X_tilde"), _dev_ptr(mass, "mass"),
+            ctypes.c_void_p(_stream_handle(stream))), "sa_cache_insert")
+
+    def stats(self) -> dict:
+        vals = [ctypes.c_int64(0) for _ in range(4)]
+        _check(self._lib.sa_cache_stats(self._h, *(ctypes.byref(v) for v in vals)), "sa_cache_stats")
+        return dict(zip(("entries", "hits", "misses", "evictions"), (v.value for v in vals)))
+
+    def forward(self, query: "SketchQuery", keys, now: float, X, offsets_host: np.ndarray,
+                X_tilde=None, mass=None, workspace=None, stream=None):
+        """One SA layer through the cache (sa_cache_forward).  offsets_host is
+        an int64 numpy array (batch + 1).  Returns (X_tilde, mass, hit mask,
+        workspace)."""
+        torch = _torch()
+        offsets_host = np.ascontiguousarray(offsets_host, dtype=np.int64)
+        B, N = int(offsets_host.shape[0]) - 1, int(X.shape[0])
+        if len(keys) != B:
+            raise ValueError("one key per user")
+        if X_tilde is None:
+            X_tilde = torch.empty((B, self.k, self.d), dtype=torch.float32, device=X.device)
+        if mass is None:
+            mass = torch.empty((B, self.k), dtype=torch.float32, device=X.device)
+        if workspace is None:
+            workspace = torch.empty(int(self._lib.sa_cache_forward_workspace_bytes(query._h, B, N)),
+                                    dtype=torch.uint8, device=X.device)
+        hit = np.zeros(max(B, 1), dtype=np.uint8)
+        _check(self._lib.sa_cache_forward(
+            self._h, query._h, ctypes.cast(_keys_array(keys), ctypes.c_void_p), float(now),
+            ctypes.c_void_p(X.data_ptr() if N > 0 else 0),
+            offsets_host.ctypes.data_as(ctypes.c_void_p), B, N, _dev_ptr(X_tilde, "X_tilde"),
+            _dev_ptr(mass, "mass"), hit.ctypes.data_as(ctypes.c_void_p),
+            _dev_ptr(workspace, "workspace"), int(workspace.numel() * workspace.element_size()),
+            ctypes.c_void_p(_stream_handle(stream))), "sa_cache_forward")
+        return X_tilde, mass, hit[:B].astype(bool), workspace
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self._lib.sa_cache_free(self._h)
+            self._h = None
+
+    def __del__(self):  # pragma: no cover
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class WidthAdapter:
+    """Y = X~ W_A on the tensor cores (sa_prepare_adapter): W_A is a (d, D)
+    fp32 CUDA tensor; the output is bf16."""
+
+    def __init__(self, W_A, stream=None):
+        torch = _torch()
+        lib = load_library()
+        if W_A.dtype != torch.float32 or W_A.dim() != 2:
+            raise TypeError("W_A must be a (d, D) float32 tensor")
+        self.d, self.D = int(W_A.shape[0]), int(W_A.shape[1])
+        handle = ctypes.c_void_p()
+        _check(lib.sa_prepare_adapter(_dev_ptr(W_A, "W_A"), self.d, self.D,
+                                      ctypes.c_void_p(_stream_handle(stream)), ctypes.byref(handle)),
+               "sa_prepare_adapter")
+        self._h, self._lib = handle, lib
+
+    def forward(self, X_tilde, out=None, device_flags=None, stream=None):
+        """X_tilde (..., d) fp32 -> (..., D) bf16."""
+        torch = _torch()
+        if X_tilde.dtype != torch.float32 or int(X_tilde.shape[-1]) != self.d:
+            raise TypeError("X_tilde must be float32 with last dimension d")
+        rows = int(X_tilde.numel()) // self.d
+        if out is None:
+            out = torch.empty(tuple(X_tilde.shape[:-1]) + (self.D,), dtype=torch.bfloat16,
+                              device=X_tilde.device)
+        fp = _dev_ptr(device_flags, "device_flags") if device_flags is not None else ctypes.c_void_p(0)
+        _check(self._lib.sa_adapter_forward(self._h, _dev_ptr(X_tilde, "X_tilde"), rows,
+                                             _dev_ptr(out, "out"), fp,
+                                             ctypes.c_void_p(_stream_handle(stream))),
+               "sa_adapter_forward")
+        return out
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self._lib.sa_adapter_free(self._h)
+            self._h = None
+
+    def __del__(self):  # pragma: no cover
+        try:
+            self.close()
+        except Exception:
+            pass

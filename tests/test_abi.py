@@ -101,8 +101,10 @@ def _kind(ctype_decl):
     """Coarse class of a C parameter or return type: pointer, 64-bit integer,
     32-bit integer/enum, float, size_t or void."""
     t = " ".join(ctype_decl.replace("*", " * ").split())
-    if "*" in t or t.startswith("sa_query") or t.startswith("sa_refine"):
+    if "*" in t or t.startswith(("sa_query", "sa_refine", "sa_cache", "sa_adapter")):
         return "ptr"
+    if t == "double":
+        return "f64"
     if "int64_t" in t:
         return "i64"
     if "size_t" in t:
@@ -125,6 +127,8 @@ def _ctypes_kind(ct):
         return "size"
     if ct is ctypes.c_float:
         return "f32"
+    if ct is ctypes.c_double:
+        return "f64"
     return "i32"
 
 
@@ -173,3 +177,28 @@ def test_backward_rejects_bad_arguments_on_the_host(lib):
                                   dummy, dummy, dummy, dummy, dummy, 1 << 20, None) == \
         binding.SA_ERR_INVALID_ARG
     assert lib.sa_workspace_bytes_backward(None, 1, 1) == 0
+
+
+def test_cache_and_adapter_reject_bad_arguments_on_the_host(lib):
+    out = ctypes.c_void_p(123)
+    for k, d, cap, ttl in [(0, 128, 4, 1.0), (16, 6, 4, 1.0), (16, 128, 0, 1.0), (16, 128, 4, 0.0),
+                           (16, 128, 4, float("nan"))]:
+        assert lib.sa_cache_create(k, d, cap, ttl, ctypes.byref(out)) == binding.SA_ERR_INVALID_ARG
+        assert out.value is None
+    lib.sa_cache_free(None)  # NULL-safe
+    dummy = ctypes.c_void_p(256)
+    assert lib.sa_cache_lookup(None, dummy, 1, 0.0, dummy, dummy, dummy, None) == \
+        binding.SA_ERR_INVALID_ARG
+    assert lib.sa_cache_insert(None, dummy, 1, 0.0, dummy, dummy, None) == \
+        binding.SA_ERR_INVALID_ARG
+    assert lib.sa_cache_stats(None, None, None, None, None) == binding.SA_ERR_INVALID_ARG
+    assert lib.sa_cache_forward(None, None, dummy, 0.0, dummy, dummy, 1, 1, dummy, dummy, dummy,
+                                dummy, 1 << 20, None) == binding.SA_ERR_INVALID_ARG
+    assert lib.sa_cache_forward_workspace_bytes(None, 1, 1) == 0
+    for d, D in [(96, 256), (128, 0), (128, 300), (256, 256)]:
+        assert lib.sa_prepare_adapter(dummy, d, D, None, ctypes.byref(out)) == \
+            binding.SA_ERR_INVALID_ARG
+    assert lib.sa_prepare_adapter(None, 128, 256, None, ctypes.byref(out)) == \
+        binding.SA_ERR_INVALID_ARG
+    lib.sa_adapter_free(None)  # NULL-safe
+    assert lib.sa_adapter_forward(None, dummy, 1, dummy, None, None) == binding.SA_ERR_INVALID_ARG
