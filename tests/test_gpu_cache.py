@@ -67,7 +67,9 @@ def test_cache_decisions_and_round_trip_match_the_model(capacity, ttl):
     assert (st["hits"], st["misses"], st["evictions"]) == (model.hits, model.misses,
                                                            model.evictions)
     assert st["entries"] == len(model.index)
-    assert model.evictions > 0 and model.hits > 0
+    assert model.hits > 0
+    if capacity < len(universe):
+        assert model.evictions > 0
     cache.close()
 
 
