@@ -28,3 +28,4 @@ from .sa_refine import (  # noqa: F401
     silu,
     swiglu_ffn,
 )
+from .sa_action import action_fuse, fusion_hidden, fusion_input  # noqa: F401
