@@ -65,6 +65,7 @@ typedef enum sa_dtype {
 #define SA_DEVFLAG_OFFSET_LAST 4u      /* offsets[batch] != total_rows */
 #define SA_DEVFLAG_TIMEOUT 8u          /* a kernel's bounded wait gave up */
 #define SA_DEVFLAG_SMEM_ALIGN 16u      /* a kernel found its shared memory misaligned (no work done) */
+#define SA_DEVFLAG_ACTION_TYPE 32u     /* an action type id >= the producer's n_types */
 
 /* Opaque handle: the precomputed query Q' for one weight set. */
 typedef struct sa_query_s* sa_query;
@@ -546,6 +547,75 @@ void sa_adapter_free(sa_adapter a);
  */
 sa_status sa_adapter_forward(sa_adapter a, const float* X_tilde, int64_t rows, void* out,
                              uint32_t* device_flags, void* stream);
+
+/*
+ * Action-side fusion (section 2.2 "Stacked Refinement 与动作侧融合" of the
+ * same notes): the producer of the history matrix X.  For behaviour i with
+ * item embedding e_i (d wide) and action type id t_i:
+ *
+ *     x_i = e_i + (SiLU(z_i W1) * (z_i W3)) W2,   z_i = [e_i ; table[t_i]],
+ *
+ * W1, W3 (d + d_a) x h with the e-rows first, W2 h x d, no biases, the
+ * action table n_types x d_a.  The page gives the abstract form (a SwiGLU
+ * network over the concatenation, residual on e_i) and no more; this is
+ * the reading built.  The library folds table W1[d:] and table W3[d:] into
+ * per-type rows at prepare time, so the producer's products have K = d.
+ */
+typedef struct sa_action_s* sa_action;
+
+/*
+ * sa_prepare_action -- the producer's parameters.
+ *
+ *   W1, W3        device, (d + d_a) x h fp32, row-major, 4-byte aligned
+ *   W2            device, h x d fp32
+ *   action_table  device, n_types x d_a fp32
+ *   d             64 or 128
+ *   d_a           1 <= d_a <= 4096
+ *   h             a multiple of 64, 64 <= h <= 4096
+ *   n_types       1 <= n_types <= 16
+ *   stream        the bf16 copies and the per-type rows are made by a kernel
+ *                 on it; the inputs may be freed once the stream has passed
+ *                 this call
+ *
+ * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED (not sm_100), SA_ERR_CUDA.
+ */
+sa_status sa_prepare_action(const float* W1, const float* W3, const float* W2,
+                            const float* action_table, int d, int d_a, int h, int n_types,
+                            void* stream, sa_action* out);
+
+/* Releases a producer (synchronises with the device).  NULL is a no-op. */
+void sa_action_free(sa_action act);
+
+/*
+ * sa_action_fuse -- X = the fused rows for `rows` behaviours (one tcgen05
+ * kernel; bf16 products with fp32 accumulation, the gate in fp32, X rounded
+ * to bf16).
+ *
+ *   E             device, rows x d bf16, 16-byte aligned: item embeddings
+ *   types         device, rows uint8: action type ids; an id >= n_types
+ *                 contributes no action term and raises SA_DEVFLAG_ACTION_TYPE
+ *   rows          0 <= rows < 2^31 - 256
+ *   X             device out, rows x d bf16, 16-byte aligned; must not
+ *                 overlap E
+ *   device_flags  device uint32 (or NULL): SA_DEVFLAG_* bits OR-ed in
+ */
+sa_status sa_action_fuse(sa_action act, const void* E, const uint8_t* types, int64_t rows, void* X,
+                         uint32_t* device_flags, void* stream);
+
+/*
+ * sa_action_sketch_forward -- the producer followed by one SA layer over its
+ * output: X is written to the workspace and compressed by sa_sketch_forward
+ * (q bf16, the same d as act).  offsets, batch, total_rows, X_tilde, mass
+ * as for sa_sketch_forward; workspace >=
+ * sa_workspace_bytes_action_sketch(q, batch, total_rows), 256-byte aligned.
+ * Device flags of both kernels are read with sa_read_device_status on the
+ * workspace.
+ */
+size_t sa_workspace_bytes_action_sketch(sa_query q, int64_t batch, int64_t total_rows);
+sa_status sa_action_sketch_forward(sa_action act, sa_query q, const void* E, const uint8_t* types,
+                                   const int64_t* offsets, int64_t batch, int64_t total_rows,
+                                   float* X_tilde, float* mass, void* workspace,
+                                   size_t workspace_bytes, void* stream);
 
 /* Static description of a status code. */
 const char* sa_status_string(sa_status s);

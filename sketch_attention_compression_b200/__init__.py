@@ -9,6 +9,7 @@ binding (binding.py).  Importing the package does not load the library;
 from .binding import (  # noqa: F401
     SA_BF16,
     SA_FP32,
+    ActionFusion,
     CacheKey,
     RefineParams,
     SAError,

@@ -20,7 +20,7 @@ SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA, \
     SA_ERR_DEVICE_FLAG = range(6)
 SA_BF16, SA_FP32 = 0, 1
 DEVFLAG_OFFSET0_NONZERO, DEVFLAG_OFFSETS_DECREASE, DEVFLAG_OFFSET_LAST, DEVFLAG_TIMEOUT, \
-    DEVFLAG_SMEM_ALIGN = 1, 2, 4, 8, 16
+    DEVFLAG_SMEM_ALIGN, DEVFLAG_ACTION_TYPE = 1, 2, 4, 8, 16, 32
 
 # name -> (restype, argtypes); mirrors include/sa.h
 _vp, _i32, _i64, _sz, _f32, _f64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, \
@@ -69,6 +69,13 @@ SIGNATURES = {
     "sa_prepare_adapter": (_i32, [_vp, _i32, _i32, _vp, ctypes.POINTER(_vp)]),
     "sa_adapter_free": (None, [_vp]),
     "sa_adapter_forward": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp]),
+    "sa_prepare_action": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp,
+                                 ctypes.POINTER(_vp)]),
+    "sa_action_free": (None, [_vp]),
+    "sa_action_fuse": (_i32, [_vp, _vp, _vp, _i64, _vp, _vp, _vp]),
+    "sa_workspace_bytes_action_sketch": (_sz, [_vp, _i64, _i64]),
+    "sa_action_sketch_forward": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _sz,
+                                        _vp]),
 }
 
 
@@ -619,6 +626,77 @@ class WidthAdapter:
     def close(self) -> None:
         if getattr(self, "_h", None):
             self._lib.sa_adapter_free(self._h)
+            self._h = None
+
+    def __del__(self):  # pragma: no cover
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class ActionFusion:
+    """The action-fusion producer (sa_prepare_action): X = E + SwiGLU-FFN of
+    [E ; table[types]].  W1, W3 (d + d_a, h), W2 (h, d) and table
+    (n_types, d_a) are fp32 CUDA tensors."""
+
+    def __init__(self, W1, W3, W2, table, stream=None):
+        torch = _torch()
+        lib = load_library()
+        for name, t in (("W1", W1), ("W3", W3), ("W2", W2), ("table", table)):
+            if t.dtype != torch.float32 or t.dim() != 2:
+                raise TypeError(f"{name} must be a 2-D float32 tensor")
+        self.h, self.d = int(W2.shape[0]), int(W2.shape[1])
+        self.n_types, self.d_a = int(table.shape[0]), int(table.shape[1])
+        if tuple(W1.shape) != (self.d + self.d_a, self.h) or tuple(W3.shape) != tuple(W1.shape):
+            raise ValueError("W1, W3 must be (d + d_a, h)")
+        handle = ctypes.c_void_p()
+        _check(lib.sa_prepare_action(_dev_ptr(W1, "W1"), _dev_ptr(W3, "W3"), _dev_ptr(W2, "W2"),
+                                     _dev_ptr(table, "table"), self.d, self.d_a, self.h,
+                                     self.n_types, ctypes.c_void_p(_stream_handle(stream)),
+                                     ctypes.byref(handle)), "sa_prepare_action")
+        self._h, self._lib = handle, lib
+
+    def fuse(self, E, types, out=None, device_flags=None, stream=None):
+        """E (rows, d) bf16 and types (rows,) uint8 CUDA tensors -> X (rows, d) bf16."""
+        torch = _torch()
+        if E.dtype != torch.bfloat16 or types.dtype != torch.uint8:
+            raise TypeError("E must be bfloat16 and types uint8")
+        rows = int(E.shape[0])
+        if out is None:
+            out = torch.empty_like(E)
+        fp = _dev_ptr(device_flags, "device_flags") if device_flags is not None else ctypes.c_void_p(0)
+        if rows > 0:
+            _check(self._lib.sa_action_fuse(self._h, _dev_ptr(E, "E"), _dev_ptr(types, "types"), rows,
+                                            _dev_ptr(out, "out"), fp,
+                                            ctypes.c_void_p(_stream_handle(stream))),
+                   "sa_action_fuse")
+        return out
+
+    def sketch_forward(self, query: "SketchQuery", E, types, offsets, X_tilde=None, mass=None,
+                       workspace=None, stream=None):
+        """The producer followed by one SA layer (sa_action_sketch_forward).
+        Returns (X_tilde, mass, workspace)."""
+        torch = _torch()
+        B, N = int(offsets.shape[0]) - 1, int(E.shape[0])
+        if X_tilde is None:
+            X_tilde = torch.empty((B, query.k, query.d), dtype=torch.float32, device=E.device)
+        if mass is None:
+            mass = torch.empty((B, query.k), dtype=torch.float32, device=E.device)
+        if workspace is None:
+            workspace = torch.empty(int(self._lib.sa_workspace_bytes_action_sketch(query._h, B, N)),
+                                    dtype=torch.uint8, device=E.device)
+        _check(self._lib.sa_action_sketch_forward(
+            self._h, query._h, ctypes.c_void_p(E.data_ptr() if N > 0 else 0),
+            ctypes.c_void_p(types.data_ptr() if N > 0 else 0), _dev_ptr(offsets, "offsets"), B, N,
+            _dev_ptr(X_tilde, "X_tilde"), _dev_ptr(mass, "mass"), _dev_ptr(workspace, "workspace"),
+            int(workspace.numel() * workspace.element_size()),
+            ctypes.c_void_p(_stream_handle(stream))), "sa_action_sketch_forward")
+        return X_tilde, mass, workspace
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self._lib.sa_action_free(self._h)
             self._h = None
 
     def __del__(self):  # pragma: no cover

@@ -27,7 +27,7 @@ INJECT_LIB = os.path.join(PKG, "_lib", "libsa_inject.so")
 INJECT_DEFINES = ["-DSA_FAULT_INJECT", "-DSA_WAIT_TIMEOUT_CYCLES=200000000ll"]
 SOURCES = ["sa_api.cu", "sa_prepare.cu", "sa_fused.cu", "sa_simt.cu", "sa_finalize.cu",
            "sa_noalloc.cu", "sa_fused_pair.cu", "sa_normalise.cu", "sa_refine.cu",
-           "sa_backward.cu", "sa_cache.cu"]
+           "sa_backward.cu", "sa_cache.cu", "sa_action.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
           "-I", os.path.join(ROOT, "include"), "-I", CSRC]

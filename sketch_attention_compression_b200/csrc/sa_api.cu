@@ -46,18 +46,31 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                    uint32_t box_rows) {
+bool make_tmap_bf16_box(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                        uint32_t box_cols, uint32_t box_rows, int swizzle_bytes) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
+  CUtensorMapSwizzle sw;
+  if (swizzle_bytes == 128 && box_cols == 64) {
+    sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  } else if (swizzle_bytes == 32 && box_cols == 16) {
+    sw = CU_TENSOR_MAP_SWIZZLE_32B;
+  } else {
+    return false;
+  }
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+  return make_tmap_bf16_box(m, base, rows, cols, 64, box_rows, 128);
 }
 
 }  // namespace sa
@@ -477,6 +490,45 @@ sa_status sa_refine_layer_forward(sa_query q, sa_refine r, const float* prev, co
                                   size_t workspace_bytes, void* stream) {
   return refine_layer(q, r, prev, P_f32, X, offsets, batch, total_rows, out, workspace,
                       workspace_bytes, stream, false);
+}
+
+size_t sa_workspace_bytes_action_sketch(sa_query q, int64_t batch, int64_t total_rows) {
+  if (q == nullptr || batch < 0 || total_rows < 0) return 0;
+  return round_up(ws_layout(q, total_rows).total, 256) +
+         round_up(static_cast<size_t>(total_rows) * q->d * 2, 256);
+}
+
+sa_status sa_action_sketch_forward(sa_action act, sa_query q, const void* E, const uint8_t* types,
+                                   const int64_t* offsets, int64_t batch, int64_t total_rows,
+                                   float* X_tilde, float* mass, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  if (act == nullptr || q == nullptr) return SA_ERR_INVALID_ARG;
+  if (q->dtype != SA_BF16) return SA_ERR_UNSUPPORTED;
+  int ad = 0, adev = -1;
+  sa::action_info(act, &ad, &adev);
+  if (ad != q->d || adev != q->device || !same_device(q)) return SA_ERR_INVALID_ARG;
+  if (batch < 0 || total_rows < 0 || total_rows >= kMaxRows) return SA_ERR_INVALID_ARG;
+  if (batch == 0) return total_rows == 0 ? SA_OK : SA_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned(workspace, 256)) return SA_ERR_INVALID_ARG;
+  if (total_rows > 0 && (E == nullptr || types == nullptr || !aligned(E, 16)))
+    return SA_ERR_INVALID_ARG;
+  if (workspace_bytes < sa_workspace_bytes_action_sketch(q, batch, total_rows))
+    return SA_ERR_WORKSPACE;
+  // X goes after the SA pass's workspace.  The flag words are cleared here
+  // and kept by the SA pass, so that the producer's bits survive it.
+  const size_t sa_bytes = round_up(ws_layout(q, total_rows).total, 256);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* X = ws + sa_bytes;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  sa::WsHeader* hdr = reinterpret_cast<sa::WsHeader*>(ws);
+  if (cudaMemsetAsync(hdr, 0, 2 * sizeof(uint32_t), st) != cudaSuccess) return SA_ERR_CUDA;
+  if (total_rows > 0) {
+    const sa_status s =
+        sa::action_fuse_enqueue(act, E, types, total_rows, X, &hdr->timeout_flags, st);
+    if (s != SA_OK) return s;
+  }
+  return run(q, nullptr, X, offsets, batch, total_rows, X_tilde, mass, workspace, sa_bytes, stream,
+             Phase::kBoth, true);
 }
 
 size_t sa_workspace_bytes_refine_stack(sa_query q, int64_t batch, int64_t total_rows) {

@@ -28,7 +28,11 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "sa.h"
+
 #define SA_HD __host__ __device__ __forceinline__
+
+struct sa_action_s;
 
 namespace sa {
 
@@ -197,6 +201,17 @@ struct PassArgs {
 // the driver's encoder is unavailable or rejects the shape.
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows);
+// The same with the box width and swizzle chosen: 64 columns with the
+// 128-byte swizzle, or 16 columns (32 bytes) with the 32-byte swizzle.
+bool make_tmap_bf16_box(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                        uint32_t box_cols, uint32_t box_rows, int swizzle_bytes);
+
+// Action-side fusion (sa_action.cu): the width d and the device of a
+// prepared producer, and the producer kernel X = E + SwiGLU-FFN([E; a]) for
+// `rows` rows enqueued on `st` (flag bits OR-ed into *flags when not null).
+void action_info(const sa_action_s* act, int* d, int* device);
+sa_status action_fuse_enqueue(const sa_action_s* act, const void* E, const uint8_t* types,
+                              int64_t rows, void* X, uint32_t* flags, cudaStream_t st);
 
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error.

@@ -18,6 +18,7 @@ enum : uint32_t {
   DEVFLAG_OFFSET_LAST = 4u,        // offsets[batch] != total_rows
   DEVFLAG_TIMEOUT = 8u,            // a bounded wait inside a kernel gave up
   DEVFLAG_SMEM_ALIGN = 16u,        // dynamic shared memory not 1024-byte aligned
+  DEVFLAG_ACTION_TYPE = 32u,       // an action type id outside the action table
 };
 
 // A wait that has not completed after this many SM clock cycles (about 2 s

@@ -24,6 +24,8 @@ Conventions (the notation of section 2.1 of that page):
 from .workloads import (  # noqa: F401
     WORKLOADS,
     Workload,
+    action_params,
+    action_types,
     bf16_bits,
     bf16_from_bits,
     generate,

@@ -234,3 +234,28 @@ def refine_params(d: int, h: int, seed: int, dtype: str = "bf16") -> dict:
     out["W3"] = (rng.standard_normal((d, h)) / math.sqrt(d)).astype(np.float32)
     out["W2"] = (rng.standard_normal((h, d)) / math.sqrt(h)).astype(np.float32)
     return out
+
+
+def action_params(d: int, d_a: int, h: int, n_types: int, seed: int) -> dict:
+    """Seeded parameters of the action-fusion producer (x = e + SwiGLU-FFN of
+    [e ; a]): the action table (n_types, d_a) ~ N(0, 1), W1, W3 (d + d_a, h)
+    ~ N(0, 1/(d + d_a)), W2 (h, d) ~ N(0, 1/h), all float32 with
+    bf16-representable values (the producer holds its weights in bf16)."""
+    rng = np.random.default_rng(seed)
+    k_in = d + d_a
+    return dict(
+        table=round_to_bf16(rng.standard_normal((n_types, d_a), dtype=np.float32)),
+        W1=round_to_bf16((rng.standard_normal((k_in, h)) / math.sqrt(k_in)).astype(np.float32)),
+        W3=round_to_bf16((rng.standard_normal((k_in, h)) / math.sqrt(k_in)).astype(np.float32)),
+        W2=round_to_bf16((rng.standard_normal((h, d)) / math.sqrt(h)).astype(np.float32)),
+        d=d, d_a=d_a, h=h, n_types=n_types)
+
+
+def action_types(rows: int, n_types: int, seed: int) -> np.ndarray:
+    """Seeded action type ids (rows,) uint8 with P(t) proportional to 2^-t:
+    a few common feedback types (a swipe, a finish) and rarer strong ones (a
+    like, a follow).  The frequencies are invented; the page names the types
+    and gives no mix."""
+    rng = np.random.default_rng(seed)
+    p = 0.5 ** np.arange(n_types)
+    return rng.choice(n_types, size=rows, p=p / p.sum()).astype(np.uint8)

@@ -101,7 +101,7 @@ def _kind(ctype_decl):
     """Coarse class of a C parameter or return type: pointer, 64-bit integer,
     32-bit integer/enum, float, size_t or void."""
     t = " ".join(ctype_decl.replace("*", " * ").split())
-    if "*" in t or t.startswith(("sa_query", "sa_refine", "sa_cache", "sa_adapter")):
+    if "*" in t or t.startswith(("sa_query", "sa_refine", "sa_cache", "sa_adapter", "sa_action")):
         return "ptr"
     if t == "double":
         return "f64"
@@ -202,3 +202,21 @@ def test_cache_and_adapter_reject_bad_arguments_on_the_host(lib):
         binding.SA_ERR_INVALID_ARG
     lib.sa_adapter_free(None)  # NULL-safe
     assert lib.sa_adapter_forward(None, dummy, 1, dummy, None, None) == binding.SA_ERR_INVALID_ARG
+
+
+def test_action_entry_points_reject_bad_arguments_on_the_host(lib):
+    out = ctypes.c_void_p(123)
+    dummy = ctypes.c_void_p(256)
+    for d, da, h, nt in [(96, 8, 128, 4), (128, 0, 128, 4), (128, 8, 100, 4), (128, 8, 0, 4),
+                         (128, 8, 128, 0), (128, 8, 128, 17), (128, 8, 8192, 4)]:
+        assert lib.sa_prepare_action(dummy, dummy, dummy, dummy, d, da, h, nt, None,
+                                     ctypes.byref(out)) == binding.SA_ERR_INVALID_ARG
+        assert out.value is None
+    assert lib.sa_prepare_action(None, dummy, dummy, dummy, 128, 8, 128, 4, None,
+                                 ctypes.byref(out)) == binding.SA_ERR_INVALID_ARG
+    lib.sa_action_free(None)  # NULL-safe
+    assert lib.sa_action_fuse(None, dummy, dummy, 1, dummy, None, None) == \
+        binding.SA_ERR_INVALID_ARG
+    assert lib.sa_action_sketch_forward(None, None, dummy, dummy, dummy, 1, 1, dummy, dummy, dummy,
+                                        1 << 20, None) == binding.SA_ERR_INVALID_ARG
+    assert lib.sa_workspace_bytes_action_sketch(None, 1, 1) == 0
