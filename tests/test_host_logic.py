@@ -18,6 +18,7 @@ def test_row_range_schedule(tmp_path):
     cuda_inc = "/usr/local/cuda/include"
     subprocess.run(["g++", "-O1", "-std=c++17",
                     "-I", os.path.join(ROOT, "sketch_attention_compression_b200", "csrc"),
+                    "-I", os.path.join(ROOT, "include"),
                     "-I", cuda_inc, os.path.join(ROOT, "tests", "host", "schedule_check.cpp"),
                     "-o", str(exe)], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
@@ -33,6 +34,7 @@ def test_shared_memory_plan(tmp_path):
     exe = tmp_path / "plan_check"
     subprocess.run(["g++", "-O1", "-std=c++17",
                     "-I", os.path.join(ROOT, "sketch_attention_compression_b200", "csrc"),
+                    "-I", os.path.join(ROOT, "include"),
                     "-I", "/usr/local/cuda/include", os.path.join(ROOT, "tests", "host", "plan_check.cpp"),
                     "-o", str(exe)], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
