@@ -779,6 +779,101 @@ def run_refine(args, rank, world, local_rank, ranks):
     print(json.dumps(line), flush=True)
 
 
+def run_action(args, rank, world, local_rank, ranks):
+    """One step = sa_action_sketch_forward over the batch: the action-fusion
+    producer X = E + SwiGLU-FFN([E; a]) (section 2.2, hidden width
+    --action-hidden, four action types) followed by the SA layer on X."""
+    import torch
+
+    from sketch_attention_compression_b200 import (ActionFusion, SketchQuery, load_library,
+                                                   read_device_status)
+    from synthetic import action_params, action_types
+    load_library()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOADS[args.workload]
+    h, n_types = args.action_hidden, 4
+    seed = rank_seed(args.workload, rank)
+    inp = workload_inputs(args, seed=seed)
+    B, N = len(inp["offsets"]) - 1, int(inp["offsets"][-1])
+    E = torch.from_numpy(inp["X"]).to(dev).to(torch.bfloat16)
+    types_np = action_types(N, n_types, seed=seed + 400)
+    types = torch.from_numpy(types_np).to(dev)
+    offsets = torch.from_numpy(inp["offsets"]).to(dev)
+    p = action_params(w.d, w.d, h, n_types, seed=seed + 401)
+    stream = torch.cuda.current_stream(dev)
+    t = {key: torch.from_numpy(p[key]).to(dev) for key in ("W1", "W3", "W2", "table")}
+    act = ActionFusion(t["W1"], t["W3"], t["W2"], t["table"], stream=stream)
+    q = SketchQuery(*(torch.from_numpy(inp[k]).to(dev).to(torch.bfloat16) for k in ("P", "W_Q", "W_K")),
+                    inp["scale"], stream=stream)
+    Xt, m, ws = act.sketch_forward(q, E, types, offsets, stream=stream)
+    Xbuf = torch.empty_like(E)
+
+    def step():
+        act.sketch_forward(q, E, types, offsets, X_tilde=Xt, mass=m, workspace=ws, stream=stream)
+
+    def producer():
+        act.fuse(E, types, out=Xbuf, stream=stream)
+    for _ in range(args.warmup):
+        step()
+        producer()
+    if read_device_status(ws, stream) != 0:
+        raise RuntimeError("device flags raised during warm-up")
+    sampler = None
+    if rank == 0:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        sampler.start()
+        time.sleep(0.05)
+    mark = sampler.mark() if sampler else 0
+    ms = _timed(step, args.steps, dev, stream, ranks)
+    ms_prod = _timed(producer, args.steps, dev, stream, ranks)
+    clocks = sampler.summary(mark) if sampler else None
+    if sampler:
+        sampler.stop()
+    if read_device_status(ws, stream) != 0:
+        raise RuntimeError("device flags raised during the timed region")
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    rows_total = ranks.sum(N)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        from oracle import action_fuse, sa_user
+        t0 = time.perf_counter()
+        rows, done = 0, 0
+        offs = inp["offsets"]
+        for b in range(B):
+            lo, hi = int(offs[b]), int(offs[b + 1])
+            Xo = action_fuse(inp["X"][lo:hi], types_np[lo:hi], p["table"], p["W1"], p["W3"], p["W2"])
+            sa_user(Xo, inp["P"], inp["W_Q"], inp["W_K"], inp["scale"])
+            rows += hi - lo
+            done = b
+            if time.perf_counter() - t0 >= args.cpu_budget:
+                break
+        dt = time.perf_counter() - t0
+        cpu = {"value": rows / dt, "unit": "rows/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"users 0..{done} ({rows} rows, {dt:.1f} s, numpy fp64 action_fuse + sa_user)"}
+    line = {
+        "metric": "action fusion + SA history rows/sec on 1 B200",
+        "value": rows_total / (ms * 1e-3), "unit": "rows/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "mode": "action_fusion + sa", "users_per_gpu": B,
+                   "rows_per_gpu": N, "d": w.d, "k": w.k, "ffn_hidden": h, "action_types": n_types,
+                   "action_width": w.d, "producer_ms": ms_prod},
+        "roofline": _roofline((4.0 * w.d + 1.0) * N, 6.0 * w.d * h * N, ms_prod, peaks, peak_kind,
+                              "action_fuse_kernel (the producer alone)",
+                              f"{6 * w.d * h} flop (E W1, E W3, G W2; the action term is a "
+                              f"per-type row) and {4 * w.d + 1} B (E read, X written, type) "
+                              f"per row x {N} rows"),
+        "clocks": clocks, "cpu_baseline": cpu,
+        "gpu_launches": 3 * args.steps + args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -798,6 +893,10 @@ def main():
                     help="time the SA backward pass (sa_sketch_backward) instead")
     ap.add_argument("--refine-layers", type=int, default=0,
                     help="time a stack of this many refinement layers instead")
+    ap.add_argument("--action-fusion", action="store_true",
+                    help="time the action-fusion producer followed by the SA layer instead")
+    ap.add_argument("--action-hidden", type=int, default=512,
+                    help="hidden width of the action-fusion FFN")
     ap.add_argument("--users", type=int, default=0,
                     help="use only the first U users of the workload (smaller case)")
     args = ap.parse_args()
@@ -824,6 +923,8 @@ def main():
             run_backward(args, rank, world, local_rank, ranks)
         elif args.refine_layers > 0:
             run_refine(args, rank, world, local_rank, ranks)
+        elif args.action_fusion:
+            run_action(args, rank, world, local_rank, ranks)
         else:
             run_ours(args, rank, world, local_rank, ranks)
     finally:

@@ -15,15 +15,22 @@
 // Kernel: persistent, one CTA per SM, pairs of 128-row tiles (slots A and
 // B), the hidden width in chunks of 64.  Warp 0 issues TMA loads (E tiles;
 // per chunk W1_e^T, W3_e^T, W2^T and the T1, T3 columns, into a two-stage
-// ring); warp 1 issues the MMAs; warps 2-9 are the epilogue.  Per slot and
-// chunk c:
-//   U = E W1_c + onehot T1_c, V = E W3_c + onehot T3_c   M 128, N 64  (TMEM)
+// ring whose W1/W3 and W2 parts have their own barriers, so each is
+// refilled as soon as both slots have read it); warp 1 issues the MMAs;
+// warps 2-9 gate slot A and warps 10-17 slot B, so that the two slots'
+// epilogues overlap.  Per slot and chunk c:
+//   [U | V] = E [W1_c | W3_c] + onehot [T1_c | T3_c]   M 128, N 128 (TMEM)
 //   G = SiLU(U) * V                   epilogue: bf16 into shared memory
 //   Y += G W2_c                       M 128, N d, K 64              (TMEM)
-// and at the end x = Y + e (e re-read from global memory, where the tile
-// just passed through L2), rounded to bf16.  The two slots alternate, so
-// the tensor cores run one slot's products while the epilogue gates the
-// other's.  TMEM: slot r holds U at 256 r, V at 256 r + 64, Y at 256 r + 128.
+// U and V are one product (N = 128) so that each K-step reads the E slice
+// from shared memory once: with N = 64 products the operand reads, not the
+// tensor cores, set the pace.
+// The residual is a product too: after the first chunk, Y += E I_16 slice
+// by slice (M 128, N 16, K 16 per 16 columns of E), from the E tile already
+// in shared memory, so that the epilogue only rounds Y to bf16 and stores
+// it.  The two slots alternate on the tensor cores, which run one slot's
+// products while the other slot's epilogue gates.  TMEM: slot r holds U at
+// 256 r, V at 256 r + 64, Y at 256 r + 128.
 // SiLU(u) = u sigma(u) with sigma(u) = (1 + tanh(u / 2)) / 2, one MUFU
 // operation per element.
 #include <cuda_bf16.h>
@@ -49,7 +56,7 @@ struct sa_action_s {
 namespace sa {
 namespace {
 
-constexpr int kActThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int kActThreads = 576;  // warp 0 TMA, warp 1 MMA, warps 2-9 and 10-17 epilogue
 constexpr int kHc = 64;           // hidden columns per chunk
 constexpr int kMaxTypes = 16;
 
@@ -61,16 +68,20 @@ struct ActPlan {
   static constexpr int kG = kE + 2 * kESlot;   // 2 slots x one 128 x 64 box
   static constexpr int kW = kG + 2 * kEBox;    // 2 weight stages
   static constexpr int kWBox = kHc * 128;      // 64 rows x 64 bf16
-  static constexpr int kW1 = 0;                // offsets inside a stage
-  static constexpr int kW3 = kW1 + (D / 64) * kWBox;
-  static constexpr int kW2 = kW3 + (D / 64) * kWBox;  // D rows x 64 bf16
+  // Inside a stage: per 64 columns of K, the W1 box then the W3 box, so that
+  // [W1_c ; W3_c] is one 128-row B operand and U, V one N = 128 product.
+  static constexpr int kW13 = 0;
+  static constexpr int kW13Box = 2 * kWBox;
+  static constexpr int kW2 = kW13 + (D / 64) * kW13Box;  // D rows x 64 bf16
   static constexpr int kT1 = kW2 + D * 128;           // 64 rows x 16 bf16, 32-byte swizzle
   static constexpr int kT3 = kT1 + kHc * 32;
   static constexpr int kStage = kT3 + kHc * 32;
-  static constexpr uint32_t kStageBytes = kStage;
+  static constexpr uint32_t kW13Bytes = 2 * (D / 64) * kWBox + 2 * kHc * 32;
+  static constexpr uint32_t kW2Bytes = D * 128;
   static constexpr uint32_t kEBytes = kESlot;
   static constexpr int kOH = kW + 2 * kStage;  // 2 slots x 128 rows x 32 B
-  static constexpr int kBars = kOH + 2 * 128 * 32;
+  static constexpr int kI = kOH + 2 * 128 * 32;  // I_16 (16 x 16 bf16, 32-byte swizzle)
+  static constexpr int kBars = kI + 1024;
   // At least 116 KB, so that one CTA holds an SM (it allocates all of TMEM).
   static constexpr int kSmem = kBars + 256 > 118784 ? kBars + 256 : 118784;
   static_assert(kStage % 1024 == 0, "stage alignment");
@@ -78,7 +89,6 @@ struct ActPlan {
 };
 
 struct ActArgs {
-  const uint16_t* E;       // [rows][d] bf16 (residual re-read)
   const uint8_t* types;    // [rows]
   uint16_t* X;             // [rows][d] bf16 out
   int64_t rows;
@@ -137,10 +147,12 @@ __global__ void __launch_bounds__(kActThreads, 1)
   uint64_t* epi_done = bars + 8;   // [2]
   uint64_t* y_full = bars + 10;    // [2]
   uint64_t* y_empty = bars + 12;   // [2]
-  uint64_t* w_full = bars + 14;    // [2]
-  uint64_t* w_empty = bars + 16;   // [2]
-  uint64_t* drain = bars + 18;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  uint64_t* w13_full = bars + 14;  // [2] W1, W3, T1, T3 of a chunk have landed
+  uint64_t* w13_empty = bars + 16; // [2] ... and both slots' U, V products have read them
+  uint64_t* w2_full = bars + 18;   // [2] W2 of a chunk has landed
+  uint64_t* w2_empty = bars + 20;  // [2] ... and both slots' Y products have read it
+  uint64_t* drain = bars + 22;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   uint32_t* local_flags = tmem_slot + 2;
   if (tid == 0) {
@@ -152,13 +164,28 @@ __global__ void __launch_bounds__(kActThreads, 1)
       mbar_init(epi_done + r, 8);
       mbar_init(y_full + r, 1);
       mbar_init(y_empty + r, 8);
-      mbar_init(w_full + r, 1);
-      mbar_init(w_empty + r, 1);
+      mbar_init(w13_full + r, 1);
+      mbar_init(w13_empty + r, 1);
+      mbar_init(w2_full + r, 1);
+      mbar_init(w2_empty + r, 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0u;
     *local_flags = 0u;
     fence_mbar_init();
+  }
+  if (warp == 2 && lane < 16) {
+    // I_16, the B operand that adds the residual e to Y (one 16-column slice
+    // per K-step of E).
+    uint32_t w[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      w[k] = ((lane & 7) >> 1) == (k & 3) && (lane >> 3) == (k >> 2)
+                 ? ((lane & 1) ? 0x3F800000u : 0x00003F80u)
+                 : 0u;
+    st_shared_v4(sbase + Pl::kI + swz32(lane, 0), w[0], w[1], w[2], w[3]);
+    st_shared_v4(sbase + Pl::kI + swz32(lane, 1), w[4], w[5], w[6], w[7]);
+    fence_proxy_async_smem();
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -175,7 +202,8 @@ __global__ void __launch_bounds__(kActThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t g = 0;          // chunks issued so far
+      uint32_t g = 0;          // chunks whose W2 part is issued
+      uint32_t g13 = 0;        // chunks whose W1/W3 part is issued
       uint32_t ep[2] = {0, 0};  // phases of e_full started per slot
       bool e_load[2] = {false, false};  // the latest of them is a TMA load
       bool ok = true;
@@ -199,28 +227,41 @@ __global__ void __launch_bounds__(kActThreads, 1)
                         static_cast<int32_t>(y));
         }
         for (int c = 0; c < C && ok; ++c, ++g) {
+          // Stage g & 1 is reused by chunk g: its W1/W3 part once both U, V
+          // products of chunk g - 2 are done, its W2 part once both Y
+          // products of chunk g - 2 are done (half a chunk later), so each
+          // part loads as early as it can.
           const int s = g & 1;
-          if (g >= 2 && !mbar_wait(w_empty + s, ((g >> 1) + 1) & 1, abort_flag, sticky)) {
+          uint8_t* st = smem + Pl::kW + s * Pl::kStage;
+          if (g >= 2 && !mbar_wait(w13_empty + s, ((g >> 1) + 1) & 1, abort_flag, sticky)) {
             ok = false;
             break;
           }
-          uint8_t* st = smem + Pl::kW + s * Pl::kStage;
-          mbar_arrive_expect_tx(w_full + s, Pl::kStageBytes);
+          mbar_arrive_expect_tx(w13_full + s, Pl::kW13Bytes);
 #pragma unroll
           for (int b = 0; b < D / 64; ++b) {
-            tma_load_2d(st + Pl::kW1 + b * Pl::kWBox, &tm_w1, w_full + s, b * 64, c * kHc);
-            tma_load_2d(st + Pl::kW3 + b * Pl::kWBox, &tm_w3, w_full + s, b * 64, c * kHc);
+            tma_load_2d(st + Pl::kW13 + b * Pl::kW13Box, &tm_w1, w13_full + s, b * 64, c * kHc);
+            tma_load_2d(st + Pl::kW13 + b * Pl::kW13Box + Pl::kWBox, &tm_w3, w13_full + s, b * 64,
+                        c * kHc);
           }
-          tma_load_2d(st + Pl::kW2, &tm_w2, w_full + s, c * kHc, 0);
-          tma_load_2d(st + Pl::kT1, &tm_t1, w_full + s, 0, c * kHc);
-          tma_load_2d(st + Pl::kT3, &tm_t3, w_full + s, 0, c * kHc);
+          tma_load_2d(st + Pl::kT1, &tm_t1, w13_full + s, 0, c * kHc);
+          tma_load_2d(st + Pl::kT3, &tm_t3, w13_full + s, 0, c * kHc);
+          ++g13;
+          if (g >= 2 && !mbar_wait(w2_empty + s, ((g >> 1) + 1) & 1, abort_flag, sticky)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(w2_full + s, Pl::kW2Bytes);
+          tma_load_2d(st + Pl::kW2, &tm_w2, w2_full + s, c * kHc, 0);
         }
       }
       if (!ok) {
         // Let the copies in flight land before the CTA releases its memory:
-        // the last phase armed on each full barrier.
+        // the last phases armed on each full barrier.
+        for (uint32_t k = (g13 >= 2 ? g13 - 2 : 0); k < g13; ++k)
+          mbar_wait_bounded(w13_full + (k & 1), (k >> 1) & 1);
         for (uint32_t k = (g >= 2 ? g - 2 : 0); k < g; ++k)
-          mbar_wait_bounded(w_full + (k & 1), (k >> 1) & 1);
+          mbar_wait_bounded(w2_full + (k & 1), (k >> 1) & 1);
         for (int r = 0; r < 2; ++r)
           if (e_load[r]) mbar_wait_bounded(e_full + r, (ep[r] - 1) & 1);
       }
@@ -228,27 +269,31 @@ __global__ void __launch_bounds__(kActThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_uv = idesc_bf16_f32(128, kHc, 0, 0);
+      constexpr uint32_t idesc_uv = idesc_bf16_f32(128, 2 * kHc, 0, 0);
       constexpr uint32_t idesc_y = idesc_bf16_f32(128, D, 0, 0);
+      constexpr uint32_t idesc_i = idesc_bf16_f32(128, 16, 0, 0);
       uint32_t g = 0;
       bool ok = true;
       auto mma1 = [&](int r, uint32_t gc) {
         const uint32_t st = sbase + Pl::kW + (gc & 1) * Pl::kStage;
         const uint64_t de = smem_desc(sbase + Pl::kE + r * Pl::kESlot, 16, 1024, 2);
-        const uint64_t d1 = smem_desc(st + Pl::kW1, 16, 1024, 2);
-        const uint64_t d3 = smem_desc(st + Pl::kW3, 16, 1024, 2);
-        const uint32_t tu = tmem + r * 256, tv = tu + 64;
+        const uint64_t d13 = smem_desc(st + Pl::kW13, 16, 1024, 2);
+        const uint32_t tu = tmem + r * 256;  // U in columns 0-63, V in 64-127
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          mma_bf16_ss(tu, de + kstep(ks, Pl::kEBox), d1 + kstep(ks, Pl::kWBox), idesc_uv,
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_bf16_ss(tu, de + kstep(ks, Pl::kEBox), d13 + kstep(ks, Pl::kW13Box), idesc_uv,
                       ks > 0 ? 1u : 0u);
-          mma_bf16_ss(tv, de + kstep(ks, Pl::kEBox), d3 + kstep(ks, Pl::kWBox), idesc_uv,
-                      ks > 0 ? 1u : 0u);
-        }
-        // The action term: onehot(type) (K = 16) times the T1, T3 columns.
+        // The action term: onehot(type) (K = 16) times [T1_c ; T3_c].
         const uint64_t doh = smem_desc(sbase + Pl::kOH + r * 4096, 16, 256, 6);
         mma_bf16_ss(tu, doh, smem_desc(st + Pl::kT1, 16, 256, 6), idesc_uv, 1u);
-        mma_bf16_ss(tv, doh, smem_desc(st + Pl::kT3, 16, 256, 6), idesc_uv, 1u);
+      };
+      // Y[:, 16 ks .. 16 ks + 16) += E[:, 16 ks .. 16 ks + 16) I_16: the residual.
+      auto residual = [&](int r) {
+        const uint64_t de = smem_desc(sbase + Pl::kE + r * Pl::kESlot, 16, 1024, 2);
+        const uint64_t di = smem_desc(sbase + Pl::kI, 16, 256, 6);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_bf16_ss(tmem + r * 256 + 128 + ks * 16, de + kstep(ks, Pl::kEBox), di, idesc_i, 1u);
       };
       auto mma2 = [&](int r, uint32_t gc, bool acc) {
         const uint32_t st = sbase + Pl::kW + (gc & 1) * Pl::kStage;
@@ -264,7 +309,7 @@ __global__ void __launch_bounds__(kActThreads, 1)
         for (int r = 0; r < 2 && ok; ++r)
           ok = mbar_wait(e_full + r, i & 1, abort_flag, sticky) &&
                mbar_wait(oh_full + r, i & 1, abort_flag, sticky);
-        if (!ok || !mbar_wait(w_full + (g0 & 1), (g0 >> 1) & 1, abort_flag, sticky)) {
+        if (!ok || !mbar_wait(w13_full + (g0 & 1), (g0 >> 1) & 1, abort_flag, sticky)) {
           ok = false;
           break;
         }
@@ -272,21 +317,27 @@ __global__ void __launch_bounds__(kActThreads, 1)
         for (int r = 0; r < 2; ++r) {
           mma1(r, g0);
           mma_commit(uv_full + r);
-          if (C == 1) mma_commit(e_empty + r);
         }
+        mma_commit(w13_empty + (g0 & 1));
         for (int c = 0; c < C && ok; ++c) {
           const uint32_t gc = g0 + c;
           for (int r = 0; r < 2 && ok; ++r) {
             if (!mbar_wait(epi_done + r, gc & 1, abort_flag, sticky) ||
-                (c == 0 && i > 0 && !mbar_wait(y_empty + r, (i - 1) & 1, abort_flag, sticky))) {
+                (c == 0 && i > 0 && !mbar_wait(y_empty + r, (i - 1) & 1, abort_flag, sticky)) ||
+                (r == 0 && !mbar_wait(w2_full + (gc & 1), (gc >> 1) & 1, abort_flag, sticky))) {
               ok = false;
               break;
             }
             tc_fence_after();
             mma2(r, gc, c > 0);
+            if (r == 1) mma_commit(w2_empty + (gc & 1));
+            if (c == 0) {
+              residual(r);
+              if (C == 1) mma_commit(e_empty + r);
+            }
             if (c == C - 1) mma_commit(y_full + r);
             if (c + 1 < C) {
-              if (r == 0 && !mbar_wait(w_full + ((gc + 1) & 1), ((gc + 1) >> 1) & 1, abort_flag,
+              if (r == 0 && !mbar_wait(w13_full + ((gc + 1) & 1), ((gc + 1) >> 1) & 1, abort_flag,
                                        sticky)) {
                 ok = false;
                 break;
@@ -294,10 +345,10 @@ __global__ void __launch_bounds__(kActThreads, 1)
               tc_fence_after();
               mma1(r, gc + 1);
               mma_commit(uv_full + r);
+              if (r == 1) mma_commit(w13_empty + ((gc + 1) & 1));
               if (c + 1 == C - 1) mma_commit(e_empty + r);
             }
           }
-          if (ok) mma_commit(w_empty + (gc & 1));
         }
         g = g0 + C;
       }
@@ -308,21 +359,23 @@ __global__ void __launch_bounds__(kActThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;              // TMEM lane quadrant
-    const int half = (warp - 2) >> 2;    // which 32 of the chunk's 64 columns
+    const int slot = (warp - 2) >> 3;        // warps 2-9 gate slot A, warps 10-17 slot B
+    const int q = warp & 3;                  // TMEM lane quadrant
+    const int half = ((warp - 2) >> 2) & 1;  // which 32 of the chunk's 64 columns
     const int row = q * 32 + lane;       // row of the tile, TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
     bool ok = true;
-    auto build_onehot = [&](int r, int64_t p) {
+    // The type id of this thread's row in slot r of pair p (-1 past the end).
+    // Loaded a pair ahead of its use, so its latency is hidden.
+    auto load_type = [&](int r, int64_t p) -> int {
+      const int64_t gr = (2 * p + r) * 128 + row;
+      return (half == 0 && p < a.pairs && gr < a.rows) ? static_cast<int>(__ldg(a.types + gr)) : -1;
+    };
+    auto build_onehot = [&](int r, int t) {
       if (half == 0) {
-        const int64_t gr = (2 * p + r) * 128 + row;
-        int t = -1;
-        if (gr < a.rows) {
-          t = a.types[gr];
-          if (t >= a.n_types) {
-            atomicOr(sticky, DEVFLAG_ACTION_TYPE);
-            t = -1;
-          }
+        if (t >= a.n_types) {
+          atomicOr(sticky, DEVFLAG_ACTION_TYPE);
+          t = -1;
         }
         uint32_t w[8];  // bf16 1.0 in column t, zeros elsewhere
 #pragma unroll
@@ -336,84 +389,72 @@ __global__ void __launch_bounds__(kActThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(oh_full + r);
     };
+    const int r = slot;
     uint32_t g = 0;
     for (int64_t p = first, i = 0; ok && p < a.pairs; p += step, ++i) {
-      if (i == 0) {
-        build_onehot(0, p);
-        build_onehot(1, p);
-      }
+      if (i == 0) build_onehot(r, load_type(r, p));
       const int64_t pn = p + step;
-      for (int c = 0; c < C && ok; ++c, ++g) {
-        for (int r = 0; r < 2; ++r) {
-          if (!mbar_wait(uv_full + r, g & 1, abort_flag, sticky)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          uint32_t u[32], v[32];
-          tmem_ld32(lane_base + r * 256 + half * 32, u);
-          tmem_ld32(lane_base + r * 256 + 64 + half * 32, v);
-          tmem_wait_ld();
-          tmem_pin32(u);
-          tmem_pin32(v);
-          const uint32_t gb = sbase + Pl::kG + r * Pl::kEBox;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t o[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int k = 8 * j + 2 * e;
-              o[e] = gate_pair(__uint_as_float(u[k]), __uint_as_float(v[k]),
-                               __uint_as_float(u[k + 1]), __uint_as_float(v[k + 1]));
-            }
-            st_shared_v4(gb + swz128(row, half * 4 + j), o[0], o[1], o[2], o[3]);
-          }
-          fence_proxy_async_smem();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(epi_done + r);
-          // The last chunk's U, V were this slot's last use of its one-hot
-          // rows: build the next pair's now, while the products finish.
-          if (c == C - 1 && pn < a.pairs) build_onehot(r, pn);
-        }
-      }
-      if (!ok) break;
-      for (int r = 0; r < 2; ++r) {
-        if (!mbar_wait(y_full + r, i & 1, abort_flag, sticky)) {
+      const int tn = load_type(r, pn);
+      for (int c = 0; c < C; ++c, ++g) {
+        if (!mbar_wait(uv_full + r, g & 1, abort_flag, sticky)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int64_t gr = (2 * p + r) * 128 + row;
-        constexpr int kCols = D / 2;  // this thread's half of the row
+        uint32_t u[32], v[32];
+        tmem_ld32(lane_base + r * 256 + half * 32, u);
+        tmem_ld32(lane_base + r * 256 + 64 + half * 32, v);
+        tmem_wait_ld();
+        tmem_pin32(u);
+        tmem_pin32(v);
+        const uint32_t gb = sbase + Pl::kG + r * Pl::kEBox;
 #pragma unroll
-        for (int cc = 0; cc < kCols / 32; ++cc) {
-          uint32_t y[32];
-          tmem_ld32(lane_base + r * 256 + 128 + half * kCols + cc * 32, y);
-          tmem_wait_ld();
-          tmem_pin32(y);
-          if (gr < a.rows) {
-            const int col0 = half * kCols + cc * 32;
-            const uint4* src = reinterpret_cast<const uint4*>(a.E + gr * D + col0);
-            uint4* dst = reinterpret_cast<uint4*>(a.X + gr * D + col0);
+        for (int j = 0; j < 4; ++j) {
+          uint32_t o[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint4 ev = src[j];
-              const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
-              uint32_t o[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float lo = __uint_as_float(ew[e] << 16), hi = __uint_as_float(ew[e] & 0xFFFF0000u);
-                o[e] = pack_bf16x2(__uint_as_float(y[8 * j + 2 * e]) + lo,
-                                   __uint_as_float(y[8 * j + 2 * e + 1]) + hi);
-              }
-              dst[j] = make_uint4(o[0], o[1], o[2], o[3]);
-            }
+          for (int e = 0; e < 4; ++e) {
+            const int k = 8 * j + 2 * e;
+            o[e] = gate_pair(__uint_as_float(u[k]), __uint_as_float(v[k]),
+                             __uint_as_float(u[k + 1]), __uint_as_float(v[k + 1]));
           }
+          st_shared_v4(gb + swz128(row, half * 4 + j), o[0], o[1], o[2], o[3]);
         }
+        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(y_empty + r);
+        if (lane == 0) mbar_arrive(epi_done + r);
+        // The last chunk's U, V were this slot's last use of its one-hot
+        // rows: build the next pair's now, while the products finish.
+        if (c == C - 1 && pn < a.pairs) build_onehot(r, tn);
+      }
+      if (!ok || !mbar_wait(y_full + r, i & 1, abort_flag, sticky)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      constexpr int kCols = D / 2;  // this thread's half of the row
+      const int64_t gr = (2 * p + r) * 128 + row;
+#pragma unroll
+      for (int cc = 0; cc < kCols / 32; ++cc) {
+        uint32_t y[32];
+        tmem_ld32(lane_base + r * 256 + 128 + half * kCols + cc * 32, y);
+        tmem_wait_ld();
+        tmem_pin32(y);
+        if (cc == kCols / 32 - 1) {
+          // Y (which already holds e) is in registers: the slot's TMEM is free.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(y_empty + r);
+        }
+        if (gr < a.rows) {
+          uint4* dst = reinterpret_cast<uint4*>(a.X + gr * D + half * kCols + cc * 32);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(pack_bf16x2(__uint_as_float(y[8 * j]), __uint_as_float(y[8 * j + 1])),
+                                pack_bf16x2(__uint_as_float(y[8 * j + 2]), __uint_as_float(y[8 * j + 3])),
+                                pack_bf16x2(__uint_as_float(y[8 * j + 4]), __uint_as_float(y[8 * j + 5])),
+                                pack_bf16x2(__uint_as_float(y[8 * j + 6]), __uint_as_float(y[8 * j + 7])));
+        }
       }
     }
   }
@@ -481,7 +522,6 @@ sa_status action_fuse_enqueue(const sa_action_s* act, const void* E, const uint8
   if (!make_tmap_bf16(&tm_e, E, static_cast<uint64_t>(rows), static_cast<uint64_t>(act->d), 128))
     return SA_ERR_CUDA;
   ActArgs args;
-  args.E = static_cast<const uint16_t*>(E);
   args.types = types;
   args.X = static_cast<uint16_t*>(X);
   args.rows = rows;
