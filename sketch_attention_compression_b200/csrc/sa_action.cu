@@ -20,11 +20,12 @@
 // warps 2-9 gate slot A and warps 10-17 slot B, so that the two slots'
 // epilogues overlap.  Per slot and chunk c:
 //   [U | V] = E [W1_c | W3_c] + onehot [T1_c | T3_c]   M 128, N 128 (TMEM)
-//   G = SiLU(U) * V                   epilogue: bf16 into shared memory
-//   Y += G W2_c                       M 128, N d, K 64              (TMEM)
+//   G = SiLU(U) * V                   epilogue: bf16 pairs back into TMEM
+//   Y += G W2_c                       M 128, N d, K 64, A from TMEM (TMEM)
 // U and V are one product (N = 128) so that each K-step reads the E slice
-// from shared memory once: with N = 64 products the operand reads, not the
-// tensor cores, set the pace.
+// from shared memory once, and G never passes through shared memory: at
+// these shapes the shared-memory operand traffic, not the tensor cores, sets
+// the pace.
 // The residual is a product too: after the first chunk, Y += E I_16 slice
 // by slice (M 128, N 16, K 16 per 16 columns of E), from the E tile already
 // in shared memory, so that the epilogue only rounds Y to bf16 and stores
@@ -65,8 +66,7 @@ struct ActPlan {
   static constexpr int kEBox = 128 * 128;      // 128 rows x 64 bf16
   static constexpr int kE = 0;                 // 2 slots x D/64 boxes
   static constexpr int kESlot = (D / 64) * kEBox;
-  static constexpr int kG = kE + 2 * kESlot;   // 2 slots x one 128 x 64 box
-  static constexpr int kW = kG + 2 * kEBox;    // 2 weight stages
+  static constexpr int kW = kE + 2 * kESlot;   // 2 weight stages
   static constexpr int kWBox = kHc * 128;      // 64 rows x 64 bf16
   // Inside a stage: per 64 columns of K, the W1 box then the W3 box, so that
   // [W1_c ; W3_c] is one 128-row B operand and U, V one N = 128 product.
@@ -97,10 +97,6 @@ struct ActArgs {
   int n_types;
   uint32_t* flags;         // may be null
 };
-
-__device__ __forceinline__ uint32_t swz128(int r, int u) {
-  return (r >> 3) * 1024 + (r & 7) * 128 + ((u ^ (r & 7)) << 4);
-}
 
 __device__ __forceinline__ uint32_t swz32(int r, int u) {
   return r * 32 + ((u ^ ((r >> 2) & 1)) << 4);
@@ -295,13 +291,15 @@ __global__ void __launch_bounds__(kActThreads, 1)
         for (int ks = 0; ks < D / 16; ++ks)
           mma_bf16_ss(tmem + r * 256 + 128 + ks * 16, de + kstep(ks, Pl::kEBox), di, idesc_i, 1u);
       };
+      // Y += G W2_c with G read from TMEM: hidden columns 32 h .. 32 h + 31
+      // are bf16 pairs in U's columns 32 h .. 32 h + 15 (h = 0, 1).
       auto mma2 = [&](int r, uint32_t gc, bool acc) {
         const uint32_t st = sbase + Pl::kW + (gc & 1) * Pl::kStage;
-        const uint64_t dg = smem_desc(sbase + Pl::kG + r * Pl::kEBox, 16, 1024, 2);
         const uint64_t d2 = smem_desc(st + Pl::kW2, 16, 1024, 2);
 #pragma unroll
         for (int ks = 0; ks < kHc / 16; ++ks)
-          mma_bf16_ss(tmem + r * 256 + 128, dg + kstep(ks, Pl::kEBox), d2 + kstep(ks, D * 128),
+          mma_bf16_ts(tmem + r * 256 + 128, tmem + r * 256 + (ks >> 1) * 32 + (ks & 1) * 8,
+                      d2 + kstep(ks, D * 128),
                       idesc_y, (acc || ks > 0) ? 1u : 0u);
       };
       for (int64_t p = first, i = 0; ok && p < a.pairs; p += step, ++i) {
@@ -407,19 +405,16 @@ __global__ void __launch_bounds__(kActThreads, 1)
         tmem_wait_ld();
         tmem_pin32(u);
         tmem_pin32(v);
-        const uint32_t gb = sbase + Pl::kG + r * Pl::kEBox;
+        // G (this thread's 32 hidden columns as 16 bf16 pairs) goes over the
+        // first half of the U columns this thread read, where the Y product
+        // reads it as its A operand.
+        uint32_t o[16];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t o[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int k = 8 * j + 2 * e;
-            o[e] = gate_pair(__uint_as_float(u[k]), __uint_as_float(v[k]),
-                             __uint_as_float(u[k + 1]), __uint_as_float(v[k + 1]));
-          }
-          st_shared_v4(gb + swz128(row, half * 4 + j), o[0], o[1], o[2], o[3]);
-        }
-        fence_proxy_async_smem();
+        for (int e = 0; e < 16; ++e)
+          o[e] = gate_pair(__uint_as_float(u[2 * e]), __uint_as_float(v[2 * e]),
+                           __uint_as_float(u[2 * e + 1]), __uint_as_float(v[2 * e + 1]));
+        tmem_st16(lane_base + r * 256 + half * 32, o);
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(epi_done + r);
