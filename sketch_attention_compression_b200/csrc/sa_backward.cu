@@ -43,7 +43,7 @@
 namespace sa {
 namespace {
 
-constexpr int kBwdThreads = 256;  // warps 0-3 roles, 4-7 one softmax group
+constexpr int kBwdThreads = 384;  // warps 0-3 roles, 4-11 the softmax group (two warps per row)
 constexpr int kBwdStages = 2;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -56,7 +56,10 @@ struct BwdPlan {
   static constexpr int kX = kG + (D / 64) * kQBox;          // stages, D / 64 boxes each
   static constexpr int kAS = kX + kBwdStages * (D / 64) * kXBox;  // [A | dS']: 2 KM / 64 boxes
   static constexpr int kGv = kAS + (2 * KM / 64) * kXBox;   // g_b: KM floats
-  static constexpr int kBars = kGv + KM * 4;
+  // Row statistics the two halves of a row swap: [tile parity][half][row]
+  // (max, sum of exponentials, sum of exponentials times dA + g, unused).
+  static constexpr int kXch = kGv + KM * 4;
+  static constexpr int kBars = kXch + 2 * 2 * 128 * 16;
   static constexpr int kSmem = kBars + 256;
   static_assert(kSmem <= 232448, "shared memory budget");
   static constexpr uint32_t kColS = 0, kColDA = KM, kColDX = 2 * KM, kColR = 2 * KM + D;
@@ -115,7 +118,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* dx_empty = dx_full + 1;   // dX_t drained
   uint64_t* r_full = dx_empty + 1;    // [2] by segment parity: R complete
   uint64_t* r_empty = r_full + 2;     // R drained
-  uint64_t* drain = r_empty + 1;      // abort path: the issuer's MMAs done
+  uint64_t* xch_full = r_empty + 1;   // [2] by tile parity: both halves' row statistics stored
+  uint64_t* as_empty = xch_full + 2;  // MMA3 and MMA4 of a tile have read [A | dS']
+  uint64_t* drain = as_empty + 1;     // abort path: the issuer's MMAs done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   int64_t* range_slot = reinterpret_cast<int64_t*>(tmem_slot + 2);  // R0, R1, b0
@@ -136,13 +141,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(gq_full, 2);
     mbar_init(g_empty, 1);
     mbar_init(s_full, 1);
-    mbar_init(s_empty, 4);
-    mbar_init(p_full, 4);
+    mbar_init(s_empty, 8);
+    mbar_init(p_full, 8);
     mbar_init(dx_full, 1);
-    mbar_init(dx_empty, 4);
+    mbar_init(dx_empty, 8);
     mbar_init(&r_full[0], 1);
     mbar_init(&r_full[1], 1);
-    mbar_init(r_empty, 4);
+    mbar_init(r_empty, 8);
+    mbar_init(&xch_full[0], 8);
+    mbar_init(&xch_full[1], 8);
+    mbar_init(as_empty, 1);
     mbar_init(drain, 1);
     *abort_flag = 0u;
     fence_mbar_init();
@@ -241,31 +249,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       SegmentWalker w{a.offsets, a.batch, R0, R1, b0};
       int64_t user, s, e, lo, hi;
       uint32_t t = 0, seg = 0;
+      // MMA1 and MMA1' of tile t + 1 are issued as soon as the softmax has
+      // read tile t's S^T and dA^T out of TMEM (and before tile t's MMA3 and
+      // MMA4, which wait for the softmax to finish), so they run under the
+      // softmax of tile t.  A segment's first tile waits for its G_b (and
+      // Q''_b), which reuse the previous segment's buffers: no look-ahead
+      // across a segment boundary.
+      auto issue_s = [&](uint32_t tt) {
+        const uint64_t xs = xk + (((tt % S) * (D / 64) * Pl::kXBox) >> 4);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t ao = ((ks >> 2) * Pl::kXBox + (ks & 3) * 32) >> 4;
+          const uint64_t bo = ((ks >> 2) * Pl::kQBox + (ks & 3) * 32) >> 4;
+          mma_bf16_ss(tmem + Pl::kColS, xs + ao, qk + bo, idesc_s, ks > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t ao = ((ks >> 2) * Pl::kXBox + (ks & 3) * 32) >> 4;
+          const uint64_t bo = ((ks >> 2) * Pl::kQBox + (ks & 3) * 32) >> 4;
+          mma_bf16_ss(tmem + Pl::kColDA, xs + ao, gk + bo, idesc_s, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full);
+      };
+      bool s_ahead = false;  // MMA1/MMA1' of tile t already issued
       while (ok && w.next(user, s, e, lo, hi)) {
         for (int64_t r = s; r < e; r += kTileRows, ++t) {
           const int st = t % S;
           const bool first = r == s, last = r + kTileRows >= e;
-          const uint64_t xs = xk + ((st * (D / 64) * Pl::kXBox) >> 4);
-          if ((first && !mbar_wait(gq_full, seg & 1u, abort_flag, sticky)) ||
-              !mbar_wait(&x_full[st], (t / S) & 1u, abort_flag, sticky) ||
-              (t > 0 && !mbar_wait(s_empty, (t - 1) & 1u, abort_flag, sticky))) {
-            ok = false;
-            break;
+          if (!s_ahead) {
+            if ((first && !mbar_wait(gq_full, seg & 1u, abort_flag, sticky)) ||
+                !mbar_wait(&x_full[st], (t / S) & 1u, abort_flag, sticky) ||
+                (t > 0 && !mbar_wait(s_empty, (t - 1) & 1u, abort_flag, sticky))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(t);
           }
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint64_t ao = ((ks >> 2) * Pl::kXBox + (ks & 3) * 32) >> 4;
-            const uint64_t bo = ((ks >> 2) * Pl::kQBox + (ks & 3) * 32) >> 4;
-            mma_bf16_ss(tmem + Pl::kColS, xs + ao, qk + bo, idesc_s, ks > 0 ? 1u : 0u);
+          s_ahead = false;
+          if (!last) {
+            if (!mbar_wait(&x_full[(t + 1) % S], ((t + 1) / S) & 1u, abort_flag, sticky) ||
+                !mbar_wait(s_empty, t & 1u, abort_flag, sticky)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(t + 1);
+            s_ahead = true;
           }
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint64_t ao = ((ks >> 2) * Pl::kXBox + (ks & 3) * 32) >> 4;
-            const uint64_t bo = ((ks >> 2) * Pl::kQBox + (ks & 3) * 32) >> 4;
-            mma_bf16_ss(tmem + Pl::kColDA, xs + ao, gk + bo, idesc_s, ks > 0 ? 1u : 0u);
-          }
-          mma_commit(s_full);
           if (!mbar_wait(p_full, t & 1u, abort_flag, sticky) ||
               (t > 0 && !mbar_wait(dx_empty, (t - 1) & 1u, abort_flag, sticky)) ||
               (first && !mbar_wait(r_empty, (seg & 1u) ^ 1u, abort_flag, sticky))) {
@@ -291,6 +322,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mma_bf16_ss(tmem + Pl::kColR, dsmn + ((ks * 2048) >> 4), xmn + ((ks * 2048) >> 4),
                         idesc_r, (!first || ks > 0) ? 1u : 0u);
           mma_commit(&x_empty[st]);
+          mma_commit(as_empty);
           if (last) {
             mma_commit(&r_full[seg & 1u]);
             mma_commit(g_empty);
@@ -301,9 +333,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- softmax, dS, drains
+    // Two warps per TMEM lane quarter: warp half hf takes prototypes
+    // [hf KM/2, (hf + 1) KM/2) of its 32 rows, and the two halves of a row
+    // swap (max, sum of exponentials, sum of exponentials times (dA + g))
+    // once per tile through shared memory, behind a bounded mbarrier wait.
     const int q = warp & 3;
+    const int hf = (warp - 4) >> 2;
     const int row = q * 32 + lane;
+    constexpr int HW = KM / 2, HC = HW / 32;
+    const int j0 = hf * HW;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    float4* xch = reinterpret_cast<float4*>(smem + Pl::kXch);
     SegmentWalker w{a.offsets, a.batch, R0, R1, b0};
     int64_t user, s, e, lo, hi;
     uint32_t t = 0, seg = 0;
@@ -320,117 +360,164 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           break;
         }
         tc_fence_after();
-        // A = softmax over the prototypes (exp2: Q'' carries log2 e).
-        // Two passes over the logits in TMEM (maximum, then exponentials),
-        // so that the row's logits and weights are never both in registers.
-        float av[KM];
-        {
-          float mx = -INFINITY;
+        // This half's logits and dA columns (exp2 softmax: Q'' carries log2 e).
+        uint32_t sv[HC][32], dv[HC][32];
 #pragma unroll
-          for (int cc = 0; cc < KM / 32; ++cc) {
-            uint32_t sr[32];
-            tmem_ld32(lane_addr + Pl::kColS + cc * 32, sr);
-            tmem_wait_ld();
-            tmem_pin32(sr);
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (FULL || cc * 32 + i < k) mx = fmaxf(mx, __uint_as_float(sr[i]));
-          }
-          float z = 0.f;
-#pragma unroll
-          for (int cc = 0; cc < KM / 32; ++cc) {
-            uint32_t sr[32];
-            tmem_ld32(lane_addr + Pl::kColS + cc * 32, sr);
-            tmem_wait_ld();
-            tmem_pin32(sr);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int j = cc * 32 + i;
-              av[j] = (FULL || j < k) ? ex2_approx(__uint_as_float(sr[i]) - mx) : 0.f;
-              z += av[j];
-            }
-          }
-          const float inv = valid ? 1.0f / z : 0.f;
-#pragma unroll
-          for (int j = 0; j < KM; ++j) av[j] = valid ? av[j] * inv : 0.f;
+        for (int cc = 0; cc < HC; ++cc) {
+          tmem_ld32(lane_addr + Pl::kColS + j0 + cc * 32, sv[cc]);
+          tmem_ld32(lane_addr + Pl::kColDA + j0 + cc * 32, dv[cc]);
         }
-        // c = sum_j A_j (dA_j + g_j), then dS'_j = ln2 A_j (dA_j + g_j - c).
-        float cs = 0.f;
+        tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < KM / 32; ++cc) {
-          uint32_t dv[32];
-          tmem_ld32(lane_addr + Pl::kColDA + cc * 32, dv);
-          tmem_wait_ld();
-          tmem_pin32(dv);
+        for (int cc = 0; cc < HC; ++cc) {
+          tmem_pin32(sv[cc]);
+          tmem_pin32(dv[cc]);
+        }
+        tc_fence_before();
+        warp_arrive(s_empty, lane);  // S^T and dA^T are in registers
+        float mx = -INFINITY;
+#pragma unroll
+        for (int cc = 0; cc < HC; ++cc)
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            cs += av[cc * 32 + i] * (__uint_as_float(dv[i]) + g_s[cc * 32 + i]);
-        }
-        // A into the first KM / 64 boxes of the tile, dS' into the others.
+            if (FULL || j0 + cc * 32 + i < k) mx = fmaxf(mx, __uint_as_float(sv[cc][i]));
+        float z = 0.f, wsum = 0.f;
 #pragma unroll
-        for (int cc = 0; cc < KM / 32; ++cc) {
-          uint32_t dv[32];
-          tmem_ld32(lane_addr + Pl::kColDA + cc * 32, dv);
-          tmem_wait_ld();
-          tmem_pin32(dv);
+        for (int cc = 0; cc < HC; ++cc) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int j = j0 + cc * 32 + i;
+            const float ev = (FULL || j < k) ? ex2_approx(__uint_as_float(sv[cc][i]) - mx) : 0.f;
+            sv[cc][i] = __float_as_uint(ev);
+            z += ev;
+            wsum = fmaf(ev, __uint_as_float(dv[cc][i]) + g_s[j], wsum);
+          }
+        }
+        const uint32_t par = t & 1u;
+        xch[(par * 2 + hf) * 128 + row] = make_float4(mx, z, wsum, 0.f);
+        warp_arrive(&xch_full[par], lane);
+        if (!warp_wait(&xch_full[par], (t >> 1) & 1u, abort_flag, sticky)) {
+          ok = false;
+          break;
+        }
+        const float4 o = xch[(par * 2 + (hf ^ 1)) * 128 + row];
+        // Combine: M = max of both halves; a half with no prototype has max
+        // -inf and contributes nothing.
+        const float M = fmaxf(mx, o.x);
+        const float sa_own = mx == -INFINITY ? 0.f : ex2_approx(mx - M);
+        const float sa_oth = o.x == -INFINITY ? 0.f : ex2_approx(o.x - M);
+        const float Z = z * sa_own + o.y * sa_oth;
+        const float inv = valid ? 1.0f / Z : 0.f;
+        const float scale = sa_own * inv;
+        const float cs = (wsum * sa_own + o.z * sa_oth) * inv;
+        // The shared tile is free once the previous tile's MMA3 and MMA4
+        // have read it.
+        if (t > 0 && !warp_wait(as_empty, (t - 1) & 1u, abort_flag, sticky)) {
+          ok = false;
+          break;
+        }
+        // A and dS' = ln2 A (dA + g - c) of this half, into the shared tile
+        // (A in the first KM / 64 boxes, dS' in the others).
+#pragma unroll
+        for (int cc = 0; cc < HC; ++cc) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             uint32_t wa[4], wd[4];
 #pragma unroll
             for (int ee = 0; ee < 4; ++ee) {
-              const int j = cc * 32 + u * 8 + 2 * ee;
-              const float d0 = kLn2 * av[j] * (__uint_as_float(dv[u * 8 + 2 * ee]) + g_s[j] - cs);
-              const float d1 =
-                  kLn2 * av[j + 1] * (__uint_as_float(dv[u * 8 + 2 * ee + 1]) + g_s[j + 1] - cs);
-              wa[ee] = pack_bf16x2(av[j], av[j + 1]);
+              const int i = u * 8 + 2 * ee;
+              const int j = j0 + cc * 32 + i;
+              const float a0 = valid ? __uint_as_float(sv[cc][i]) * scale : 0.f;
+              const float a1 = valid ? __uint_as_float(sv[cc][i + 1]) * scale : 0.f;
+              const float d0 = kLn2 * a0 * (__uint_as_float(dv[cc][i]) + g_s[j] - cs);
+              const float d1 = kLn2 * a1 * (__uint_as_float(dv[cc][i + 1]) + g_s[j + 1] - cs);
+              wa[ee] = pack_bf16x2(a0, a1);
               wd[ee] = valid ? pack_bf16x2(d0, d1) : 0u;
             }
-            const int col = cc * 32 + u * 8;  // prototype of the unit's first element
+            const int col = j0 + cc * 32 + u * 8;  // prototype of the unit's first element
             const uint32_t ua = sbase + Pl::kAS + (col >> 6) * Pl::kXBox + swz(row, (col & 63) >> 3);
             const uint32_t ud = ua + (KM / 64) * Pl::kXBox;
             st_shared_v4(ua, wa[0], wa[1], wa[2], wa[3]);
             st_shared_v4(ud, wd[0], wd[1], wd[2], wd[3]);
           }
         }
-        tc_fence_before();
-        warp_arrive(s_empty, lane);
-        if (!valid) {
-          // Rows past the segment's end: cleared (0 * NaN is NaN in MMA4).
+        if (!valid && (D / 64 > 1 || hf == 0)) {
+          // Rows past the segment's end: cleared (0 * NaN is NaN in MMA4);
+          // each half clears one 64-column box (d = 64: the first half).
+          const int cb = D / 64 > 1 ? hf : 0;
+          const uint32_t xrow = sbase + Pl::kX + (st * (D / 64) + cb) * Pl::kXBox + row * 128;
 #pragma unroll
-          for (int cb = 0; cb < D / 64; ++cb) {
-            const uint32_t xrow = sbase + Pl::kX + (st * (D / 64) + cb) * Pl::kXBox + row * 128;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) st_shared_v4(xrow + i * 16, 0u, 0u, 0u, 0u);
-          }
+          for (int i = 0; i < 8; ++i) st_shared_v4(xrow + i * 16, 0u, 0u, 0u, 0u);
         }
         fence_proxy_async_smem();
         warp_arrive(p_full, lane);
 
-        // dX_t: TMEM row -> bf16 -> global.
-        if (!warp_wait(dx_full, t & 1u, abort_flag, sticky)) { ok = false; break; }
+        // dX_t: TMEM row -> bf16 -> global; each half drains d / 2 columns.
+        // With 128 prototypes the warp stages its 32 rows in the part of
+        // the [A | dS'] tile that it alone writes (A's box hf, rows 32 q ..),
+        // free once MMA3 has read it, then stores whole rows: 128 (d = 64:
+        // 64) bytes of a row per 8 (4) lanes, instead of 16 bytes of 32 rows.
+        // With 64 prototypes both halves write each A and dS' box, so the
+        // rows go straight from registers.
+        if (!warp_wait(dx_full, t & 1u, abort_flag, sticky)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
+        {
+          constexpr int XC = D / 64;      // 32-column chunks per half
+          constexpr int U = D / 16;       // 16-byte units per half row
+          uint32_t xv[XC][32];
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t xv[32];
-          tmem_ld32(lane_addr + Pl::kColDX + cc * 32, xv);
+          for (int cc = 0; cc < XC; ++cc) tmem_ld32(lane_addr + Pl::kColDX + hf * (D / 2) + cc * 32, xv[cc]);
           tmem_wait_ld();
-          tmem_pin32(xv);
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(ba.dX + (r + row) * D + cc * 32);
+#pragma unroll
+          for (int cc = 0; cc < XC; ++cc) tmem_pin32(xv[cc]);
+          tc_fence_before();
+          warp_arrive(dx_empty, lane);
+          if constexpr (KM == 64) {
+            if (valid) {
+#pragma unroll
+              for (int cc = 0; cc < XC; ++cc) {
+                uint4* dst = reinterpret_cast<uint4*>(ba.dX + (r + row) * D + hf * (D / 2) + cc * 32);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  dst[u] = make_uint4(
+                      pack_bf16x2(__uint_as_float(xv[cc][8 * u]), __uint_as_float(xv[cc][8 * u + 1])),
+                      pack_bf16x2(__uint_as_float(xv[cc][8 * u + 2]), __uint_as_float(xv[cc][8 * u + 3])),
+                      pack_bf16x2(__uint_as_float(xv[cc][8 * u + 4]), __uint_as_float(xv[cc][8 * u + 5])),
+                      pack_bf16x2(__uint_as_float(xv[cc][8 * u + 6]), __uint_as_float(xv[cc][8 * u + 7])));
+              }
+            }
+          } else {
+          const uint32_t box = sbase + Pl::kAS + hf * Pl::kXBox;
+#pragma unroll
+          for (int cc = 0; cc < XC; ++cc)
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-              dst[u] = make_uint4(pack_bf16x2(__uint_as_float(xv[8 * u]), __uint_as_float(xv[8 * u + 1])),
-                                  pack_bf16x2(__uint_as_float(xv[8 * u + 2]), __uint_as_float(xv[8 * u + 3])),
-                                  pack_bf16x2(__uint_as_float(xv[8 * u + 4]), __uint_as_float(xv[8 * u + 5])),
-                                  pack_bf16x2(__uint_as_float(xv[8 * u + 6]), __uint_as_float(xv[8 * u + 7])));
+              st_shared_v4(box + swz(row, cc * 4 + u),
+                           pack_bf16x2(__uint_as_float(xv[cc][8 * u]), __uint_as_float(xv[cc][8 * u + 1])),
+                           pack_bf16x2(__uint_as_float(xv[cc][8 * u + 2]), __uint_as_float(xv[cc][8 * u + 3])),
+                           pack_bf16x2(__uint_as_float(xv[cc][8 * u + 4]), __uint_as_float(xv[cc][8 * u + 5])),
+                           pack_bf16x2(__uint_as_float(xv[cc][8 * u + 6]), __uint_as_float(xv[cc][8 * u + 7])));
+          __syncwarp();
+          constexpr int RPI = 32 / U;  // rows per warp store
+#pragma unroll
+          for (int it = 0; it < U; ++it) {
+            const int rr = q * 32 + it * RPI + lane / U;
+            const int u = lane % U;
+            if (rr < nrows) {
+              const uint4 v = ld_shared_v4u(box + swz(rr, u));
+              *reinterpret_cast<uint4*>(ba.dX + (r + rr) * D + hf * (D / 2) + u * 8) = v;
+            }
+          }
+          __syncwarp();
           }
         }
-        tc_fence_before();
-        warp_arrive(dx_empty, lane);
 
         if (last) {
           // R_b (ln 2 dL/dQ') to the outputs or to this user's partial slot;
-          // the mass outputs carry zeros.
+          // the mass outputs carry zeros.  Each half drains d / 2 columns.
           if (!warp_wait(&r_full[seg & 1u], (seg >> 1) & 1u, abort_flag, sticky)) { ok = false; break; }
           tc_fence_after();
           const int64_t slotp = segment_slot(c, lo, hi, R0, R1);
@@ -439,20 +526,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int j = (KM == 128 ? q * 32 : q * 16) + lane;
           const bool has = (KM == 128 || lane < 16) && j < k;
 #pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
+          for (int cc = 0; cc < D / 64; ++cc) {
             uint32_t v[32];
-            tmem_ld32(lane_addr + Pl::kColR + cc * 32, v);
+            tmem_ld32(lane_addr + Pl::kColR + hf * (D / 2) + cc * 32, v);
             tmem_wait_ld();
             tmem_pin32(v);
             if (has) {
-              float4* dst = reinterpret_cast<float4*>(dr + static_cast<int64_t>(j) * D + cc * 32);
+              float4* dst = reinterpret_cast<float4*>(dr + static_cast<int64_t>(j) * D + hf * (D / 2) +
+                                                      cc * 32);
 #pragma unroll
               for (int w4 = 0; w4 < 8; ++w4)
                 dst[w4] = make_float4(__uint_as_float(v[4 * w4]), __uint_as_float(v[4 * w4 + 1]),
                                       __uint_as_float(v[4 * w4 + 2]), __uint_as_float(v[4 * w4 + 3]));
             }
           }
-          if (has) dm[j] = 0.f;
+          if (has && hf == 0) dm[j] = 0.f;
           tc_fence_before();
           warp_arrive(r_empty, lane);
         }
@@ -505,10 +593,7 @@ __global__ void bwd_prep_kernel(const float* __restrict__ Gin, const float* __re
 
 }  // namespace
 
-// C[b] = alpha * op(A[b]) op(B[b]) (+ C[b] when accumulate), row-major, fp64
-// accumulation; op transposes when the flag is set.  A[b] is m x l after
-// op, B[b] is l x n after op; `batch` independent products (strides 0 for a
-// shared operand).  Small products only (the parameter gradients).
+// out = sum over b of R[b] (n entries each), fp64 accumulation in user order.
 __global__ void sum_users_kernel(const float* __restrict__ R, int64_t batch, int64_t n,
                                  float* __restrict__ out) {
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
@@ -526,36 +611,84 @@ cudaError_t launch_sum_users(const float* R, int64_t batch, int64_t n, float* ou
   return cudaGetLastError();
 }
 
-__global__ void bwd_gemm_kernel(const float* __restrict__ A, int64_t sa, bool ta,
-                                const float* __restrict__ B, int64_t sb, bool tb,
-                                float* __restrict__ C, int64_t sc, int m, int n, int l,
-                                double alpha, bool accumulate) {
-  const int64_t b = blockIdx.y;
+// C[b] = alpha * op(A[b]) op(B[b]) (+ C[b] when accumulate), row-major, fp64
+// accumulation; op transposes when the flag is set.  A[b] is m x l after
+// op, B[b] is l x n after op; `batch` independent products (strides 0 for a
+// shared operand).  Small products only (the parameter gradients).
+// Tiles of 32 x 32 outputs per block of 16 x 16 threads (2 x 2 each), the
+// shared dimension in steps of 32 through shared memory, loads coalesced
+// along whichever index is contiguous in memory.
+constexpr int kGemmTile = 32;
+
+__global__ void __launch_bounds__(256)
+    bwd_gemm_kernel(const float* __restrict__ A, int64_t sa, bool ta, const float* __restrict__ B,
+                    int64_t sb, bool tb, float* __restrict__ C, int64_t sc, int m, int n, int l,
+                    double alpha, bool accumulate) {
+  __shared__ float As[kGemmTile][kGemmTile + 1];  // [i][p]
+  __shared__ float Bs[kGemmTile][kGemmTile + 1];  // [p][j]
+  const int64_t b = blockIdx.z;
   const float* Ab = A + b * sa;
   const float* Bb = B + b * sb;
   float* Cb = C + b * sc;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-       e < static_cast<int64_t>(m) * n; e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int i = static_cast<int>(e / n), j = static_cast<int>(e % n);
-    double s = 0.0;
-    for (int p = 0; p < l; ++p) {
-      const double x = ta ? Ab[static_cast<int64_t>(p) * m + i] : Ab[static_cast<int64_t>(i) * l + p];
-      const double y = tb ? Bb[static_cast<int64_t>(j) * l + p] : Bb[static_cast<int64_t>(p) * n + j];
-      s += x * y;
+  const int i0 = blockIdx.y * kGemmTile, j0 = blockIdx.x * kGemmTile;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
+  for (int p0 = 0; p0 < l; p0 += kGemmTile) {
+    for (int idx = threadIdx.x; idx < kGemmTile * kGemmTile; idx += 256) {
+      const int x = idx % kGemmTile, y = idx / kGemmTile;  // x runs along contiguous memory
+      {
+        const int ii = ta ? x : y, pp = ta ? y : x;
+        const int gi = i0 + ii, gp = p0 + pp;
+        As[ii][pp] = (gi < m && gp < l)
+                         ? (ta ? Ab[static_cast<int64_t>(gp) * m + gi] : Ab[static_cast<int64_t>(gi) * l + gp])
+                         : 0.f;
+      }
+      {
+        const int pp = tb ? x : y, jj = tb ? y : x;
+        const int gp = p0 + pp, gj = j0 + jj;
+        Bs[pp][jj] = (gp < l && gj < n)
+                         ? (tb ? Bb[static_cast<int64_t>(gj) * l + gp] : Bb[static_cast<int64_t>(gp) * n + gj])
+                         : 0.f;
+      }
     }
-    const double v = alpha * s;
-    Cb[e] = static_cast<float>(accumulate ? Cb[e] + v : v);
+    __syncthreads();
+#pragma unroll 8
+    for (int pp = 0; pp < kGemmTile; ++pp) {
+      const double a0 = As[2 * ty][pp], a1 = As[2 * ty + 1][pp];
+      const double b0 = Bs[pp][2 * tx], b1 = Bs[pp][2 * tx + 1];
+      acc[0][0] = fma(a0, b0, acc[0][0]);
+      acc[0][1] = fma(a0, b1, acc[0][1]);
+      acc[1][0] = fma(a1, b0, acc[1][0]);
+      acc[1][1] = fma(a1, b1, acc[1][1]);
+    }
+    __syncthreads();
   }
+#pragma unroll
+  for (int u = 0; u < 2; ++u)
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const int i = i0 + 2 * ty + u, j = j0 + 2 * tx + v;
+      if (i < m && j < n) {
+        const int64_t e = static_cast<int64_t>(i) * n + j;
+        const double r = alpha * acc[u][v];
+        Cb[e] = static_cast<float>(accumulate ? Cb[e] + r : r);
+      }
+    }
 }
 
 cudaError_t launch_bwd_gemm(const float* A, int64_t sa, bool ta, const float* B, int64_t sb,
                             bool tb, float* C, int64_t sc, int m, int n, int l, double alpha,
                             bool accumulate, int64_t batch, cudaStream_t st) {
-  const int64_t elems = static_cast<int64_t>(m) * n;
-  const unsigned gx = static_cast<unsigned>((elems + 255) / 256 < 1024 ? (elems + 255) / 256 : 1024);
-  bwd_gemm_kernel<<<dim3(gx, static_cast<unsigned>(batch)), 256, 0, st>>>(
-      A, sa, ta, B, sb, tb, C, sc, m, n, l, alpha, accumulate);
-  return cudaGetLastError();
+  for (int64_t b0 = 0; b0 < batch; b0 += 65535) {  // grid z is at most 65535
+    const int64_t nb = batch - b0 < 65535 ? batch - b0 : 65535;
+    const dim3 grid(static_cast<unsigned>((n + kGemmTile - 1) / kGemmTile),
+                    static_cast<unsigned>((m + kGemmTile - 1) / kGemmTile), static_cast<unsigned>(nb));
+    bwd_gemm_kernel<<<grid, 256, 0, st>>>(A + b0 * sa, sa, ta, B + b0 * sb, sb, tb, C + b0 * sc, sc, m,
+                                          n, l, alpha, accumulate);
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_bwd_prep(const float* G, const float* g, int64_t batch, int k, int km, int d,
