@@ -81,7 +81,10 @@ struct ActPlan {
   static constexpr uint32_t kEBytes = kESlot;
   static constexpr int kOH = kW + 2 * kStage;  // 2 slots x 128 rows x 32 B
   static constexpr int kI = kOH + 2 * 128 * 32;  // I_16 (16 x 16 bf16, 32-byte swizzle)
-  static constexpr int kBars = kI + 1024;
+  // Store staging: per epilogue warp 32 rows x 32 columns of X (bf16).
+  static constexpr int kStg = kI + 1024;
+  static constexpr int kStgWarp = 32 * 64;
+  static constexpr int kBars = kStg + 16 * kStgWarp;
   // At least 116 KB, so that one CTA holds an SM (it allocates all of TMEM).
   static constexpr int kSmem = kBars + 256 > 118784 ? kBars + 256 : 118784;
   static_assert(kStage % 1024 == 0, "stage alignment");
@@ -428,7 +431,12 @@ __global__ void __launch_bounds__(kActThreads, 1)
       }
       tc_fence_after();
       constexpr int kCols = D / 2;  // this thread's half of the row
-      const int64_t gr = (2 * p + r) * 128 + row;
+      const int64_t gr0 = (2 * p + r) * 128;
+      // Each 32-column chunk goes through the warp's own staging area (row
+      // i at 64 i bytes, its four 16-byte units rotated by i / 2 so that a
+      // warp's stores spread over the banks), and out as whole 64-byte row
+      // pieces, 8 rows per warp store, instead of 16 bytes of 32 rows.
+      const uint32_t stg = sbase + Pl::kStg + (warp - 2) * Pl::kStgWarp;
 #pragma unroll
       for (int cc = 0; cc < kCols / 32; ++cc) {
         uint32_t y[32];
@@ -441,15 +449,28 @@ __global__ void __launch_bounds__(kActThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(y_empty + r);
         }
-        if (gr < a.rows) {
-          uint4* dst = reinterpret_cast<uint4*>(a.X + gr * D + half * kCols + cc * 32);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dst[j] = make_uint4(pack_bf16x2(__uint_as_float(y[8 * j]), __uint_as_float(y[8 * j + 1])),
-                                pack_bf16x2(__uint_as_float(y[8 * j + 2]), __uint_as_float(y[8 * j + 3])),
-                                pack_bf16x2(__uint_as_float(y[8 * j + 4]), __uint_as_float(y[8 * j + 5])),
-                                pack_bf16x2(__uint_as_float(y[8 * j + 6]), __uint_as_float(y[8 * j + 7])));
+        for (int j = 0; j < 4; ++j)
+          st_shared_v4(stg + lane * 64 + (((j + (lane >> 1)) & 3) << 4),
+                       pack_bf16x2(__uint_as_float(y[8 * j]), __uint_as_float(y[8 * j + 1])),
+                       pack_bf16x2(__uint_as_float(y[8 * j + 2]), __uint_as_float(y[8 * j + 3])),
+                       pack_bf16x2(__uint_as_float(y[8 * j + 4]), __uint_as_float(y[8 * j + 5])),
+                       pack_bf16x2(__uint_as_float(y[8 * j + 6]), __uint_as_float(y[8 * j + 7])));
+        __syncwarp();
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          const int i = it * 8 + (lane >> 2), j = lane & 3;  // staged row i, unit j
+          const int64_t gr = gr0 + q * 32 + i;
+          if (gr < a.rows) {
+            uint32_t v0, v1, v2, v3;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
+                         : "r"(stg + i * 64 + (((j + (i >> 1)) & 3) << 4)));
+            *reinterpret_cast<uint4*>(a.X + gr * D + half * kCols + cc * 32 + j * 8) =
+                make_uint4(v0, v1, v2, v3);
+          }
         }
+        __syncwarp();
       }
     }
   }
