@@ -381,16 +381,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (FULL || j0 + cc * 32 + i < k) mx = fmaxf(mx, __uint_as_float(sv[cc][i]));
+        // dv becomes dA + g (g_b read four at a time), sv the exponentials.
         float z = 0.f, wsum = 0.f;
 #pragma unroll
         for (int cc = 0; cc < HC; ++cc) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int j = j0 + cc * 32 + i;
-            const float ev = (FULL || j < k) ? ex2_approx(__uint_as_float(sv[cc][i]) - mx) : 0.f;
-            sv[cc][i] = __float_as_uint(ev);
-            z += ev;
-            wsum = fmaf(ev, __uint_as_float(dv[cc][i]) + g_s[j], wsum);
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 g4 = reinterpret_cast<const float4*>(g_s + j0 + cc * 32)[i4];
+            const float gg[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+            for (int i1 = 0; i1 < 4; ++i1) {
+              const int i = i4 * 4 + i1;
+              const int j = j0 + cc * 32 + i;
+              const float ev = (FULL || j < k) ? ex2_approx(__uint_as_float(sv[cc][i]) - mx) : 0.f;
+              const float dg = __uint_as_float(dv[cc][i]) + gg[i1];
+              sv[cc][i] = __float_as_uint(ev);
+              dv[cc][i] = __float_as_uint(dg);
+              z += ev;
+              wsum = fmaf(ev, dg, wsum);
+            }
           }
         }
         const uint32_t par = t & 1u;
@@ -426,11 +435,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
             for (int ee = 0; ee < 4; ++ee) {
               const int i = u * 8 + 2 * ee;
-              const int j = j0 + cc * 32 + i;
               const float a0 = valid ? __uint_as_float(sv[cc][i]) * scale : 0.f;
               const float a1 = valid ? __uint_as_float(sv[cc][i + 1]) * scale : 0.f;
-              const float d0 = kLn2 * a0 * (__uint_as_float(dv[cc][i]) + g_s[j] - cs);
-              const float d1 = kLn2 * a1 * (__uint_as_float(dv[cc][i + 1]) + g_s[j + 1] - cs);
+              const float d0 = kLn2 * a0 * (__uint_as_float(dv[cc][i]) - cs);
+              const float d1 = kLn2 * a1 * (__uint_as_float(dv[cc][i + 1]) - cs);
               wa[ee] = pack_bf16x2(a0, a1);
               wd[ee] = valid ? pack_bf16x2(d0, d1) : 0u;
             }
