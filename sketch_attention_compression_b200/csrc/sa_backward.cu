@@ -345,169 +345,207 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     float4* xch = reinterpret_cast<float4*>(smem + Pl::kXch);
     SegmentWalker w{a.offsets, a.batch, R0, R1, b0};
+    // Software-pipelined over tiles: while MMA3 and MMA4 of tile t run, the
+    // group already loads tile t + 1's logits and takes their exponentials;
+    // only then does it drain dX_t.  (The issuer has started MMA1 of tile
+    // t + 1 once the group released tile t's S^T and dA^T.)
+    uint32_t sv[HC][32];   // the current tile's exponentials (as float bits)
+    float mx = -INFINITY, z = 0.f;
+    // Loads this half's logits of the tile now in S^T and takes its
+    // maximum and exponentials (exp2 softmax: Q'' carries log2 e).
+    auto load_exps = [&]() {
+#pragma unroll
+      for (int cc = 0; cc < HC; ++cc) tmem_ld32(lane_addr + Pl::kColS + j0 + cc * 32, sv[cc]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int cc = 0; cc < HC; ++cc) tmem_pin32(sv[cc]);
+      mx = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < HC; ++cc)
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (FULL || j0 + cc * 32 + i < k) mx = fmaxf(mx, __uint_as_float(sv[cc][i]));
+      z = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < HC; ++cc)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float ev =
+              (FULL || j0 + cc * 32 + i < k) ? ex2_approx(__uint_as_float(sv[cc][i]) - mx) : 0.f;
+          sv[cc][i] = __float_as_uint(ev);
+          z += ev;
+        }
+    };
     int64_t user, s, e, lo, hi;
+    bool ok = w.next(user, s, e, lo, hi);
+    int64_t r = s;
     uint32_t t = 0, seg = 0;
-    bool ok = true;
-    while (ok && w.next(user, s, e, lo, hi)) {
-      for (int64_t r = s; r < e; r += kTileRows, ++t) {
-        const bool first = r == s, last = r + kTileRows >= e;
-        const int nrows = static_cast<int>((e - r) < kTileRows ? (e - r) : kTileRows);
-        const bool valid = row < nrows;
-        const int st = t % S;
+    bool have_s = false;
+    while (ok) {
+      const bool first = r == s, last = r + kTileRows >= e;
+      const int nrows = static_cast<int>((e - r) < kTileRows ? (e - r) : kTileRows);
+      const bool valid = row < nrows;
+      const int st = t % S;
+      if (!have_s) {
         if ((first && !warp_wait(gq_full, seg & 1u, abort_flag, sticky)) ||
             !warp_wait(s_full, t & 1u, abort_flag, sticky)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        // This half's logits and dA columns (exp2 softmax: Q'' carries log2 e).
-        uint32_t sv[HC][32], dv[HC][32];
+        load_exps();
+      }
+      // dA of this half (dv becomes dA + g, g_b read four at a time); then
+      // S^T and dA^T are free for the next tile's MMA1.
+      uint32_t dv[HC][32];
 #pragma unroll
-        for (int cc = 0; cc < HC; ++cc) {
-          tmem_ld32(lane_addr + Pl::kColS + j0 + cc * 32, sv[cc]);
-          tmem_ld32(lane_addr + Pl::kColDA + j0 + cc * 32, dv[cc]);
-        }
-        tmem_wait_ld();
+      for (int cc = 0; cc < HC; ++cc) tmem_ld32(lane_addr + Pl::kColDA + j0 + cc * 32, dv[cc]);
+      tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < HC; ++cc) {
-          tmem_pin32(sv[cc]);
-          tmem_pin32(dv[cc]);
-        }
-        tc_fence_before();
-        warp_arrive(s_empty, lane);  // S^T and dA^T are in registers
-        float mx = -INFINITY;
+      for (int cc = 0; cc < HC; ++cc) tmem_pin32(dv[cc]);
+      tc_fence_before();
+      warp_arrive(s_empty, lane);
+      float wsum = 0.f;
 #pragma unroll
-        for (int cc = 0; cc < HC; ++cc)
+      for (int cc = 0; cc < HC; ++cc) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (FULL || j0 + cc * 32 + i < k) mx = fmaxf(mx, __uint_as_float(sv[cc][i]));
-        // dv becomes dA + g (g_b read four at a time), sv the exponentials.
-        float z = 0.f, wsum = 0.f;
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 g4 = reinterpret_cast<const float4*>(g_s + j0 + cc * 32)[i4];
+          const float gg[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
-        for (int cc = 0; cc < HC; ++cc) {
-#pragma unroll
-          for (int i4 = 0; i4 < 8; ++i4) {
-            const float4 g4 = reinterpret_cast<const float4*>(g_s + j0 + cc * 32)[i4];
-            const float gg[4] = {g4.x, g4.y, g4.z, g4.w};
-#pragma unroll
-            for (int i1 = 0; i1 < 4; ++i1) {
-              const int i = i4 * 4 + i1;
-              const int j = j0 + cc * 32 + i;
-              const float ev = (FULL || j < k) ? ex2_approx(__uint_as_float(sv[cc][i]) - mx) : 0.f;
-              const float dg = __uint_as_float(dv[cc][i]) + gg[i1];
-              sv[cc][i] = __float_as_uint(ev);
-              dv[cc][i] = __float_as_uint(dg);
-              z += ev;
-              wsum = fmaf(ev, dg, wsum);
-            }
+          for (int i1 = 0; i1 < 4; ++i1) {
+            const int i = i4 * 4 + i1;
+            const float dg = __uint_as_float(dv[cc][i]) + gg[i1];
+            dv[cc][i] = __float_as_uint(dg);
+            wsum = fmaf(__uint_as_float(sv[cc][i]), dg, wsum);
           }
         }
-        const uint32_t par = t & 1u;
-        xch[(par * 2 + hf) * 128 + row] = make_float4(mx, z, wsum, 0.f);
-        warp_arrive(&xch_full[par], lane);
-        if (!warp_wait(&xch_full[par], (t >> 1) & 1u, abort_flag, sticky)) {
-          ok = false;
-          break;
-        }
-        const float4 o = xch[(par * 2 + (hf ^ 1)) * 128 + row];
-        // Combine: M = max of both halves; a half with no prototype has max
-        // -inf and contributes nothing.
-        const float M = fmaxf(mx, o.x);
-        const float sa_own = mx == -INFINITY ? 0.f : ex2_approx(mx - M);
-        const float sa_oth = o.x == -INFINITY ? 0.f : ex2_approx(o.x - M);
-        const float Z = z * sa_own + o.y * sa_oth;
-        const float inv = valid ? 1.0f / Z : 0.f;
-        const float scale = sa_own * inv;
-        const float cs = (wsum * sa_own + o.z * sa_oth) * inv;
-        // The shared tile is free once the previous tile's MMA3 and MMA4
-        // have read it.
-        if (t > 0 && !warp_wait(as_empty, (t - 1) & 1u, abort_flag, sticky)) {
-          ok = false;
-          break;
-        }
-        // A and dS' = ln2 A (dA + g - c) of this half, into the shared tile
-        // (A in the first KM / 64 boxes, dS' in the others).
+      }
+      const uint32_t par = t & 1u;
+      xch[(par * 2 + hf) * 128 + row] = make_float4(mx, z, wsum, 0.f);
+      warp_arrive(&xch_full[par], lane);
+      if (!warp_wait(&xch_full[par], (t >> 1) & 1u, abort_flag, sticky)) {
+        ok = false;
+        break;
+      }
+      const float4 o = xch[(par * 2 + (hf ^ 1)) * 128 + row];
+      // Combine: M = max of both halves; a half with no prototype has max
+      // -inf and contributes nothing.
+      const float M = fmaxf(mx, o.x);
+      const float sa_own = mx == -INFINITY ? 0.f : ex2_approx(mx - M);
+      const float sa_oth = o.x == -INFINITY ? 0.f : ex2_approx(o.x - M);
+      const float Z = z * sa_own + o.y * sa_oth;
+      const float inv = valid ? 1.0f / Z : 0.f;
+      const float scale = sa_own * inv;
+      const float cs = (wsum * sa_own + o.z * sa_oth) * inv;
+      // The shared tile is free once the previous tile's MMA3 and MMA4
+      // have read it.
+      if (t > 0 && !warp_wait(as_empty, (t - 1) & 1u, abort_flag, sticky)) {
+        ok = false;
+        break;
+      }
+      // A and dS' = ln2 A (dA + g - c) of this half, into the shared tile
+      // (A in the first KM / 64 boxes, dS' in the others).
 #pragma unroll
-        for (int cc = 0; cc < HC; ++cc) {
+      for (int cc = 0; cc < HC; ++cc) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint32_t wa[4], wd[4];
+        for (int u = 0; u < 4; ++u) {
+          uint32_t wa[4], wd[4];
 #pragma unroll
-            for (int ee = 0; ee < 4; ++ee) {
-              const int i = u * 8 + 2 * ee;
-              const float a0 = valid ? __uint_as_float(sv[cc][i]) * scale : 0.f;
-              const float a1 = valid ? __uint_as_float(sv[cc][i + 1]) * scale : 0.f;
-              const float d0 = kLn2 * a0 * (__uint_as_float(dv[cc][i]) - cs);
-              const float d1 = kLn2 * a1 * (__uint_as_float(dv[cc][i + 1]) - cs);
-              wa[ee] = pack_bf16x2(a0, a1);
-              wd[ee] = valid ? pack_bf16x2(d0, d1) : 0u;
-            }
-            const int col = j0 + cc * 32 + u * 8;  // prototype of the unit's first element
-            const uint32_t ua = sbase + Pl::kAS + (col >> 6) * Pl::kXBox + swz(row, (col & 63) >> 3);
-            const uint32_t ud = ua + (KM / 64) * Pl::kXBox;
-            st_shared_v4(ua, wa[0], wa[1], wa[2], wa[3]);
-            st_shared_v4(ud, wd[0], wd[1], wd[2], wd[3]);
+          for (int ee = 0; ee < 4; ++ee) {
+            const int i = u * 8 + 2 * ee;
+            const float a0 = valid ? __uint_as_float(sv[cc][i]) * scale : 0.f;
+            const float a1 = valid ? __uint_as_float(sv[cc][i + 1]) * scale : 0.f;
+            const float d0 = kLn2 * a0 * (__uint_as_float(dv[cc][i]) - cs);
+            const float d1 = kLn2 * a1 * (__uint_as_float(dv[cc][i + 1]) - cs);
+            wa[ee] = pack_bf16x2(a0, a1);
+            wd[ee] = valid ? pack_bf16x2(d0, d1) : 0u;
           }
+          const int col = j0 + cc * 32 + u * 8;  // prototype of the unit's first element
+          const uint32_t ua = sbase + Pl::kAS + (col >> 6) * Pl::kXBox + swz(row, (col & 63) >> 3);
+          const uint32_t ud = ua + (KM / 64) * Pl::kXBox;
+          st_shared_v4(ua, wa[0], wa[1], wa[2], wa[3]);
+          st_shared_v4(ud, wd[0], wd[1], wd[2], wd[3]);
         }
-        if (!valid && (D / 64 > 1 || hf == 0)) {
-          // Rows past the segment's end: cleared (0 * NaN is NaN in MMA4);
-          // each half clears one 64-column box (d = 64: the first half).
-          const int cb = D / 64 > 1 ? hf : 0;
-          const uint32_t xrow = sbase + Pl::kX + (st * (D / 64) + cb) * Pl::kXBox + row * 128;
+      }
+      if (!valid && (D / 64 > 1 || hf == 0)) {
+        // Rows past the segment's end: cleared (0 * NaN is NaN in MMA4);
+        // each half clears one 64-column box (d = 64: the first half).
+        const int cb = D / 64 > 1 ? hf : 0;
+        const uint32_t xrow = sbase + Pl::kX + (st * (D / 64) + cb) * Pl::kXBox + row * 128;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) st_shared_v4(xrow + i * 16, 0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();
-        warp_arrive(p_full, lane);
+        for (int i = 0; i < 8; ++i) st_shared_v4(xrow + i * 16, 0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
+      warp_arrive(p_full, lane);
 
-        // dX_t: TMEM row -> bf16 -> global; each half drains d / 2 columns.
-        // With 128 prototypes the warp stages its 32 rows in the part of
-        // the [A | dS'] tile that it alone writes (A's box hf, rows 32 q ..),
-        // free once MMA3 has read it, then stores whole rows: 128 (d = 64:
-        // 64) bytes of a row per 8 (4) lanes, instead of 16 bytes of 32 rows.
-        // With 64 prototypes both halves write each A and dS' box, so the
-        // rows go straight from registers.
-        if (!warp_wait(dx_full, t & 1u, abort_flag, sticky)) {
+      // The next tile (the next segment's first after a segment's last):
+      // its logits and exponentials, while MMA3 and MMA4 of this tile run.
+      int64_t nu = user, ns = s, ne = e, nlo = lo, nhi = hi, nr = r + kTileRows;
+      bool has_next = true;
+      if (last) {
+        has_next = w.next(nu, ns, ne, nlo, nhi);
+        nr = ns;
+      }
+      have_s = false;
+      if (has_next) {
+        if ((last && !warp_wait(gq_full, (seg + 1) & 1u, abort_flag, sticky)) ||
+            !warp_wait(s_full, (t + 1) & 1u, abort_flag, sticky)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        {
-          constexpr int XC = D / 64;      // 32-column chunks per half
-          constexpr int U = D / 16;       // 16-byte units per half row
-          uint32_t xv[XC][32];
+        load_exps();
+        have_s = true;
+      }
+
+      // dX_t: TMEM row -> bf16 -> global; each half drains d / 2 columns,
+      // 32 at a time.  With 128 prototypes the warp stages its 32 rows in
+      // the part of the [A | dS'] tile that it alone writes (A's box hf,
+      // rows 32 q ..), free once MMA3 has read it, then stores whole rows:
+      // 128 (d = 64: 64) bytes of a row per 8 (4) lanes, instead of 16
+      // bytes of 32 rows.  With 64 prototypes both halves write each A and
+      // dS' box, so the rows go straight from registers.
+      if (!warp_wait(dx_full, t & 1u, abort_flag, sticky)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      {
+        constexpr int XC = D / 64;  // 32-column chunks per half
+        constexpr int U = D / 16;   // 16-byte units per half row
+        const uint32_t box = sbase + Pl::kAS + hf * Pl::kXBox;
 #pragma unroll
-          for (int cc = 0; cc < XC; ++cc) tmem_ld32(lane_addr + Pl::kColDX + hf * (D / 2) + cc * 32, xv[cc]);
+        for (int cc = 0; cc < XC; ++cc) {
+          uint32_t xv[32];
+          tmem_ld32(lane_addr + Pl::kColDX + hf * (D / 2) + cc * 32, xv);
           tmem_wait_ld();
-#pragma unroll
-          for (int cc = 0; cc < XC; ++cc) tmem_pin32(xv[cc]);
-          tc_fence_before();
-          warp_arrive(dx_empty, lane);
+          tmem_pin32(xv);
+          if (cc == XC - 1) {
+            tc_fence_before();
+            warp_arrive(dx_empty, lane);
+          }
           if constexpr (KM == 64) {
             if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(ba.dX + (r + row) * D + hf * (D / 2) + cc * 32);
 #pragma unroll
-              for (int cc = 0; cc < XC; ++cc) {
-                uint4* dst = reinterpret_cast<uint4*>(ba.dX + (r + row) * D + hf * (D / 2) + cc * 32);
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                  dst[u] = make_uint4(
-                      pack_bf16x2(__uint_as_float(xv[cc][8 * u]), __uint_as_float(xv[cc][8 * u + 1])),
-                      pack_bf16x2(__uint_as_float(xv[cc][8 * u + 2]), __uint_as_float(xv[cc][8 * u + 3])),
-                      pack_bf16x2(__uint_as_float(xv[cc][8 * u + 4]), __uint_as_float(xv[cc][8 * u + 5])),
-                      pack_bf16x2(__uint_as_float(xv[cc][8 * u + 6]), __uint_as_float(xv[cc][8 * u + 7])));
-              }
+              for (int u = 0; u < 4; ++u)
+                dst[u] = make_uint4(pack_bf16x2(__uint_as_float(xv[8 * u]), __uint_as_float(xv[8 * u + 1])),
+                                    pack_bf16x2(__uint_as_float(xv[8 * u + 2]), __uint_as_float(xv[8 * u + 3])),
+                                    pack_bf16x2(__uint_as_float(xv[8 * u + 4]), __uint_as_float(xv[8 * u + 5])),
+                                    pack_bf16x2(__uint_as_float(xv[8 * u + 6]), __uint_as_float(xv[8 * u + 7])));
             }
           } else {
-          const uint32_t box = sbase + Pl::kAS + hf * Pl::kXBox;
-#pragma unroll
-          for (int cc = 0; cc < XC; ++cc)
 #pragma unroll
             for (int u = 0; u < 4; ++u)
               st_shared_v4(box + swz(row, cc * 4 + u),
-                           pack_bf16x2(__uint_as_float(xv[cc][8 * u]), __uint_as_float(xv[cc][8 * u + 1])),
-                           pack_bf16x2(__uint_as_float(xv[cc][8 * u + 2]), __uint_as_float(xv[cc][8 * u + 3])),
-                           pack_bf16x2(__uint_as_float(xv[cc][8 * u + 4]), __uint_as_float(xv[cc][8 * u + 5])),
-                           pack_bf16x2(__uint_as_float(xv[cc][8 * u + 6]), __uint_as_float(xv[cc][8 * u + 7])));
+                           pack_bf16x2(__uint_as_float(xv[8 * u]), __uint_as_float(xv[8 * u + 1])),
+                           pack_bf16x2(__uint_as_float(xv[8 * u + 2]), __uint_as_float(xv[8 * u + 3])),
+                           pack_bf16x2(__uint_as_float(xv[8 * u + 4]), __uint_as_float(xv[8 * u + 5])),
+                           pack_bf16x2(__uint_as_float(xv[8 * u + 6]), __uint_as_float(xv[8 * u + 7])));
+          }
+        }
+        if constexpr (KM == 128) {
           __syncwarp();
           constexpr int RPI = 32 / U;  // rows per warp store
 #pragma unroll
@@ -520,40 +558,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
           }
           __syncwarp();
-          }
-        }
-
-        if (last) {
-          // R_b (ln 2 dL/dQ') to the outputs or to this user's partial slot;
-          // the mass outputs carry zeros.  Each half drains d / 2 columns.
-          if (!warp_wait(&r_full[seg & 1u], (seg >> 1) & 1u, abort_flag, sticky)) { ok = false; break; }
-          tc_fence_after();
-          const int64_t slotp = segment_slot(c, lo, hi, R0, R1);
-          float* dm = slotp < 0 ? a.out_m + user * a.k : a.part_m + slotp * a.k;
-          float* dr = slotp < 0 ? a.out_x + user * a.k * D : a.part_x + slotp * a.k * D;
-          const int j = (KM == 128 ? q * 32 : q * 16) + lane;
-          const bool has = (KM == 128 || lane < 16) && j < k;
-#pragma unroll
-          for (int cc = 0; cc < D / 64; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(lane_addr + Pl::kColR + hf * (D / 2) + cc * 32, v);
-            tmem_wait_ld();
-            tmem_pin32(v);
-            if (has) {
-              float4* dst = reinterpret_cast<float4*>(dr + static_cast<int64_t>(j) * D + hf * (D / 2) +
-                                                      cc * 32);
-#pragma unroll
-              for (int w4 = 0; w4 < 8; ++w4)
-                dst[w4] = make_float4(__uint_as_float(v[4 * w4]), __uint_as_float(v[4 * w4 + 1]),
-                                      __uint_as_float(v[4 * w4 + 2]), __uint_as_float(v[4 * w4 + 3]));
-            }
-          }
-          if (has && hf == 0) dm[j] = 0.f;
-          tc_fence_before();
-          warp_arrive(r_empty, lane);
         }
       }
-      ++seg;
+
+      if (last) {
+        // R_b (ln 2 dL/dQ') to the outputs or to this user's partial slot;
+        // the mass outputs carry zeros.  Each half drains d / 2 columns.
+        if (!warp_wait(&r_full[seg & 1u], (seg >> 1) & 1u, abort_flag, sticky)) { ok = false; break; }
+        tc_fence_after();
+        const int64_t slotp = segment_slot(c, lo, hi, R0, R1);
+        float* dm = slotp < 0 ? a.out_m + user * a.k : a.part_m + slotp * a.k;
+        float* dr = slotp < 0 ? a.out_x + user * a.k * D : a.part_x + slotp * a.k * D;
+        const int j = (KM == 128 ? q * 32 : q * 16) + lane;
+        const bool has = (KM == 128 || lane < 16) && j < k;
+#pragma unroll
+        for (int cc = 0; cc < D / 64; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(lane_addr + Pl::kColR + hf * (D / 2) + cc * 32, v);
+          tmem_wait_ld();
+          tmem_pin32(v);
+          if (has) {
+            float4* dst = reinterpret_cast<float4*>(dr + static_cast<int64_t>(j) * D + hf * (D / 2) +
+                                                    cc * 32);
+#pragma unroll
+            for (int w4 = 0; w4 < 8; ++w4)
+              dst[w4] = make_float4(__uint_as_float(v[4 * w4]), __uint_as_float(v[4 * w4 + 1]),
+                                    __uint_as_float(v[4 * w4 + 2]), __uint_as_float(v[4 * w4 + 3]));
+          }
+        }
+        if (has && hf == 0) dm[j] = 0.f;
+        tc_fence_before();
+        warp_arrive(r_empty, lane);
+      }
+      if (!has_next) break;
+      if (last) ++seg;
+      user = nu;
+      s = ns;
+      e = ne;
+      lo = nlo;
+      hi = nhi;
+      r = nr;
+      ++t;
     }
   }
 
