@@ -874,6 +874,97 @@ def run_action(args, rank, world, local_rank, ranks):
     print(json.dumps(line), flush=True)
 
 
+def run_cache(args, rank, world, local_rank, ranks):
+    """The sketch cache on the workload (section 2.4): one step = one SA layer
+    served through sa_cache_forward for every user of the batch, at a fixed
+    group hit rate (the notes report about 0.6 in serving with a one-hour
+    TTL and 0.5 in training with three hours).  The hit users keep their
+    keys; the others arrive with a new history timestamp each step, so they
+    miss, are compressed from their rows and inserted.  Also timed: all
+    hits, all misses, and the width adapter (D = 1024) on the batch's
+    sketches."""
+    import torch
+
+    from sketch_attention_compression_b200 import (SketchCache, SketchQuery, WidthAdapter,
+                                                   load_library)
+    load_library()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOADS[args.workload]
+    inp = workload_inputs(args, seed=rank_seed(args.workload, rank))
+    B, N = len(inp["offsets"]) - 1, int(inp["offsets"][-1])
+    X = torch.from_numpy(inp["X"]).to(dev).to(torch.bfloat16)
+    stream = torch.cuda.current_stream(dev)
+    q = SketchQuery(*(torch.from_numpy(inp[k]).to(dev).to(torch.bfloat16) for k in ("P", "W_Q", "W_K")),
+                    inp["scale"], stream=stream)
+    offsets_host = np.ascontiguousarray(inp["offsets"], dtype=np.int64)
+    Xt = torch.empty((B, w.k, w.d), dtype=torch.float32, device=dev)
+    m = torch.empty((B, w.k), dtype=torch.float32, device=dev)
+    total_steps = 4 * (args.warmup + args.steps) + 8
+    cache = SketchCache(w.k, w.d, capacity=B * (total_steps + 2), ttl=3600.0)
+    ws = None
+    clock = [0.0]
+    ts_counter = [1000]
+
+    def make_step(hit_rate):
+        n_hit = int(round(hit_rate * B))
+        base_keys = [(rank * 100000 + b, 1, 0, 7) for b in range(B)]
+
+        def step():
+            nonlocal ws
+            clock[0] += 0.001
+            ts_counter[0] += 1
+            keys = [base_keys[b] if b < n_hit else (base_keys[b][0], 1, ts_counter[0], 7)
+                    for b in range(B)]
+            _, _, hit, ws = cache.forward(q, keys, clock[0], X, offsets_host, X_tilde=Xt, mass=m,
+                                          workspace=ws, stream=stream)
+            return hit
+        return step, n_hit
+
+    timings = {}
+    for name, rate in (("hit_0.6", 0.6), ("hit_0.5", 0.5), ("all_hits", 1.0), ("all_misses", 0.0)):
+        step, n_hit = make_step(rate)
+        for _ in range(args.warmup):
+            hit = step()
+        assert int(hit.sum()) == n_hit, (name, int(hit.sum()), n_hit)
+        timings[name] = _timed(step, args.steps, dev, stream, ranks)
+    rng = np.random.default_rng(7)
+    W_A = torch.from_numpy((rng.standard_normal((w.d, 1024)) / np.sqrt(w.d)).astype(np.float32)).to(dev)
+    ad = WidthAdapter(W_A, stream=stream)
+    Y = ad.forward(Xt.reshape(-1, w.d), stream=stream)
+
+    def adapt():
+        ad.forward(Xt.reshape(-1, w.d), out=Y, stream=stream)
+    for _ in range(args.warmup):
+        adapt()
+    ms_adapter = _timed(adapt, args.steps, dev, stream, ranks)
+    if rank != 0:
+        return
+    ms = timings["hit_0.6"]
+    peaks, _ = load_peaks()
+    rows_ad = B * w.k
+    line = {
+        "metric": "users served per second through the sketch cache at a 0.6 hit rate",
+        "value": ranks.sum(B) / (ms * 1e-3), "unit": "users/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "mode": "sketch cache", "users_per_gpu": B,
+                   "rows_per_gpu": N, "d": w.d, "k": w.k,
+                   "ms_per_step_by_hit_rate": {k: round(v, 4) for k, v in timings.items()},
+                   "adapter": {"rows": rows_ad, "D": 1024, "ms": round(ms_adapter, 4),
+                               "tflops": 2.0 * w.d * 1024 * rows_ad / (ms_adapter * 1e-3) / 1e12,
+                               "frac_of_bf16_peak": 2.0 * w.d * 1024 * rows_ad /
+                               (ms_adapter * 1e-3) / 1e12 / peaks["bf16_tflops"]}},
+        "roofline": None,
+        "note": ("a composed path (host index, host-to-device slot lists, gather, SA pass over "
+                 "the missed users' rows, scatter): its kernels' rooflines are on the SA lines; "
+                 "the adapter is a few-microsecond GEMM"),
+        "clocks": None, "cpu_baseline": None, "gpu_launches": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -893,6 +984,8 @@ def main():
                     help="time the SA backward pass (sa_sketch_backward) instead")
     ap.add_argument("--refine-layers", type=int, default=0,
                     help="time a stack of this many refinement layers instead")
+    ap.add_argument("--cache", action="store_true",
+                    help="time the layer served through the sketch cache (and the width adapter)")
     ap.add_argument("--action-fusion", action="store_true",
                     help="time the action-fusion producer followed by the SA layer instead")
     ap.add_argument("--action-hidden", type=int, default=512,
@@ -925,6 +1018,8 @@ def main():
             run_refine(args, rank, world, local_rank, ranks)
         elif args.action_fusion:
             run_action(args, rank, world, local_rank, ranks)
+        elif args.cache:
+            run_cache(args, rank, world, local_rank, ranks)
         else:
             run_ours(args, rank, world, local_rank, ranks)
     finally:

@@ -497,9 +497,9 @@ sa_status sa_cache_stats(sa_cache c, int64_t* entries, int64_t* hits, int64_t* m
 
 /*
  * sa_cache_forward -- one SA layer served through the cache: look the keys
- * up, copy the hits to the outputs, gather the missed users' history rows
- * into a compact array on the device, run sa_sketch_forward on the misses
- * only, scatter their sketches to the outputs and insert them.
+ * up and copy the hits to the outputs; each run of consecutive missed users
+ * (whose rows and outputs are contiguous) is compressed in place by one
+ * sa_sketch_forward over its range of X, and its sketches are inserted.
  *
  *   c, q           a cache and a prepared query of the same k and d
  *   keys           host, batch keys

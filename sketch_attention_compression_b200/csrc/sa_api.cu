@@ -341,6 +341,19 @@ sa_status sa_sketch_forward(sa_query q, const void* X, const int64_t* offsets, i
              stream, Phase::kBoth);
 }
 
+}  // extern "C"
+
+namespace sa {
+sa_status sketch_forward_flags(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
+                               int64_t total_rows, float* X_tilde, float* mass, void* workspace,
+                               size_t workspace_bytes, void* stream, bool keep_flags) {
+  return run(q, nullptr, X, offsets, batch, total_rows, X_tilde, mass, workspace, workspace_bytes,
+             stream, Phase::kBoth, keep_flags);
+}
+}  // namespace sa
+
+extern "C" {
+
 sa_status sa_sketch_partials(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
                              int64_t total_rows, float* X_tilde, float* mass, void* workspace,
                              size_t workspace_bytes, void* stream) {

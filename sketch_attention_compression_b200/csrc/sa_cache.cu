@@ -15,9 +15,9 @@
 // later of two equal keys wins.  Data moves only on the device: a gather of
 // hit slots into the caller's outputs, a scatter of new sketches into slots.
 // sa_cache_forward runs the whole section 2.4 flow for a batch: look up,
-// gather the hits, compact the missed users' history rows on the device, run
-// the SA layer on them only, scatter those sketches to the outputs and insert
-// them.
+// gather the hits, run the SA layer in place on each run of consecutive
+// missed users (their rows and outputs are contiguous) and insert those
+// sketches.
 //
 // Width adapter.  Section 2.3 widens the sketch for the ranking model with a
 // linear W_A in R^{d x D} (D = 1024 in the final configuration); the adapted
@@ -184,24 +184,6 @@ __global__ void cache_scatter_kernel(const float4* __restrict__ in_x, const floa
     const int64_t i = e % kd4;
     dst_x[s * kd4 + i] = in_x[e];
     if (i < k) dst_m[s * k + i] = in_m[b * k + i];
-  }
-}
-
-// Compacted history: row r of user i (coff[i] <= r < coff[i + 1]) is source
-// row src[i] + (r - coff[i]); rows are copied in 16-byte units.
-__global__ void gather_rows_kernel(const uint4* __restrict__ X, const int64_t* __restrict__ coff,
-                                   const int64_t* __restrict__ src, int64_t users, int64_t rows,
-                                   int row_units, uint4* __restrict__ out) {
-  const int64_t n = rows * row_units;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = e / row_units;
-    int64_t lo = 0, hi = users - 1;  // largest i with coff[i] <= r
-    while (lo < hi) {
-      const int64_t mid = (lo + hi + 1) >> 1;
-      if (coff[mid] <= r) lo = mid; else hi = mid - 1;
-    }
-    out[e] = X[(src[lo] + (r - coff[lo])) * row_units + e % row_units];
   }
 }
 
@@ -488,11 +470,8 @@ sa_status sa_cache_stats(sa_cache c, int64_t* entries, int64_t* hits, int64_t* m
 size_t sa_cache_forward_workspace_bytes(sa_query q, int64_t batch, int64_t total_rows) {
   int k = 0, d = 0, dt = 0, kp = 0;
   if (sa_query_info(q, &k, &d, &dt, &kp) != SA_OK || batch < 0 || total_rows < 0) return 0;
-  const size_t elem = dt == SA_BF16 ? 2 : 4;
-  const size_t B = static_cast<size_t>(batch);
   return sa::rup(sa_workspace_bytes(q, batch, total_rows)) +
-         sa::rup(static_cast<size_t>(total_rows) * d * elem) + sa::rup((B + 1) * 8) +
-         2 * sa::rup(B * 8) + sa::rup(B * k * d * 4) + sa::rup(B * k * 4);
+         sa::rup((2 * static_cast<size_t>(batch) + 1) * 8);
 }
 
 sa_status sa_cache_forward(sa_cache c, sa_query q, const sa_cache_key* keys, double now,
@@ -516,55 +495,48 @@ sa_status sa_cache_forward(sa_cache c, sa_query q, const sa_cache_key* keys, dou
   // Hits go straight to the outputs.
   sa_status s = sa_cache_lookup(c, keys, batch, now, hit, X_tilde, mass, stream);
   if (s != SA_OK) return s;
-  std::vector<int64_t> coff(1, 0), src, pos;
-  for (int64_t b = 0; b < batch; ++b) {
-    if (hit[b]) continue;
-    src.push_back(offsets_host[b]);
-    pos.push_back(b);
-    coff.push_back(coff.back() + offsets_host[b + 1] - offsets_host[b]);
+  // A run of consecutive missed users owns a contiguous range of X and of
+  // the outputs: it is compressed in place by one SA layer over that range
+  // (offsets taken relative to the run's first row), and inserted from the
+  // outputs.  No rows are copied.
+  std::vector<std::pair<int64_t, int64_t>> runs;  // [b0, b1)
+  for (int64_t b = 0; b < batch;) {
+    if (hit[b]) {
+      ++b;
+      continue;
+    }
+    int64_t e = b;
+    while (e < batch && !hit[e]) ++e;
+    runs.emplace_back(b, e);
+    b = e;
   }
-  const int64_t bm = static_cast<int64_t>(pos.size());
-  if (bm == 0) return SA_OK;
-  const int64_t nm = coff.back();
-  const size_t elem = dt == SA_BF16 ? 2 : 4;
-  const size_t B = static_cast<size_t>(batch);
+  if (runs.empty()) return SA_OK;
+  std::vector<int64_t> loc;  // the runs' relative offsets, one after another
+  std::vector<size_t> pos;
+  for (const auto& r : runs) {
+    pos.push_back(loc.size());
+    for (int64_t b = r.first; b <= r.second; ++b) loc.push_back(offsets_host[b] - offsets_host[r.first]);
+  }
   // The SA pass's workspace comes first, so that its device flags are read
   // with sa_read_device_status on the whole workspace.
   uint8_t* w = static_cast<uint8_t*>(workspace);
   void* ws_sa = w;
   const size_t ws_sa_cap = sa_workspace_bytes(q, batch, total_rows);
-  w += sa::rup(ws_sa_cap);
-  uint8_t* xc = w;
-  w += sa::rup(static_cast<size_t>(total_rows) * d * elem);
-  int64_t* d_coff = reinterpret_cast<int64_t*>(w);
-  w += sa::rup((B + 1) * 8);
-  int64_t* d_src = reinterpret_cast<int64_t*>(w);
-  w += sa::rup(B * 8);
-  int64_t* d_pos = reinterpret_cast<int64_t*>(w);
-  w += sa::rup(B * 8);
-  float* xt_m = reinterpret_cast<float*>(w);
-  w += sa::rup(B * k * d * 4);
-  float* m_m = reinterpret_cast<float*>(w);
-  if (!sa::upload(d_coff, coff, st) || !sa::upload(d_src, src, st) || !sa::upload(d_pos, pos, st))
-    return SA_ERR_CUDA;
-  // The missed users' rows, compacted, then one SA layer over them.
-  const int row_units = static_cast<int>(d * elem / 16);
-  if (nm > 0) {
-    sa::gather_rows_kernel<<<sa::grid_for_elems(nm * row_units), 256, 0, st>>>(
-        static_cast<const uint4*>(X), d_coff, d_src, bm, nm, row_units, reinterpret_cast<uint4*>(xc));
-    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  int64_t* d_loc = reinterpret_cast<int64_t*>(w + sa::rup(ws_sa_cap));
+  if (!sa::upload(d_loc, loc, st)) return SA_ERR_CUDA;
+  const size_t row_bytes = static_cast<size_t>(d) * (dt == SA_BF16 ? 2 : 4);
+  const size_t kd = static_cast<size_t>(k) * d;
+  for (size_t i = 0; i < runs.size(); ++i) {
+    const int64_t b0 = runs[i].first, b1 = runs[i].second;
+    const int64_t r0 = offsets_host[b0], nrows = offsets_host[b1] - r0;
+    s = sa::sketch_forward_flags(q, static_cast<const uint8_t*>(X) + r0 * row_bytes, d_loc + pos[i],
+                                 b1 - b0, nrows, X_tilde + b0 * kd, mass + b0 * k, ws_sa, ws_sa_cap,
+                                 stream, i > 0);
+    if (s != SA_OK) return s;
+    s = sa_cache_insert(c, keys + b0, b1 - b0, now, X_tilde + b0 * kd, mass + b0 * k, stream);
+    if (s != SA_OK) return s;
   }
-  s = sa_sketch_forward(q, xc, d_coff, bm, nm, xt_m, m_m, ws_sa, ws_sa_cap, stream);
-  if (s != SA_OK) return s;
-  const int kd4 = k * d / 4;
-  sa::cache_scatter_kernel<<<sa::grid_for_elems(bm * kd4), 256, 0, st>>>(
-      reinterpret_cast<const float4*>(xt_m), m_m, d_pos, bm, kd4, k,
-      reinterpret_cast<float4*>(X_tilde), mass);
-  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
-  std::vector<sa_cache_key> mk;
-  mk.reserve(bm);
-  for (int64_t i = 0; i < bm; ++i) mk.push_back(keys[pos[i]]);
-  return sa_cache_insert(c, mk.data(), bm, now, xt_m, m_m, stream);
+  return SA_OK;
 }
 
 sa_status sa_prepare_adapter(const float* W_A, int d, int D, void* stream, sa_adapter* out) {

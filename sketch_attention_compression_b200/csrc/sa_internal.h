@@ -210,6 +210,12 @@ bool make_tmap_bf16_box(CUtensorMap* m, const void* base, uint64_t rows, uint64_
 // prepared producer, and the producer kernel X = E + SwiGLU-FFN([E; a]) for
 // `rows` rows enqueued on `st` (flag bits OR-ed into *flags when not null).
 void action_info(const sa_action_s* act, int* d, int* device);
+
+// sa_sketch_forward with the choice of keeping the workspace header's flag
+// words (a later call of a sequence that reports every call's flags).
+sa_status sketch_forward_flags(sa_query q, const void* X, const int64_t* offsets, int64_t batch,
+                               int64_t total_rows, float* X_tilde, float* mass, void* workspace,
+                               size_t workspace_bytes, void* stream, bool keep_flags);
 sa_status action_fuse_enqueue(const sa_action_s* act, const void* E, const uint8_t* types,
                               int64_t rows, void* X, uint32_t* flags, cudaStream_t st);
 

@@ -9,8 +9,8 @@ through the C ABI.
   (the cache only moves fp32 data: bit-exact).
 * Cached forward: a first call misses every user and must match the SA
   oracle; a second call with some of the same keys returns exactly the
-  sketches the first call stored for them and computes the others, whose
-  ragged rows the library gathers on the device.
+  sketches the first call stored for them and computes the others (three
+  runs of consecutive misses, each compressed in place over its rows).
 * Adapter: Y = X~ W_A against the oracle on the bf16-rounded operands
   (ragged row tails, d = 64 and 128, D = 256 and 1024): the only rounding
   left is fp32 accumulation and the bf16 output, |err| <= 2^-8 |Y| + 1e-6
