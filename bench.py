@@ -908,14 +908,14 @@ def run_cache(args, rank, world, local_rank, ranks):
 
     def make_step(hit_rate):
         n_hit = int(round(hit_rate * B))
-        base_keys = [(rank * 100000 + b, 1, 0, 7) for b in range(B)]
+        # (user, model version, history timestamp, config) per user
+        keys = np.array([(rank * 100000 + b, 1, 0, 7) for b in range(B)], dtype=np.int64)
 
         def step():
             nonlocal ws
             clock[0] += 0.001
             ts_counter[0] += 1
-            keys = [base_keys[b] if b < n_hit else (base_keys[b][0], 1, ts_counter[0], 7)
-                    for b in range(B)]
+            keys[n_hit:, 2] = ts_counter[0]  # the misses: a new history timestamp
             _, _, hit, ws = cache.forward(q, keys, clock[0], X, offsets_host, X_tilde=Xt, mass=m,
                                           workspace=ws, stream=stream)
             return hit

@@ -87,10 +87,12 @@ class CacheKey(ctypes.Structure):
 
 
 def _keys_array(keys):
-    """A ctypes array of CacheKey from a sequence of 4-tuples."""
-    arr = (CacheKey * max(len(keys), 1))()
-    for i, key in enumerate(keys):
-        arr[i] = CacheKey(*(int(x) for x in key))
+    """The keys as a C-contiguous (n, 4) int64 array: the memory layout of n
+    sa_cache_key structs (user, model_version, history_ts, config).  Accepts
+    such an array as is, or any sequence of 4-tuples."""
+    arr = np.ascontiguousarray(keys, dtype=np.int64).reshape(-1, 4)
+    if arr.shape[0] == 0:
+        arr = np.zeros((1, 4), dtype=np.int64)
     return arr
 
 _lib: Optional[ctypes.CDLL] = None
@@ -536,14 +538,14 @@ class SketchCache:
         B = len(keys)
         hit = np.zeros(max(B, 1), dtype=np.uint8)
         _check(self._lib.sa_cache_lookup(
-            self._h, ctypes.cast(_keys_array(keys), ctypes.c_void_p), B, float(now),
+            self._h, _keys_array(keys).ctypes.data_as(ctypes.c_void_p), B, float(now),
             hit.ctypes.data_as(ctypes.c_void_p), _dev_ptr(X_tilde, "X_tilde"), _dev_ptr(mass, "mass"),
             ctypes.c_void_p(_stream_handle(stream))), "sa_cache_lookup")
         return hit[:B].astype(bool)
 
     def insert(self, keys, now: float, X_tilde, mass, stream=None) -> None:
         _check(self._lib.sa_cache_insert(
-            self._h, ctypes.cast(_keys_array(keys), ctypes.c_void_p), len(keys), float(now),
+            self._h, _keys_array(keys).ctypes.data_as(ctypes.c_void_p), len(keys), float(now),
             _dev_ptr(X_tilde, "X_tilde"), _dev_ptr(mass, "mass"),
             ctypes.c_void_p(_stream_handle(stream))), "sa_cache_insert")
 
@@ -571,7 +573,7 @@ class SketchCache:
                                     dtype=torch.uint8, device=X.device)
         hit = np.zeros(max(B, 1), dtype=np.uint8)
         _check(self._lib.sa_cache_forward(
-            self._h, query._h, ctypes.cast(_keys_array(keys), ctypes.c_void_p), float(now),
+            self._h, query._h, _keys_array(keys).ctypes.data_as(ctypes.c_void_p), float(now),
             ctypes.c_void_p(X.data_ptr() if N > 0 else 0),
             offsets_host.ctypes.data_as(ctypes.c_void_p), B, N, _dev_ptr(X_tilde, "X_tilde"),
             _dev_ptr(mass, "mass"), hit.ctypes.data_as(ctypes.c_void_p),

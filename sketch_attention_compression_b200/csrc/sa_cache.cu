@@ -53,6 +53,19 @@ struct KeyLess {
 
 }  // namespace
 
+// Pinned host staging for the slot and offset lists a call copies to the
+// device.  Calls alternate between two halves; a call waits (on its half's
+// event) only for the copies of the call two before it, so the host runs
+// ahead of the device instead of waiting for each copy as a copy from
+// pageable memory would.
+struct SaStaging {
+  int64_t* host = nullptr;
+  size_t cap = 0;
+  size_t used = 0;
+  cudaEvent_t ev = nullptr;
+  bool recorded = false;
+};
+
 struct sa_cache_s {
   int device;
   int k;
@@ -63,6 +76,8 @@ struct sa_cache_s {
   float* pool_m;   // [capacity][k]
   int64_t* d_slots = nullptr;  // per-call slot list on the device
   int64_t d_slots_cap = 0;
+  SaStaging stg[2];
+  uint64_t calls = 0;
   std::map<sa_cache_key, int64_t, KeyLess> index;
   std::vector<sa_cache_key> slot_key;
   std::vector<bool> used;
@@ -205,12 +220,74 @@ bool ensure_slots(sa_cache_s* c, int64_t n, cudaStream_t st) {
   return true;
 }
 
-// Copies a host vector of slots to the device list (pageable source: the
-// call returns once the data is staged, so the vector may be reused).
-bool upload(int64_t* dst, const std::vector<int64_t>& v, cudaStream_t st) {
+// The staging half of a call that copies at most n values: its copies of
+// two calls ago are waited for, then it is reset (and grown if needed).
+SaStaging* begin_call(sa_cache_s* c, size_t n) {
+  SaStaging* s = &c->stg[c->calls & 1];
+  if (s->recorded && cudaEventSynchronize(s->ev) != cudaSuccess) return nullptr;
+  s->recorded = false;
+  if (s->ev == nullptr && cudaEventCreateWithFlags(&s->ev, cudaEventDisableTiming) != cudaSuccess)
+    return nullptr;
+  if (n > s->cap) {
+    cudaFreeHost(s->host);
+    s->host = nullptr;
+    s->cap = 0;
+    const size_t cap = std::max<size_t>(n, 1024);
+    if (cudaMallocHost(&s->host, cap * sizeof(int64_t)) != cudaSuccess) return nullptr;
+    s->cap = cap;
+  }
+  s->used = 0;
+  return s;
+}
+
+// Marks the end of a call's copies on the stream.
+bool end_call(sa_cache_s* c, SaStaging* s, cudaStream_t st) {
+  ++c->calls;
+  s->recorded = cudaEventRecord(s->ev, st) == cudaSuccess;
+  return s->recorded;
+}
+
+// Copies a host vector to the device through the call's pinned staging.
+bool upload(SaStaging* s, int64_t* dst, const std::vector<int64_t>& v, cudaStream_t st) {
   if (v.empty()) return true;
-  return cudaMemcpyAsync(dst, v.data(), v.size() * sizeof(int64_t), cudaMemcpyHostToDevice, st) ==
+  if (s->used + v.size() > s->cap) return false;
+  int64_t* h = s->host + s->used;
+  std::copy(v.begin(), v.end(), h);
+  s->used += v.size();
+  return cudaMemcpyAsync(dst, h, v.size() * sizeof(int64_t), cudaMemcpyHostToDevice, st) ==
          cudaSuccess;
+}
+
+sa_status lookup_impl(sa_cache_s* c, SaStaging* sg, const sa_cache_key* keys, int64_t batch,
+                      double now, uint8_t* hit, float* X_tilde, float* mass, cudaStream_t st) {
+  std::vector<int64_t> slots(batch);
+  for (int64_t b = 0; b < batch; ++b) {
+    slots[b] = lookup_one(c, keys[b], now);
+    hit[b] = slots[b] >= 0 ? 1 : 0;
+  }
+  if (!ensure_slots(c, batch, st) || !upload(sg, c->d_slots, slots, st)) return SA_ERR_CUDA;
+  const int kd4 = c->k * c->d / 4;
+  cache_gather_kernel<<<grid_for_elems(batch * kd4), 256, 0, st>>>(
+      reinterpret_cast<const float4*>(c->pool_x), c->pool_m, c->d_slots, batch, kd4, c->k,
+      reinterpret_cast<float4*>(X_tilde), mass);
+  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+sa_status insert_impl(sa_cache_s* c, SaStaging* sg, const sa_cache_key* keys, int64_t batch,
+                      double now, const float* X_tilde, const float* mass, cudaStream_t st) {
+  std::vector<int64_t> slots(batch);
+  for (int64_t b = 0; b < batch; ++b) slots[b] = insert_one(c, keys[b], now);
+  // Two equal keys in one batch share a slot: only the later one is copied.
+  std::map<int64_t, int64_t> last;
+  for (int64_t b = 0; b < batch; ++b) last[slots[b]] = b;
+  for (int64_t b = 0; b < batch; ++b)
+    if (last[slots[b]] != b) slots[b] = -1;
+  if (!ensure_slots(c, batch, st) || !upload(sg, c->d_slots, slots, st)) return SA_ERR_CUDA;
+  const int kd4 = c->k * c->d / 4;
+  cache_scatter_kernel<<<grid_for_elems(batch * kd4), 256, 0, st>>>(
+      reinterpret_cast<const float4*>(X_tilde), mass, c->d_slots, batch, kd4, c->k,
+      reinterpret_cast<float4*>(c->pool_x), c->pool_m);
+  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ width adapter
@@ -366,6 +443,57 @@ bool al(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) =
 
 size_t rup(size_t x) { return (x + 255) / 256 * 256; }
 
+sa_status forward_impl(sa_cache_s* c, SaStaging* sg, sa_query q, const sa_cache_key* keys,
+                       double now, const void* X, const int64_t* offsets_host, int64_t batch,
+                       int64_t total_rows, int k, int d, int dt, float* X_tilde, float* mass,
+                       uint8_t* hit, void* workspace, cudaStream_t st) {
+  // Hits go straight to the outputs.
+  sa_status s = lookup_impl(c, sg, keys, batch, now, hit, X_tilde, mass, st);
+  if (s != SA_OK) return s;
+  // A run of consecutive missed users owns a contiguous range of X and of
+  // the outputs: it is compressed in place by one SA layer over that range
+  // (offsets taken relative to the run's first row), and inserted from the
+  // outputs.  No rows are copied.
+  std::vector<std::pair<int64_t, int64_t>> runs;  // [b0, b1)
+  for (int64_t b = 0; b < batch;) {
+    if (hit[b]) {
+      ++b;
+      continue;
+    }
+    int64_t e = b;
+    while (e < batch && !hit[e]) ++e;
+    runs.emplace_back(b, e);
+    b = e;
+  }
+  if (runs.empty()) return SA_OK;
+  std::vector<int64_t> loc;  // the runs' relative offsets, one after another
+  std::vector<size_t> pos;
+  for (const auto& r : runs) {
+    pos.push_back(loc.size());
+    for (int64_t b = r.first; b <= r.second; ++b) loc.push_back(offsets_host[b] - offsets_host[r.first]);
+  }
+  // The SA pass's workspace comes first, so that its device flags are read
+  // with sa_read_device_status on the whole workspace.
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  void* ws_sa = w;
+  const size_t ws_sa_cap = sa_workspace_bytes(q, batch, total_rows);
+  int64_t* d_loc = reinterpret_cast<int64_t*>(w + rup(ws_sa_cap));
+  if (!upload(sg, d_loc, loc, st)) return SA_ERR_CUDA;
+  const size_t row_bytes = static_cast<size_t>(d) * (dt == SA_BF16 ? 2 : 4);
+  const size_t kd = static_cast<size_t>(k) * d;
+  for (size_t i = 0; i < runs.size(); ++i) {
+    const int64_t b0 = runs[i].first, b1 = runs[i].second;
+    const int64_t r0 = offsets_host[b0], nrows = offsets_host[b1] - r0;
+    s = sketch_forward_flags(q, static_cast<const uint8_t*>(X) + r0 * row_bytes, d_loc + pos[i],
+                             b1 - b0, nrows, X_tilde + b0 * kd, mass + b0 * k, ws_sa, ws_sa_cap, st,
+                             i > 0);
+    if (s != SA_OK) return s;
+    s = insert_impl(c, sg, keys + b0, b1 - b0, now, X_tilde + b0 * kd, mass + b0 * k, st);
+    if (s != SA_OK) return s;
+  }
+  return SA_OK;
+}
+
 }  // namespace
 }  // namespace sa
 
@@ -404,9 +532,14 @@ sa_status sa_cache_create(int k, int d, int64_t capacity, double ttl_seconds, sa
 
 void sa_cache_free(sa_cache c) {
   if (c == nullptr) return;
+  cudaDeviceSynchronize();
   cudaFree(c->pool_x);
   cudaFree(c->pool_m);
   cudaFree(c->d_slots);
+  for (auto& s : c->stg) {
+    cudaFreeHost(s.host);
+    if (s.ev != nullptr) cudaEventDestroy(s.ev);
+  }
   delete c;
 }
 
@@ -419,17 +552,10 @@ sa_status sa_cache_lookup(sa_cache c, const sa_cache_key* keys, int64_t batch, d
     return SA_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(c->mu);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  std::vector<int64_t> slots(batch);
-  for (int64_t b = 0; b < batch; ++b) {
-    slots[b] = sa::lookup_one(c, keys[b], now);
-    hit[b] = slots[b] >= 0 ? 1 : 0;
-  }
-  if (!sa::ensure_slots(c, batch, st) || !sa::upload(c->d_slots, slots, st)) return SA_ERR_CUDA;
-  const int kd4 = c->k * c->d / 4;
-  sa::cache_gather_kernel<<<sa::grid_for_elems(batch * kd4), 256, 0, st>>>(
-      reinterpret_cast<const float4*>(c->pool_x), c->pool_m, c->d_slots, batch, kd4, c->k,
-      reinterpret_cast<float4*>(X_tilde), mass);
-  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+  SaStaging* sg = sa::begin_call(c, static_cast<size_t>(batch));
+  if (sg == nullptr) return SA_ERR_CUDA;
+  const sa_status s = sa::lookup_impl(c, sg, keys, batch, now, hit, X_tilde, mass, st);
+  return sa::end_call(c, sg, st) ? s : SA_ERR_CUDA;
 }
 
 sa_status sa_cache_insert(sa_cache c, const sa_cache_key* keys, int64_t batch, double now,
@@ -441,19 +567,10 @@ sa_status sa_cache_insert(sa_cache c, const sa_cache_key* keys, int64_t batch, d
     return SA_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(c->mu);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  std::vector<int64_t> slots(batch);
-  for (int64_t b = 0; b < batch; ++b) slots[b] = sa::insert_one(c, keys[b], now);
-  // Two equal keys in one batch share a slot: only the later one is copied.
-  std::map<int64_t, int64_t> last;
-  for (int64_t b = 0; b < batch; ++b) last[slots[b]] = b;
-  for (int64_t b = 0; b < batch; ++b)
-    if (last[slots[b]] != b) slots[b] = -1;
-  if (!sa::ensure_slots(c, batch, st) || !sa::upload(c->d_slots, slots, st)) return SA_ERR_CUDA;
-  const int kd4 = c->k * c->d / 4;
-  sa::cache_scatter_kernel<<<sa::grid_for_elems(batch * kd4), 256, 0, st>>>(
-      reinterpret_cast<const float4*>(X_tilde), mass, c->d_slots, batch, kd4, c->k,
-      reinterpret_cast<float4*>(c->pool_x), c->pool_m);
-  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+  SaStaging* sg = sa::begin_call(c, static_cast<size_t>(batch));
+  if (sg == nullptr) return SA_ERR_CUDA;
+  const sa_status s = sa::insert_impl(c, sg, keys, batch, now, X_tilde, mass, st);
+  return sa::end_call(c, sg, st) ? s : SA_ERR_CUDA;
 }
 
 sa_status sa_cache_stats(sa_cache c, int64_t* entries, int64_t* hits, int64_t* misses,
@@ -492,52 +609,16 @@ sa_status sa_cache_forward(sa_cache c, sa_query q, const sa_cache_key* keys, dou
   if (workspace_bytes < sa_cache_forward_workspace_bytes(q, batch, total_rows))
     return SA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // Hits go straight to the outputs.
-  sa_status s = sa_cache_lookup(c, keys, batch, now, hit, X_tilde, mass, stream);
-  if (s != SA_OK) return s;
-  // A run of consecutive missed users owns a contiguous range of X and of
-  // the outputs: it is compressed in place by one SA layer over that range
-  // (offsets taken relative to the run's first row), and inserted from the
-  // outputs.  No rows are copied.
-  std::vector<std::pair<int64_t, int64_t>> runs;  // [b0, b1)
-  for (int64_t b = 0; b < batch;) {
-    if (hit[b]) {
-      ++b;
-      continue;
-    }
-    int64_t e = b;
-    while (e < batch && !hit[e]) ++e;
-    runs.emplace_back(b, e);
-    b = e;
-  }
-  if (runs.empty()) return SA_OK;
-  std::vector<int64_t> loc;  // the runs' relative offsets, one after another
-  std::vector<size_t> pos;
-  for (const auto& r : runs) {
-    pos.push_back(loc.size());
-    for (int64_t b = r.first; b <= r.second; ++b) loc.push_back(offsets_host[b] - offsets_host[r.first]);
-  }
-  // The SA pass's workspace comes first, so that its device flags are read
-  // with sa_read_device_status on the whole workspace.
-  uint8_t* w = static_cast<uint8_t*>(workspace);
-  void* ws_sa = w;
-  const size_t ws_sa_cap = sa_workspace_bytes(q, batch, total_rows);
-  int64_t* d_loc = reinterpret_cast<int64_t*>(w + sa::rup(ws_sa_cap));
-  if (!sa::upload(d_loc, loc, st)) return SA_ERR_CUDA;
-  const size_t row_bytes = static_cast<size_t>(d) * (dt == SA_BF16 ? 2 : 4);
-  const size_t kd = static_cast<size_t>(k) * d;
-  for (size_t i = 0; i < runs.size(); ++i) {
-    const int64_t b0 = runs[i].first, b1 = runs[i].second;
-    const int64_t r0 = offsets_host[b0], nrows = offsets_host[b1] - r0;
-    s = sa::sketch_forward_flags(q, static_cast<const uint8_t*>(X) + r0 * row_bytes, d_loc + pos[i],
-                                 b1 - b0, nrows, X_tilde + b0 * kd, mass + b0 * k, ws_sa, ws_sa_cap,
-                                 stream, i > 0);
-    if (s != SA_OK) return s;
-    s = sa_cache_insert(c, keys + b0, b1 - b0, now, X_tilde + b0 * kd, mass + b0 * k, stream);
-    if (s != SA_OK) return s;
-  }
-  return SA_OK;
+  std::lock_guard<std::mutex> lock(c->mu);
+  // Lookup slots, the runs' offsets (at most 2 batch + 1) and insert slots.
+  SaStaging* sg = sa::begin_call(c, 4 * static_cast<size_t>(batch) + 1);
+  if (sg == nullptr) return SA_ERR_CUDA;
+  const sa_status s = sa::forward_impl(c, sg, q, keys, now, X, offsets_host, batch, total_rows, k, d, dt,
+                                   X_tilde, mass, hit, workspace, st);
+  return sa::end_call(c, sg, st) ? s : SA_ERR_CUDA;
 }
+
+
 
 sa_status sa_prepare_adapter(const float* W_A, int d, int D, void* stream, sa_adapter* out) {
   if (out == nullptr) return SA_ERR_INVALID_ARG;
