@@ -77,6 +77,23 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar, int lane) {
   if (lane == 0) mbar_arrive(bar);
 }
 
+// TMA store of a 2-D box from shared memory (bulk async-group completion),
+// and the waits on this thread's outstanding stores.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t x,
+                                             int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// The stores no longer read shared memory (the source may be overwritten).
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// The stores have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Byte offset of 16-byte unit u of row r in a 128-byte-swizzled box.
 __device__ __forceinline__ uint32_t swz(int r, int u) {
   return (r >> 3) * 1024 + (r & 7) * 128 + ((u ^ (r & 7)) << 4);
@@ -92,7 +109,8 @@ template <int D, int KM, bool FULL>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     sa_backward_kernel(const __grid_constant__ CUtensorMap tm_x,
                        const __grid_constant__ CUtensorMap tm_q,
-                       const __grid_constant__ CUtensorMap tm_g, const BwdArgs ba) {
+                       const __grid_constant__ CUtensorMap tm_g,
+                       const __grid_constant__ CUtensorMap tm_dx, const BwdArgs ba) {
   using Pl = BwdPlan<D, KM>;
   constexpr int S = kBwdStages;
   const PassArgs& a = ba.p;
@@ -339,6 +357,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // once per tile through shared memory, behind a bounded mbarrier wait.
     const int q = warp & 3;
     const int hf = (warp - 4) >> 2;
+    // d = k = 128: whole tiles of dX leave by TMA store from the staging rows.
+    constexpr bool kTmaDx = KM == 128 && D == 128;
     const int row = q * 32 + lane;
     constexpr int HW = KM / 2, HC = HW / 32;
     const int j0 = hf * HW;
@@ -444,6 +464,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = false;
         break;
       }
+      // This warp's dX store of the previous tile may still read its staging
+      // rows (in the box about to be written).
+      if (kTmaDx) {
+        if (lane == 0) bulk_wait_read();
+        __syncwarp();
+      }
       // A and dS' = ln2 A (dA + g - c) of this half, into the shared tile
       // (A in the first KM / 64 boxes, dS' in the others).
 #pragma unroll
@@ -545,7 +571,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                            pack_bf16x2(__uint_as_float(xv[8 * u + 6]), __uint_as_float(xv[8 * u + 7])));
           }
         }
-        if constexpr (KM == 128) {
+        if (kTmaDx && nrows == kTileRows) {
+          // A whole tile: one TMA store of the warp's 32 staged rows.
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_dx, box + q * 4096, hf * (D / 2), static_cast<int32_t>(r + q * 32));
+            bulk_commit();
+          }
+        } else if constexpr (KM == 128) {
           __syncwarp();
           constexpr int RPI = 32 / U;  // rows per warp store
 #pragma unroll
@@ -600,6 +634,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       r = nr;
       ++t;
     }
+    // This warp's last dX stores complete before the CTA exits.
+    if (kTmaDx && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -761,7 +797,15 @@ cudaError_t launch_bwd_one(const CUtensorMap& tx, const CUtensorMap& tq, const C
   auto kern = ba.p.k == KM ? sa_backward_kernel<D, KM, true> : sa_backward_kernel<D, KM, false>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Pl::kSmem);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kBwdThreads, Pl::kSmem, st>>>(tx, tq, tg, ba);
+  // dX as 32-row x 64-column boxes (one warp's rows of one half), 128-byte
+  // swizzle: the layout the drain stages them in.
+  CUtensorMap tdx;
+  if (ba.p.total_rows > 0 &&
+      !make_tmap_bf16_box(&tdx, ba.dX, static_cast<uint64_t>(ba.p.total_rows), static_cast<uint64_t>(D),
+                          64, 32, 128))
+    return cudaErrorInvalidValue;
+  if (ba.p.total_rows == 0) tdx = tx;  // unused: no tile is drained
+  kern<<<grid, kBwdThreads, Pl::kSmem, st>>>(tx, tq, tg, tdx, ba);
   return cudaGetLastError();
 }
 }  // namespace
