@@ -450,7 +450,8 @@ sa_status sa_refine_stack_forward(int layers, const sa_query* qs, const sa_refin
  * The index is host memory guarded by a mutex; the sketches move only on
  * the device.  Calls on one cache that move data (lookup, insert, forward)
  * must be ordered with one another by the caller: the library reuses one
- * device slot list, so use one stream per cache.
+ * device slot list, so use one stream per cache.  Every call must be made
+ * with the cache's device current (SA_ERR_INVALID_ARG otherwise).
  */
 typedef struct sa_cache_key {
   int64_t user;

@@ -441,6 +441,12 @@ cudaError_t launch_adapter(const sa_adapter_s* ad, const float* X, int64_t rows,
 
 bool al(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// The caller's current device is the one the object's memory lives on.
+bool on_device(int device) {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess && dev == device;
+}
+
 size_t rup(size_t x) { return (x + 255) / 256 * 256; }
 
 sa_status forward_impl(sa_cache_s* c, SaStaging* sg, sa_query q, const sa_cache_key* keys,
@@ -548,7 +554,7 @@ sa_status sa_cache_lookup(sa_cache c, const sa_cache_key* keys, int64_t batch, d
   if (c == nullptr || batch < 0) return SA_ERR_INVALID_ARG;
   if (batch == 0) return SA_OK;
   if (keys == nullptr || hit == nullptr || X_tilde == nullptr || mass == nullptr ||
-      !sa::al(X_tilde, 16) || !sa::al(mass, 4))
+      !sa::al(X_tilde, 16) || !sa::al(mass, 4) || !sa::on_device(c->device))
     return SA_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(c->mu);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -563,7 +569,7 @@ sa_status sa_cache_insert(sa_cache c, const sa_cache_key* keys, int64_t batch, d
   if (c == nullptr || batch < 0) return SA_ERR_INVALID_ARG;
   if (batch == 0) return SA_OK;
   if (keys == nullptr || X_tilde == nullptr || mass == nullptr || !sa::al(X_tilde, 16) ||
-      !sa::al(mass, 4))
+      !sa::al(mass, 4) || !sa::on_device(c->device))
     return SA_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(c->mu);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -601,7 +607,7 @@ sa_status sa_cache_forward(sa_cache c, sa_query q, const sa_cache_key* keys, dou
   if (batch == 0) return total_rows == 0 ? SA_OK : SA_ERR_INVALID_ARG;
   if (keys == nullptr || offsets_host == nullptr || X_tilde == nullptr || mass == nullptr ||
       hit == nullptr || workspace == nullptr || (total_rows > 0 && X == nullptr) ||
-      !sa::al(workspace, 256) || !sa::al(X, 16))
+      !sa::al(workspace, 256) || !sa::al(X, 16) || !sa::on_device(c->device))
     return SA_ERR_INVALID_ARG;
   if (offsets_host[0] != 0 || offsets_host[batch] != total_rows) return SA_ERR_INVALID_ARG;
   for (int64_t b = 0; b < batch; ++b)
@@ -667,8 +673,7 @@ sa_status sa_adapter_forward(sa_adapter a, const float* X_tilde, int64_t rows, v
       !sa::al(device_flags, 4))
     return SA_ERR_INVALID_ARG;
   if (rows > (int64_t{1} << 31) * 128 - 128) return SA_ERR_INVALID_ARG;
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev != a->device) return SA_ERR_INVALID_ARG;
+  if (!sa::on_device(a->device)) return SA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const cudaError_t err =
       a->d == 64 ? sa::launch_adapter<64>(a, X_tilde, rows, static_cast<uint16_t*>(out), device_flags, st)
