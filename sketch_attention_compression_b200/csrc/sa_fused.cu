@@ -54,9 +54,10 @@
 // the others).  The softmax over all k prototypes of a row combines the
 // slices: each CTA computes its slice's maximum m_h and sum
 // z_h = sum_j exp2(s_j - m_h), i.e. the slice's total in log2 form
-// L_h = m_h + log2 z_h, and sends L_h of every row to the other CTAs with
-// st.async (the value and its arrival on the receiver's barrier in one
-// hop).  Each CTA then takes M = max_h L_h and Z = sum_h exp2(L_h - M) over
+// L_h = m_h + log2 z_h, and sends L_h of every row to the other CTAs: each
+// softmax warp's 32 values go to each other CTA as one 128-byte bulk copy
+// that lands in the receiver's slots and counts as arrived bytes on its
+// barrier.  Each CTA then takes M = max_h L_h and Z = sum_h exp2(L_h - M) over
 // all C values (in rank order, so every CTA gets the same M and Z bit for
 // bit) and scales its exponentials by exp2(m_h - M) / Z.  The values land
 // in slots that take the place of the drain staging (cluster CTAs drain
@@ -64,7 +65,10 @@
 // tile: a CTA sends tile u + 2 of a softmax group only after it has
 // received every CTA's tile u + 1, which each CTA sends only after it has
 // read its tile u slots, so no slot or barrier phase is overwritten early
-// and no acknowledgement has to travel back.
+// and no acknowledgement has to travel back.  The same order covers the
+// copies' sources: a CTA rewrites its own tile u slot (tile u + 2) only
+// after every CTA's tile u + 1 arrived, and each sent that only after this
+// CTA's tile u copy to it had landed.
 //
 // Per-user queries (the SA step of a refinement layer, section 2.2 "Stacked
 // Refinement" of the notes): the one Q' buffer is reloaded per segment.
@@ -152,9 +156,9 @@ constexpr int kMaxCluster = 8;
 
 // FULL: no prototype column needs masking (k == KM, or k == KM * C for a
 // cluster).  CLU: prototype-split cluster of C CTAs (KM == 128 each); 0 none,
-// 1 for C <= 4 (row-major exchange slots), 2 for C > 4 (source-major).  The
-// slot layout is a template choice: a runtime branch between the two cost
-// the C = 2 pass 13 % in code generation.
+// 1 for C <= 4, 2 for C > 4 (how many exchange sources the softmax reads;
+// a template choice, because reading all eight slots behind a runtime
+// bound cost the small clusters in code generation).
 template <int D, int KM, bool FULL, int CLU>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_sa_kernel(const __grid_constant__ CUtensorMap tm_x,
@@ -530,50 +534,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         float inv;
         if constexpr (kClu) {
           // Send L_h of this row to every other CTA and wait for theirs.
-          // Each [group][parity] region holds 128 rows x 8 sources; up to
-          // 4 CTAs it is row-major (16 bytes per row: one 16-byte load
-          // gets a row's values), beyond that source-major (a warp's 32
-          // sends to one CTA then cover 128 contiguous bytes, where 32
-          // scattered sectors per send would cost more than the loads).
+          // Each [group][parity] region holds 8 sources x 128 rows,
+          // source-major: a warp's 32 values are 128 contiguous bytes,
+          // which lane p sends to CTA p with one bulk copy (a message per
+          // row and CTA cost more than the rest of the exchange).  The
+          // slot is rewritten two tiles of the group later, after every
+          // CTA's next tile has arrived here, which each CTA sends only
+          // once this tile's copies to it have landed.
           const uint32_t u = t >> 1, par = u & 1u;
           uint64_t* sfull = &stats_full[grp * 2 + par];
           if (q == 0 && lane == 0) mbar_arrive_expect_tx(sfull, (ncl - 1) * 128 * 4);
           if (q == 0) xch_armed = u + 1;
           const float Lh = mx + lg2_approx(zl);
           const uint32_t sfull_a = smem_u32(sfull);
-          constexpr bool kWide = CLU == 2;
+          constexpr int kSrc = CLU == 2 ? kMaxCluster : 4;  // sources the reads cover
           const uint32_t region = xch_a + (grp * 2 + par) * 4096;
-          const uint32_t mine = kWide ? region + h * 512 + row * 4 : region + row * 16 + h * 4;
-          for (uint32_t p = 0; p < ncl; ++p)
-            if (p != h) st_async_f32(map_to_cta(mine, p), Lh, map_to_cta(sfull_a, p));
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(region + h * 512 + row * 4), "f"(Lh)
+                       : "memory");
+          fence_proxy_async_smem();
+          __syncwarp();
+          const uint32_t wslot = region + h * 512 + q * 128;
+          if (static_cast<uint32_t>(lane) < ncl && static_cast<uint32_t>(lane) != h)
+            bulk_copy_to_cta(map_to_cta(wslot, lane), wslot, 128, map_to_cta(sfull_a, lane));
           xch_sent = u + 1;
-          asm volatile("st.shared.f32 [%0], %1;" ::"r"(mine), "f"(Lh) : "memory");
           if (!warp_wait_cluster(sfull, (u >> 1) & 1u, abort_flag, sticky)) {
             ok = false;
             break;
           }
           xch_waited = u + 1;
-          float Lv[kMaxCluster];
-          if constexpr (kWide) {
+          float Lv[kSrc];
 #pragma unroll
-            for (int p = 0; p < kMaxCluster; ++p)
-              Lv[p] = p < static_cast<int>(ncl) ? ld_shared_f32(region + p * 512 + row * 4)
-                                                : -INFINITY;
-          } else {
-            const float4 v = ld_shared_v4f(region + row * 16);
-            Lv[0] = v.x; Lv[1] = v.y; Lv[2] = v.z; Lv[3] = v.w;
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-              if (p >= static_cast<int>(ncl)) Lv[p] = -INFINITY;
-#pragma unroll
-            for (int p = 4; p < kMaxCluster; ++p) Lv[p] = -INFINITY;
-          }
+          for (int p = 0; p < kSrc; ++p)
+            Lv[p] = p < static_cast<int>(ncl) ? ld_shared_f32(region + p * 512 + row * 4)
+                                              : -INFINITY;
           float Mx = Lv[0];
 #pragma unroll
-          for (int p = 1; p < kMaxCluster; ++p) Mx = fmaxf(Mx, Lv[p]);
+          for (int p = 1; p < kSrc; ++p) Mx = fmaxf(Mx, Lv[p]);
           float Z = 0.f;
 #pragma unroll
-          for (int p = 0; p < kMaxCluster; ++p)
+          for (int p = 0; p < kSrc; ++p)
             if (p < static_cast<int>(ncl)) Z += ex2_approx(Lv[p] - Mx);
           inv = valid ? ex2_approx(mx - Mx) / Z : 0.f;
         } else {
@@ -745,10 +744,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, 512);
   }
   if constexpr (kClu) {
-    // Row totals travel between the CTAs with st.async, which the cluster
-    // barrier does not order.  On the normal path every value a CTA was
-    // sent has been waited for.  If any CTA of the cluster gave up, a value
-    // may still be in flight to a CTA that stopped waiting, so before the
+    // Row totals travel between the CTAs as bulk copies, which the cluster
+    // barrier does not order (and which read the sender's shared memory
+    // until they land).  On the normal path every value a CTA was sent has
+    // been waited for.  If any CTA of the cluster gave up, a copy may still
+    // be in flight to a CTA that stopped waiting, so before the
     // final barrier each CTA waits until everything sent to it has landed:
     //   1. every CTA publishes its abort flag and, per softmax warp, its
     //      exchange counts (in the offset cache, unused from here on), then

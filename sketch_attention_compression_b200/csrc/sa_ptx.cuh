@@ -410,12 +410,19 @@ __device__ __forceinline__ void st_async_v2f(uint32_t remote, float a, float b,
       : "memory");
 }
 
-// One float into another CTA's shared memory, signalled as 4 transaction
-// bytes on that CTA's mbarrier (both addresses from map_to_cta).
-__device__ __forceinline__ void st_async_f32(uint32_t remote, float a, uint32_t remote_bar) {
+// Copies `bytes` (a multiple of 16; both addresses 16-byte aligned) of this
+// CTA's shared memory at `local` into another CTA's shared memory at
+// `remote`, signalled as that many transaction bytes on the receiver's
+// mbarrier (remote addresses from map_to_cta).  The copy engine reads the
+// source asynchronously: the source may be rewritten only once the
+// receiver's barrier phase is known to have completed.  Stores made to the
+// source by the generic proxy must be fenced (fence_proxy_async_smem) first.
+__device__ __forceinline__ void bulk_copy_to_cta(uint32_t remote, uint32_t local, uint32_t bytes,
+                                                 uint32_t remote_bar) {
   asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(remote),
-      "f"(a), "r"(remote_bar)
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+      "[%3];" ::"r"(remote),
+      "r"(local), "r"(bytes), "r"(remote_bar)
       : "memory");
 }
 
