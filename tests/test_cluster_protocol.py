@@ -2,20 +2,25 @@
 
 The prototype-split cluster pass (more than 128 prototypes; section 2.2 of
 the SequenceO1 reading notes puts the final layers at about a thousand)
-combines each row's softmax over C CTAs.  Every CTA sends its slice total of
-tile u to every other CTA with st.async: the value lands in the receiver's
-slot [group][u & 1][sender] and adds its bytes to the receiver's barrier
-[group][u & 1]; the receiver arms that barrier once per tile (one arrival
-plus the expected bytes), waits for the phase to complete, then reads the
-slots.  No acknowledgement travels back: the argument is that a CTA can only
-send tile u + 2 of a group after it received every CTA's tile u + 1, which
-each CTA sends only after reading its own tile u slots.
+combines each row's softmax over C CTAs.  Every softmax warp writes its
+rows' slice totals of tile u into its own slot [group][u & 1][self] and
+sends that run to every other CTA as one bulk copy: the copy engine reads
+the sender's slot when it delivers (not when the copy is issued), the data
+lands in the receiver's slot [group][u & 1][sender] and adds its bytes to
+the receiver's barrier [group][u & 1]; the receiver arms that barrier once
+per tile (one arrival plus the expected bytes), waits for the phase to
+complete, then reads the slots.  No acknowledgement travels back: the
+argument is that a CTA can only send tile u + 2 of a group after it
+received every CTA's tile u + 1, which each CTA sends only after reading its
+own tile u slots, and after its tile u copy from this CTA had landed.
 
 This test runs that protocol on a model of the mbarrier (pending arrivals,
 transaction bytes that may arrive before or after the arming, phase parity)
 with arbitrary interleavings and arbitrary delivery delays, and checks that
   * every read sees the values of its own tile from every sender;
   * no value lands in a slot that still holds an unread value;
+  * no copy reads a source slot that its sender has already rewritten for a
+    later tile;
   * no barrier phase completes on bytes of another tile;
   * no wait finds its barrier two phases ahead (the hardware waits on the
     phase parity);
@@ -75,6 +80,9 @@ def simulate(C, tiles, seed, buffers=2, warps=4):
     slots = [[[[[None] * warps for _ in range(C)] for _ in range(buffers)] for _ in range(groups)]
              for _ in range(C)]
     # each (CTA, group, warp) walks its tiles u = g, g + 2, ... (local v = u // 2)
+    # own[CTA][group][buf][warp] = the tile whose values the warp last wrote
+    # into its own slot (the source of its copies)
+    own = [[[[None] * warps for _ in range(buffers)] for _ in range(groups)] for _ in range(C)]
     step = {(h, g, w): ("send", g) for h in range(C) for g in range(groups) for w in range(warps)}
     in_flight = []  # (receiver, group, buf, sender, warp, tile)
     errors = []
@@ -96,6 +104,9 @@ def simulate(C, tiles, seed, buffers=2, warps=4):
         kind, what = rng.choice(choices)
         if kind == "deliver":
             recv, g, b, sender, w, tile = in_flight.pop(what)
+            if own[sender][g][b][w] != tile:
+                errors.append(f"CTA {sender} warp {w}: copy of tile {tile} read its source "
+                              f"after it was rewritten for tile {own[sender][g][b][w]}")
             cell = slots[recv][g][b][sender][w]
             if cell is not None and not cell[1]:
                 errors.append(f"CTA {recv}: slot [{g}][{b}][{sender}][{w}] overwritten by tile "
@@ -110,6 +121,7 @@ def simulate(C, tiles, seed, buffers=2, warps=4):
         if st == "send":
             if w == 0:
                 on_complete(bars[h][g][par].arrive_expect((C - 1) * warps, u), h, g, par, u)
+            own[h][g][par][w] = u
             for p in range(C):
                 if p != h:
                     in_flight.append((p, g, par, h, w, u))
@@ -153,6 +165,13 @@ def test_single_buffered_exchange_is_caught():
             found = True
             break
     assert found
+
+
+def test_source_rewrite_is_caught():
+    # Single-buffered, a warp can also rewrite its own slot for its next
+    # tile while a copy of the current tile still has to read it.
+    assert any(any("read its source" in e for e in simulate(4, tiles=12, seed=seed, buffers=1))
+               for seed in range(400))
 
 
 def simulate_abort(C, tiles, seed, warps=4, settle=True):
