@@ -451,7 +451,10 @@ sa_status sa_refine_stack_forward(int layers, const sa_query* qs, const sa_refin
  * the device.  Calls on one cache that move data (lookup, insert, forward)
  * must be ordered with one another by the caller: the library reuses one
  * device slot list, so use one stream per cache.  Every call must be made
- * with the cache's device current (SA_ERR_INVALID_ARG otherwise).
+ * with the cache's device current (SA_ERR_INVALID_ARG otherwise), and `now`
+ * must be finite (SA_ERR_INVALID_ARG otherwise).  SA_ERR_CUDA from a call
+ * also covers a failed host allocation in the index; the cache's index may
+ * then be partly updated, so free the cache.
  */
 typedef struct sa_cache_key {
   int64_t user;
@@ -464,11 +467,14 @@ typedef struct sa_cache_s* sa_cache;
 
 /* A cache of `capacity` sketches of k x d (k >= 1, d >= 4 and a multiple of
  * 4, capacity >= 1) with a time-to-live of ttl_seconds (> 0).  Allocates
- * capacity * k * (d + 1) * 4 bytes on the current device.  Errors:
- * SA_ERR_INVALID_ARG, SA_ERR_CUDA. */
+ * capacity * k * (d + 1) * 4 bytes on the current device (SA_ERR_INVALID_ARG
+ * if that count does not fit in size_t).  Errors: SA_ERR_INVALID_ARG,
+ * SA_ERR_CUDA. */
 sa_status sa_cache_create(int k, int d, int64_t capacity, double ttl_seconds, sa_cache* out);
 
-/* Releases the cache and its device memory.  NULL is a no-op. */
+/* Waits for the cache's device, then releases the cache and its device
+ * memory (any device may be current; it is current again on return).  NULL
+ * is a no-op. */
 void sa_cache_free(sa_cache c);
 
 /*
@@ -584,7 +590,8 @@ sa_status sa_prepare_action(const float* W1, const float* W3, const float* W2,
                             const float* action_table, int d, int d_a, int h, int n_types,
                             void* stream, sa_action* out);
 
-/* Releases a producer (synchronises with the device).  NULL is a no-op. */
+/* Waits for the producer's device, then releases the producer (any device
+ * may be current; it is current again on return).  NULL is a no-op. */
 void sa_action_free(sa_action act);
 
 /*

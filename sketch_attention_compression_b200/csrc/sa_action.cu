@@ -608,10 +608,16 @@ sa_status sa_prepare_action(const float* W1, const float* W3, const float* W2,
 
 void sa_action_free(sa_action act) {
   if (act == nullptr) return;
+  // Producer kernels enqueued earlier may still read the weights: wait for
+  // the producer's device (made current for this call only).
+  int prev = -1;
+  const bool switched = cudaGetDevice(&prev) == cudaSuccess && prev != act->device &&
+                        cudaSetDevice(act->device) == cudaSuccess;
   cudaDeviceSynchronize();
   cudaFree(act->w13t);
   cudaFree(act->w2t);
   cudaFree(act->t13t);
+  if (switched) cudaSetDevice(prev);
   delete act;
 }
 

@@ -29,6 +29,8 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cmath>
+#include <cstdint>
 #include <map>
 #include <mutex>
 #include <new>
@@ -509,6 +511,9 @@ sa_status sa_cache_create(int k, int d, int64_t capacity, double ttl_seconds, sa
   if (out == nullptr) return SA_ERR_INVALID_ARG;
   *out = nullptr;
   if (k < 1 || d < 4 || d % 4 != 0 || capacity < 1 || !(ttl_seconds > 0.0)) return SA_ERR_INVALID_ARG;
+  // The pool's byte count, capacity * k * (d + 1) * 4, must not wrap.
+  const uint64_t per_slot = static_cast<uint64_t>(k) * (static_cast<uint64_t>(d) + 1) * 4;
+  if (static_cast<uint64_t>(capacity) > SIZE_MAX / per_slot) return SA_ERR_INVALID_ARG;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
   sa_cache_s* c = new (std::nothrow) sa_cache_s;
@@ -527,17 +532,29 @@ sa_status sa_cache_create(int k, int d, int64_t capacity, double ttl_seconds, sa
     delete c;
     return SA_ERR_CUDA;
   }
-  c->slot_key.resize(capacity);
-  c->used.assign(capacity, false);
-  c->t_insert.assign(capacity, 0.0);
-  c->t_use.assign(capacity, 0.0);
-  for (int64_t s = 0; s < capacity; ++s) c->free_slots.insert(c->free_slots.end(), s);
+  try {
+    c->slot_key.resize(capacity);
+    c->used.assign(capacity, false);
+    c->t_insert.assign(capacity, 0.0);
+    c->t_use.assign(capacity, 0.0);
+    for (int64_t s = 0; s < capacity; ++s) c->free_slots.insert(c->free_slots.end(), s);
+  } catch (const std::bad_alloc&) {
+    cudaFree(c->pool_x);
+    cudaFree(c->pool_m);
+    delete c;
+    return SA_ERR_CUDA;
+  }
   *out = c;
   return SA_OK;
 }
 
 void sa_cache_free(sa_cache c) {
   if (c == nullptr) return;
+  // Kernels enqueued by earlier calls may still read the pool and the slot
+  // list: wait for the cache's device (made current for this call only).
+  int prev = -1;
+  const bool switched = cudaGetDevice(&prev) == cudaSuccess && prev != c->device &&
+                        cudaSetDevice(c->device) == cudaSuccess;
   cudaDeviceSynchronize();
   cudaFree(c->pool_x);
   cudaFree(c->pool_m);
@@ -546,12 +563,13 @@ void sa_cache_free(sa_cache c) {
     cudaFreeHost(s.host);
     if (s.ev != nullptr) cudaEventDestroy(s.ev);
   }
+  if (switched) cudaSetDevice(prev);
   delete c;
 }
 
 sa_status sa_cache_lookup(sa_cache c, const sa_cache_key* keys, int64_t batch, double now,
                           uint8_t* hit, float* X_tilde, float* mass, void* stream) {
-  if (c == nullptr || batch < 0) return SA_ERR_INVALID_ARG;
+  if (c == nullptr || batch < 0 || !std::isfinite(now)) return SA_ERR_INVALID_ARG;
   if (batch == 0) return SA_OK;
   if (keys == nullptr || hit == nullptr || X_tilde == nullptr || mass == nullptr ||
       !sa::al(X_tilde, 16) || !sa::al(mass, 4) || !sa::on_device(c->device))
@@ -560,13 +578,18 @@ sa_status sa_cache_lookup(sa_cache c, const sa_cache_key* keys, int64_t batch, d
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   SaStaging* sg = sa::begin_call(c, static_cast<size_t>(batch));
   if (sg == nullptr) return SA_ERR_CUDA;
-  const sa_status s = sa::lookup_impl(c, sg, keys, batch, now, hit, X_tilde, mass, st);
+  sa_status s;
+  try {
+    s = sa::lookup_impl(c, sg, keys, batch, now, hit, X_tilde, mass, st);
+  } catch (const std::bad_alloc&) {
+    s = SA_ERR_CUDA;
+  }
   return sa::end_call(c, sg, st) ? s : SA_ERR_CUDA;
 }
 
 sa_status sa_cache_insert(sa_cache c, const sa_cache_key* keys, int64_t batch, double now,
                           const float* X_tilde, const float* mass, void* stream) {
-  if (c == nullptr || batch < 0) return SA_ERR_INVALID_ARG;
+  if (c == nullptr || batch < 0 || !std::isfinite(now)) return SA_ERR_INVALID_ARG;
   if (batch == 0) return SA_OK;
   if (keys == nullptr || X_tilde == nullptr || mass == nullptr || !sa::al(X_tilde, 16) ||
       !sa::al(mass, 4) || !sa::on_device(c->device))
@@ -575,7 +598,12 @@ sa_status sa_cache_insert(sa_cache c, const sa_cache_key* keys, int64_t batch, d
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   SaStaging* sg = sa::begin_call(c, static_cast<size_t>(batch));
   if (sg == nullptr) return SA_ERR_CUDA;
-  const sa_status s = sa::insert_impl(c, sg, keys, batch, now, X_tilde, mass, st);
+  sa_status s;
+  try {
+    s = sa::insert_impl(c, sg, keys, batch, now, X_tilde, mass, st);
+  } catch (const std::bad_alloc&) {
+    s = SA_ERR_CUDA;
+  }
   return sa::end_call(c, sg, st) ? s : SA_ERR_CUDA;
 }
 
@@ -603,7 +631,8 @@ sa_status sa_cache_forward(sa_cache c, sa_query q, const sa_cache_key* keys, dou
                            void* workspace, size_t workspace_bytes, void* stream) {
   int k = 0, d = 0, dt = 0, kp = 0;
   if (c == nullptr || sa_query_info(q, &k, &d, &dt, &kp) != SA_OK) return SA_ERR_INVALID_ARG;
-  if (k != c->k || d != c->d || batch < 0 || total_rows < 0) return SA_ERR_INVALID_ARG;
+  if (k != c->k || d != c->d || batch < 0 || total_rows < 0 || !std::isfinite(now))
+    return SA_ERR_INVALID_ARG;
   if (batch == 0) return total_rows == 0 ? SA_OK : SA_ERR_INVALID_ARG;
   if (keys == nullptr || offsets_host == nullptr || X_tilde == nullptr || mass == nullptr ||
       hit == nullptr || workspace == nullptr || (total_rows > 0 && X == nullptr) ||
@@ -619,8 +648,13 @@ sa_status sa_cache_forward(sa_cache c, sa_query q, const sa_cache_key* keys, dou
   // Lookup slots, the runs' offsets (at most 2 batch + 1) and insert slots.
   SaStaging* sg = sa::begin_call(c, 4 * static_cast<size_t>(batch) + 1);
   if (sg == nullptr) return SA_ERR_CUDA;
-  const sa_status s = sa::forward_impl(c, sg, q, keys, now, X, offsets_host, batch, total_rows, k, d, dt,
-                                   X_tilde, mass, hit, workspace, st);
+  sa_status s;
+  try {
+    s = sa::forward_impl(c, sg, q, keys, now, X, offsets_host, batch, total_rows, k, d, dt, X_tilde,
+                         mass, hit, workspace, st);
+  } catch (const std::bad_alloc&) {
+    s = SA_ERR_CUDA;
+  }
   return sa::end_call(c, sg, st) ? s : SA_ERR_CUDA;
 }
 

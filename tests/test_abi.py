@@ -181,8 +181,9 @@ def test_backward_rejects_bad_arguments_on_the_host(lib):
 
 def test_cache_and_adapter_reject_bad_arguments_on_the_host(lib):
     out = ctypes.c_void_p(123)
+    # ... the last: capacity * k * (d + 1) * 4 bytes would not fit in size_t
     for k, d, cap, ttl in [(0, 128, 4, 1.0), (16, 6, 4, 1.0), (16, 128, 0, 1.0), (16, 128, 4, 0.0),
-                           (16, 128, 4, float("nan"))]:
+                           (16, 128, 4, float("nan")), (1024, 1024, 1 << 50, 1.0)]:
         assert lib.sa_cache_create(k, d, cap, ttl, ctypes.byref(out)) == binding.SA_ERR_INVALID_ARG
         assert out.value is None
     lib.sa_cache_free(None)  # NULL-safe

@@ -131,6 +131,18 @@ def test_cached_forward_rejects_bad_host_offsets():
         with pytest.raises(SAError):
             cache.forward(q, keys, 0.0, X, np.array(bad, dtype=np.int64))
     assert cache.stats()["misses"] == 0  # rejected before any lookup
+    # a time that is not finite would break the index's ordering
+    offs = np.array([0, 10, 30], dtype=np.int64)
+    Xt = torch.zeros((2, 64, 128), dtype=torch.float32, device="cuda")
+    m = torch.zeros((2, 64), dtype=torch.float32, device="cuda")
+    for now in (float("nan"), float("inf")):
+        with pytest.raises(SAError):
+            cache.forward(q, keys, now, X, offs)
+        with pytest.raises(SAError):
+            cache.lookup(keys, now, Xt, m)
+        with pytest.raises(SAError):
+            cache.insert(keys, now, Xt, m)
+    assert cache.stats() == {"entries": 0, "hits": 0, "misses": 0, "evictions": 0}
     cache.close()
     q.close()
 
