@@ -559,8 +559,10 @@ sa_status sa_refine_stack_forward(int layers, const sa_query* qs, const sa_refin
     if (qs[l] == nullptr || rs[l] == nullptr) return SA_ERR_INVALID_ARG;
     if (qs[l]->k != qs[0]->k || qs[l]->d != qs[0]->d) return SA_ERR_INVALID_ARG;
   }
+  if (batch < 0 || total_rows < 0) return SA_ERR_INVALID_ARG;
   if (batch == 0) return total_rows == 0 ? SA_OK : SA_ERR_INVALID_ARG;
-  if (workspace == nullptr || workspace_bytes < sa_workspace_bytes_refine_stack(qs[0], batch, total_rows))
+  if (out == nullptr || workspace == nullptr) return SA_ERR_INVALID_ARG;
+  if (workspace_bytes < sa_workspace_bytes_refine_stack(qs[0], batch, total_rows))
     return SA_ERR_WORKSPACE;
   // Layer outputs alternate between `out` and a buffer after the layer
   // workspace, so that the last layer writes `out` and no layer writes the
