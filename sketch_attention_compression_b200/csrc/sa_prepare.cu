@@ -74,32 +74,37 @@ __global__ void prepare_query_kernel(const void* __restrict__ P, const void* __r
   if (q_bf16 != nullptr) q_bf16[static_cast<size_t>(j) * d + e] = double_to_bf16_rne(acc);
 }
 
-// Q'_b = Q_b M for all users: out row (b, j) = sum_f Q[b][j][f] M[f][:],
-// fp32 multiply-adds in f order.  Rows j in [k, k_rows) are zero (the
-// padded prototypes of the bf16 copy).  A CTA of 256 threads computes 32
-// rows x 64 columns: thread (ty, tx) owns rows 2ty, 2ty+1 and columns
-// 4tx..4tx+3.  Its 32 rows of Q and 64 columns of M (all d of f) are
+// Per-user query rows Q'_b = Q_b M for all users (fp32; a few MFLOP per
+// call): out row (b, j) = sum_f Q[b][j][f] M[f][:], and rows j in
+// [k, k_rows) are zero (the padded prototypes of the bf16 copy).  A CTA of
+// 256 threads computes a tile of 32 rows x 64 columns: thread (ty, tx) owns
+// rows 2ty, 2ty+1 and columns 4tx..4tx+3, each an fmaf chain over f in
+// ascending order.  Its 32 rows of Q and 64 columns of M (all d of f) are
 // staged in shared memory in one step, so the CTA waits for global memory
-// once.
+// once.  The staging moves 16-byte units and finds a unit's user and row
+// with one 32-bit division per unit (rows stay below 2^31); Q is read in
+// units when it is 16-byte aligned, else word by word.
 constexpr int kUqRows = 32, kUqCols = 64;
+constexpr int kUqPad = 4;  // Q rows d + 4 floats apart: whole units, and rows 2ty, 2ty+1 on different banks
 
 size_t user_query_smem(int d) {
-  return (static_cast<size_t>(kUqRows) * (d + 1) + static_cast<size_t>(d) * kUqCols) *
+  return (static_cast<size_t>(kUqRows) * (d + kUqPad) + static_cast<size_t>(d) * kUqCols) *
          sizeof(float);
 }
 
+template <bool kVecQ>
 __global__ void __launch_bounds__(256)
-    user_query_kernel(const float* __restrict__ Q, const float* __restrict__ M, int64_t B, int k,
-                      int k_rows, int d, float* __restrict__ out_f32,
+    user_query_kernel(const float* __restrict__ Q, const float* __restrict__ M, uint32_t total,
+                      int k, int k_rows, int d, float* __restrict__ out_f32,
                       uint16_t* __restrict__ out_bf16) {
-  extern __shared__ float uq_sh[];
-  float* qs = uq_sh;                            // [32][d + 1]
-  float* ms = uq_sh + kUqRows * (d + 1);        // [d][64]
+  extern __shared__ __align__(16) float uq_sh[];
+  const int ld = d + kUqPad;
+  float* qs = uq_sh;                  // [32][d + 4]
+  float* ms = uq_sh + kUqRows * ld;   // [d][64]
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kUqRows;
+  const uint32_t row0 = blockIdx.x * kUqRows;
   const int col0 = blockIdx.y * kUqCols;
-  const int64_t total = B * k_rows;
   // Launched as a programmatic dependent of the stream's previous kernel
   // (for back-to-back calls, the previous call's finalize, which already
   // waited for the fused pass that read the old Q'_b): nothing is read or
@@ -107,25 +112,34 @@ __global__ void __launch_bounds__(256)
   // then start its own set-up (it waits for this grid before reading).
   grid_dependency_wait();
   grid_dependency_launch();
-  for (int i = tid; i < kUqRows * d; i += 256) {
-    const int rr = i / d, ff = i - rr * d;
-    const int64_t R = row0 + rr;
-    float v = 0.f;
+  const int d4 = d >> 2;
+  for (int i = tid; i < kUqRows * d4; i += 256) {
+    const int rr = i / d4, u = i - rr * d4;
+    const uint32_t R = row0 + static_cast<uint32_t>(rr);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (R < total) {
-      const int64_t b = R / k_rows;
-      const int j = static_cast<int>(R - b * k_rows);
-      if (j < k) v = Q[(b * k + j) * d + ff];
+      const uint32_t b = R / static_cast<uint32_t>(k_rows);
+      const int j = static_cast<int>(R - b * static_cast<uint32_t>(k_rows));
+      if (j < k) {
+        const float* src = Q + (static_cast<int64_t>(b) * k + j) * d + 4 * u;
+        if constexpr (kVecQ) {
+          v = *reinterpret_cast<const float4*>(src);
+        } else {
+          v = make_float4(src[0], src[1], src[2], src[3]);
+        }
+      }
     }
-    qs[rr * (d + 1) + ff] = v;
+    *reinterpret_cast<float4*>(qs + rr * ld + 4 * u) = v;
   }
-  for (int i = tid; i < d * kUqCols; i += 256) {
-    const int ff = i / kUqCols, cc = i % kUqCols;
-    ms[i] = M[static_cast<int64_t>(ff) * d + col0 + cc];
+  for (int i = tid; i < d * (kUqCols / 4); i += 256) {
+    const int ff = i >> 4, u = i & 15;
+    *reinterpret_cast<float4*>(ms + ff * kUqCols + 4 * u) =
+        *reinterpret_cast<const float4*>(M + static_cast<int64_t>(ff) * d + col0 + 4 * u);
   }
   __syncthreads();
   float acc[2][4] = {};
-  const float* q0p = qs + (2 * ty) * (d + 1);
-  const float* q1p = q0p + (d + 1);
+  const float* q0p = qs + (2 * ty) * ld;
+  const float* q1p = q0p + ld;
 #pragma unroll 8
   for (int ff = 0; ff < d; ++ff) {
     const float q0 = q0p[ff], q1 = q1p[ff];
@@ -139,16 +153,19 @@ __global__ void __launch_bounds__(256)
     acc[1][2] = fmaf(q1, mv.z, acc[1][2]);
     acc[1][3] = fmaf(q1, mv.w, acc[1][3]);
   }
+  // Four consecutive columns: one 16-byte fp32 store, one 8-byte bf16 store
+  // (the outputs are 256-byte aligned and d is a multiple of 64).
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
-    const int64_t R = row0 + 2 * ty + hh;
+    const uint32_t R = row0 + static_cast<uint32_t>(2 * ty + hh);
     if (R >= total) continue;
-    const int64_t o = R * d + col0 + 4 * tx;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (out_f32 != nullptr) out_f32[o + u] = acc[hh][u];
-      if (out_bf16 != nullptr) out_bf16[o + u] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[hh][u]));
-    }
+    const int64_t o = static_cast<int64_t>(R) * d + col0 + 4 * tx;
+    if (out_f32 != nullptr)
+      *reinterpret_cast<float4*>(out_f32 + o) =
+          make_float4(acc[hh][0], acc[hh][1], acc[hh][2], acc[hh][3]);
+    if (out_bf16 != nullptr)
+      *reinterpret_cast<uint2*>(out_bf16 + o) =
+          make_uint2(pack_bf16x2(acc[hh][0], acc[hh][1]), pack_bf16x2(acc[hh][2], acc[hh][3]));
   }
 }
 
@@ -159,12 +176,17 @@ cudaError_t launch_user_query(const float* queries, const float* M, int64_t batc
                               cudaStream_t stream) {
   const int64_t rows = batch * k_rows;
   if (rows <= 0) return cudaSuccess;
+  if (rows >= (int64_t{1} << 31) || d % kUqCols != 0 ||
+      (reinterpret_cast<uintptr_t>(out_f32) & 15u) != 0 ||
+      (reinterpret_cast<uintptr_t>(out_bf16) & 7u) != 0)
+    return cudaErrorInvalidValue;
+  const bool vec = (reinterpret_cast<uintptr_t>(queries) & 15u) == 0;
+  auto kern = vec ? user_query_kernel<true> : user_query_kernel<false>;
   const dim3 grid(static_cast<unsigned>((rows + kUqRows - 1) / kUqRows),
                   static_cast<unsigned>(d / kUqCols));
   const size_t smem = user_query_smem(d);
-  cudaError_t err = cudaFuncSetAttribute(user_query_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+  cudaError_t err =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -176,8 +198,8 @@ cudaError_t launch_user_query(const float* queries, const float* M, int64_t batc
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, user_query_kernel, queries, M, batch, k, k_rows, d, out_f32,
-                            out_bf16);
+  return cudaLaunchKernelEx(&cfg, kern, queries, M, static_cast<uint32_t>(rows), k, k_rows, d,
+                            out_f32, out_bf16);
 }
 
 cudaError_t launch_prepare_projection(const void* W_Q, const void* W_K, int d, double scale,

@@ -152,6 +152,37 @@ def test_errors():
     q.close()
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_queries_only_4_byte_aligned(dtype):
+    # The Q'_b kernel stages 16-byte units of Q when the array is 16-byte
+    # aligned and single words otherwise; both give the same sketches, bit
+    # for bit, and match the oracle.
+    import torch
+    from sketch_attention_compression_b200 import SketchQuery
+    lengths = [300, 129, 1, 0, 700]
+    inp = make_inputs(lengths, d=128, k=100, dtype=dtype, seed=41)
+    queries = user_queries(len(lengths), 100, 128, seed=42)
+    dev = to_device(inp)
+    q = SketchQuery(dev["P"], dev["W_Q"], dev["W_K"], inp["scale"])
+    flat = torch.from_numpy(queries.astype(np.float32).ravel()).cuda()
+    buf = torch.zeros(flat.numel() + 4, dtype=torch.float32, device="cuda")
+    buf[1:1 + flat.numel()] = flat
+    shape = (len(lengths), 100, 128)
+    Q16, Q4 = flat.view(shape), buf[1:1 + flat.numel()].view(shape)
+    assert Q16.data_ptr() % 16 == 0 and Q4.data_ptr() % 16 == 4
+    outs = []
+    for Qd in (Q16, Q4):
+        Xt, m = q.forward_user_queries(Qd, dev["X"], dev["offsets"], check=True)
+        outs.append((Xt.cpu(), m.cpu()))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    q.close()
+    Xt_o, m_o = sa_batch_user_queries(inp["X"], inp["offsets"], queries, inp["W_Q"], inp["W_K"],
+                                      inp["scale"])
+    for b in range(len(lengths)):
+        assert_user_close(outs[1][0][b].double().numpy(), outs[1][1][b].double().numpy(),
+                          Xt_o[b], m_o[b], dtype, f"user {b}")
+
+
 def test_mass_normalise():
     # X~_j / m_j against the oracle's mass_normalised, 0 for the empty
     # user's rows; in place gives the same bits.
