@@ -4,8 +4,9 @@
 // of every user is covered by exactly one segment; cta_of_row names the CTA
 // that covered each row; users inside one CTA range go straight to the
 // outputs; split users use distinct partial slots below 2G; the finalize
-// pass reduces every split user exactly once, over exactly the slots that
-// the partial pass wrote for it, in ascending CTA order.  The 32-way search
+// pass (one unit per user, from the user's offsets and one range search)
+// reduces every split user exactly once, over exactly the slots that the
+// partial pass wrote for it, in ascending CTA order.  The 32-way search
 // the kernels use (warp_range_begin) is replayed here step by step and must
 // agree with the serial search.
 #include <cstdio>
@@ -100,19 +101,21 @@ static int check(const std::vector<int64_t>& off, int64_t sms) {
     while (off[u + 1] <= r) ++u;
     if (cta_of_row(off.data(), u, B, N, G, r) != owner[r]) return fail("cta_of_row", r, owner[r]);
   }
-  // finalize ownership, same arithmetic as finalize_kernel
+  // finalize ownership, same arithmetic as finalize_kernel: per user, the
+  // CTAs holding its first and last rows; split if they differ; the first
+  // CTA's slot by whether that CTA's range starts at the user's first row
+  // (found with the warp search the kernel uses), then 2c for later CTAs.
   std::map<int64_t, std::vector<int64_t>> reduced;
-  for (int64_t cb = 1; cb < G; ++cb) {
-    int64_t b, bp;
-    const int64_t Rc = range_begin(off.data(), B, N, cb, G, &b);
-    const int64_t Rp = range_begin(off.data(), B, N, cb - 1, G, &bp);
-    if (b >= B) continue;
+  for (int64_t b = 0; b < B; ++b) {
     const int64_t lo = off[b], hi = off[b + 1];
-    if (!(lo < Rc && lo >= Rp && hi > Rc)) continue;
-    if (reduced.count(b)) return fail("user reduced twice", b, cb);
+    if (lo >= hi) continue;
+    const int64_t c_lo = cta_of_row(off.data(), b, B, N, G, lo);
     const int64_t c_hi = cta_of_row(off.data(), b, B, N, G, hi - 1 < N - 1 ? hi - 1 : N - 1);
-    std::vector<int64_t> slots{2 * (cb - 1) + (lo <= Rp ? 0 : 1)};
-    for (int64_t cc = cb; cc <= c_hi; ++cc) slots.push_back(2 * cc);
+    if (c_hi <= c_lo) continue;
+    int64_t ub;
+    const int64_t first = warp_search_replay(off.data(), B, N, c_lo, G, &ub);
+    std::vector<int64_t> slots{2 * c_lo + (lo <= first ? 0 : 1)};
+    for (int64_t cc = c_lo + 1; cc <= c_hi; ++cc) slots.push_back(2 * cc);
     reduced[b] = slots;
   }
   for (int64_t b = 0; b < B; ++b) {
