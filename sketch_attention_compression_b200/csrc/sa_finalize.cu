@@ -12,8 +12,8 @@
 //    offsets[B] == N); violations set bits in the workspace header.
 //
 // Block roles: the grid strides over units of a user: a run of consecutive
-// chunks, where a chunk is 2048 entries of the user's k*d sketch (one
-// 16-byte piece per thread) and 512 of its k masses, and the runs are long
+// chunks, where a chunk is 1024 entries of the user's k*d sketch (one
+// 16-byte piece per thread) and 256 of its k masses, and the runs are long
 // enough that the units of the users that can be split fit in about one
 // wave.  The user's two offsets
 // decide the unit in one round trip: an empty user is zero-filled; for the others
@@ -30,10 +30,10 @@
 namespace sa {
 namespace {
 
-constexpr int kFinThreads = 512;
+constexpr int kFinThreads = 256;
 constexpr int kChunkFloats = 4 * kFinThreads;  // sketch entries per chunk
 constexpr int kFinBatch = 8;                   // slots loaded per round trip
-constexpr int kFinBlocksPerSm = 1;             // resident blocks per SM (128 registers, no spills)
+constexpr int kFinBlocksPerSm = 2;             // resident blocks per SM (128 registers, no spills)
 constexpr int64_t kFinWave = 148 * kFinBlocksPerSm;  // blocks of one wave on a B200
 
 __device__ __forceinline__ float4 add4(float4 s, float4 v) {
