@@ -77,30 +77,29 @@ __global__ void prepare_query_kernel(const void* __restrict__ P, const void* __r
 // Per-user query rows Q'_b = Q_b M for all users (fp32; a few MFLOP per
 // call): out row (b, j) = sum_f Q[b][j][f] M[f][:], and rows j in
 // [k, k_rows) are zero (the padded prototypes of the bf16 copy).  A CTA of
-// 256 threads computes a tile of 32 rows x 64 columns: thread (ty, tx) owns
-// rows 2ty, 2ty+1 and columns 4tx..4tx+3, each an fmaf chain over f in
-// ascending order.  Its 32 rows of Q and 64 columns of M (all d of f) are
-// staged in shared memory in one step, so the CTA waits for global memory
-// once.  The staging moves 16-byte units and finds a unit's user and row
-// with one 32-bit division per unit (rows stay below 2^31); Q is read in
-// units when it is 16-byte aligned, else word by word.
-constexpr int kUqRows = 32, kUqCols = 64;
-constexpr int kUqPad = 4;  // Q rows d + 4 floats apart: whole units, and rows 2ty, 2ty+1 on different banks
+// 128 threads computes a tile of 32 rows x 64 columns: thread (ty, tx) owns
+// rows 4ty..4ty+3 and columns 4tx..4tx+3, each an fmaf chain over f in
+// ascending order.  The tile's 32 rows of Q (transposed: [f][row], so a
+// thread's four row values are one 16-byte read) and 64 columns of M (all d
+// of f) are staged in shared memory in one step, so the CTA waits for
+// global memory once; per f a warp then reads 3 shared-memory wavefronts
+// for 16 multiply-adds per thread.  The staging reads Q in 16-byte units
+// when it is 16-byte aligned, else word by word, and finds a unit's user
+// and row with one 32-bit division (rows stay below 2^31).
+constexpr int kUqRows = 32, kUqCols = 64, kUqThreads = 128;
 
 size_t user_query_smem(int d) {
-  return (static_cast<size_t>(kUqRows) * (d + kUqPad) + static_cast<size_t>(d) * kUqCols) *
-         sizeof(float);
+  return (static_cast<size_t>(d) * kUqRows + static_cast<size_t>(d) * kUqCols) * sizeof(float);
 }
 
 template <bool kVecQ>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kUqThreads)
     user_query_kernel(const float* __restrict__ Q, const float* __restrict__ M, uint32_t total,
                       int k, int k_rows, int d, float* __restrict__ out_f32,
                       uint16_t* __restrict__ out_bf16) {
   extern __shared__ __align__(16) float uq_sh[];
-  const int ld = d + kUqPad;
-  float* qs = uq_sh;                  // [32][d + 4]
-  float* ms = uq_sh + kUqRows * ld;   // [d][64]
+  float* qt = uq_sh;                 // [d][32]: qt[f][r] = Q row r of the tile, entry f
+  float* ms = uq_sh + d * kUqRows;   // [d][64]
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
   const uint32_t row0 = blockIdx.x * kUqRows;
@@ -112,9 +111,11 @@ __global__ void __launch_bounds__(256)
   // then start its own set-up (it waits for this grid before reading).
   grid_dependency_wait();
   grid_dependency_launch();
+  // Q: a warp takes one 16-byte unit of 32 consecutive rows, so its
+  // transposed stores are 32 consecutive words.
   const int d4 = d >> 2;
-  for (int i = tid; i < kUqRows * d4; i += 256) {
-    const int rr = i / d4, u = i - rr * d4;
+  for (int i = tid; i < kUqRows * d4; i += kUqThreads) {
+    const int rr = i & (kUqRows - 1), u = i >> 5;
     const uint32_t R = row0 + static_cast<uint32_t>(rr);
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (R < total) {
@@ -129,43 +130,43 @@ __global__ void __launch_bounds__(256)
         }
       }
     }
-    *reinterpret_cast<float4*>(qs + rr * ld + 4 * u) = v;
+    qt[(4 * u + 0) * kUqRows + rr] = v.x;
+    qt[(4 * u + 1) * kUqRows + rr] = v.y;
+    qt[(4 * u + 2) * kUqRows + rr] = v.z;
+    qt[(4 * u + 3) * kUqRows + rr] = v.w;
   }
-  for (int i = tid; i < d * (kUqCols / 4); i += 256) {
+  for (int i = tid; i < d * (kUqCols / 4); i += kUqThreads) {
     const int ff = i >> 4, u = i & 15;
     *reinterpret_cast<float4*>(ms + ff * kUqCols + 4 * u) =
         *reinterpret_cast<const float4*>(M + static_cast<int64_t>(ff) * d + col0 + 4 * u);
   }
   __syncthreads();
-  float acc[2][4] = {};
-  const float* q0p = qs + (2 * ty) * ld;
-  const float* q1p = q0p + ld;
-#pragma unroll 8
+  float acc[4][4] = {};
+#pragma unroll 4
   for (int ff = 0; ff < d; ++ff) {
-    const float q0 = q0p[ff], q1 = q1p[ff];
+    const float4 qv = *reinterpret_cast<const float4*>(qt + ff * kUqRows + 4 * ty);
     const float4 mv = *reinterpret_cast<const float4*>(ms + ff * kUqCols + 4 * tx);
-    acc[0][0] = fmaf(q0, mv.x, acc[0][0]);
-    acc[0][1] = fmaf(q0, mv.y, acc[0][1]);
-    acc[0][2] = fmaf(q0, mv.z, acc[0][2]);
-    acc[0][3] = fmaf(q0, mv.w, acc[0][3]);
-    acc[1][0] = fmaf(q1, mv.x, acc[1][0]);
-    acc[1][1] = fmaf(q1, mv.y, acc[1][1]);
-    acc[1][2] = fmaf(q1, mv.z, acc[1][2]);
-    acc[1][3] = fmaf(q1, mv.w, acc[1][3]);
+    const float q[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      acc[r][0] = fmaf(q[r], mv.x, acc[r][0]);
+      acc[r][1] = fmaf(q[r], mv.y, acc[r][1]);
+      acc[r][2] = fmaf(q[r], mv.z, acc[r][2]);
+      acc[r][3] = fmaf(q[r], mv.w, acc[r][3]);
+    }
   }
   // Four consecutive columns: one 16-byte fp32 store, one 8-byte bf16 store
-  // (the outputs are 256-byte aligned and d is a multiple of 64).
+  // (the outputs are 16- and 8-byte aligned and d is a multiple of 64).
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const uint32_t R = row0 + static_cast<uint32_t>(2 * ty + hh);
+  for (int r = 0; r < 4; ++r) {
+    const uint32_t R = row0 + static_cast<uint32_t>(4 * ty + r);
     if (R >= total) continue;
     const int64_t o = static_cast<int64_t>(R) * d + col0 + 4 * tx;
     if (out_f32 != nullptr)
-      *reinterpret_cast<float4*>(out_f32 + o) =
-          make_float4(acc[hh][0], acc[hh][1], acc[hh][2], acc[hh][3]);
+      *reinterpret_cast<float4*>(out_f32 + o) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
     if (out_bf16 != nullptr)
       *reinterpret_cast<uint2*>(out_bf16 + o) =
-          make_uint2(pack_bf16x2(acc[hh][0], acc[hh][1]), pack_bf16x2(acc[hh][2], acc[hh][3]));
+          make_uint2(pack_bf16x2(acc[r][0], acc[r][1]), pack_bf16x2(acc[r][2], acc[r][3]));
   }
 }
 
@@ -190,7 +191,7 @@ cudaError_t launch_user_query(const float* queries, const float* M, int64_t batc
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(256);
+  cfg.blockDim = dim3(kUqThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
