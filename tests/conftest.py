@@ -12,4 +12,4 @@ def pytest_configure(config):
     config.addinivalue_line(
         "markers", "gpu: needs a CUDA GPU (B200, sm_100a) and the built libsa.so")
     config.addinivalue_line(
-        "markers", "slow: full-size workload; runs on the GPU box only")
+        "markers", "slow: full-size workload; needs a B200 with the full workload resident")
