@@ -21,9 +21,10 @@
 // arithmetic on the two offsets), and if they differ the user is split and
 // the unit sums its slots: 2c for each later CTA c (the user starts before
 // their ranges), and for the first CTA slot 2c if that CTA's range starts
-// at the user's first row, else 2c + 1.  Only that last choice needs a
-// range start, which warp 0 searches while every thread's slot loads are in
-// flight.  The validation bits are taken by chunk 0 of each user.
+// at the user's first row, else 2c + 1.  That last choice has a closed form
+// when the user before is not empty; otherwise warp 0 searches the range
+// start while every thread's slot loads are in flight.  The validation bits
+// are taken by the first unit of each user.
 #include "sa_internal.h"
 #include "sa_ptx.cuh"
 
@@ -61,6 +62,7 @@ __global__ void __launch_bounds__(kFinThreads, kFinBlocksPerSm)
     const int g = static_cast<int>(u - b * groups);
     const int ch0 = g * per_unit, ch1 = min(ch0 + per_unit, chunks);
     const int64_t lo = a.offsets[b], hi = a.offsets[b + 1];
+    const int64_t prev = b > 0 ? a.offsets[b - 1] : -1;
     if (g == 0 && threadIdx.x == 0) {
       uint32_t bits = 0;
       if (b == 0 && lo != 0) bits |= DEVFLAG_OFFSET0_NONZERO;
@@ -113,14 +115,25 @@ __global__ void __launch_bounds__(kFinThreads, kFinBlocksPerSm)
         }
       }
       if (ch == ch0) {  // once per unit, while the loads above are in flight
-        if (threadIdx.x < 32) {
-          int64_t ub;
-          const int64_t r = warp_range_begin(a.offsets, B, N, c_lo, G, threadIdx.x, &ub);
-          if (threadIdx.x == 0) s_first = r;
+        if (prev < lo) {
+          // The user before b is not empty (or b = 0): range c_lo starts at
+          // lo exactly when its cost target falls in b's start cost or
+          // first tile (a target in an earlier user gives a start before
+          // that user's end, which is below lo).
+          const int64_t tau = c_lo > 0 ? range_target(B, N, c_lo, G) : 0;
+          const int64_t cb = lo + kUserStartCost * b;  // cost_before_user(b)
+          first = c_lo > 0 ? (tau >= cb && tau < cb + kUserStartCost + kTileRows) : lo == 0;
+        } else {
+          // Empty users (or bad offsets) just before b: find the range start.
+          if (threadIdx.x < 32) {
+            int64_t ub;
+            const int64_t r = warp_range_begin(a.offsets, B, N, c_lo, G, threadIdx.x, &ub);
+            if (threadIdx.x == 0) s_first = r;
+          }
+          __syncthreads();
+          first = lo <= s_first;
+          __syncthreads();  // s_first is rewritten by the block's next unit
         }
-        __syncthreads();
-        first = lo <= s_first;
-        __syncthreads();  // s_first is rewritten by the block's next unit
       }
       float4 sx = first ? x0 : x1;
       float sm = first ? m0 : m1;

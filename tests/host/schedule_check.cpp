@@ -104,7 +104,8 @@ static int check(const std::vector<int64_t>& off, int64_t sms) {
   // finalize ownership, same arithmetic as finalize_kernel: per user, the
   // CTAs holding its first and last rows; split if they differ; the first
   // CTA's slot by whether that CTA's range starts at the user's first row
-  // (found with the warp search the kernel uses), then 2c for later CTAs.
+  // (in closed form after a non-empty user, else found with the warp search
+  // the kernel uses), then 2c for later CTAs.
   std::map<int64_t, std::vector<int64_t>> reduced;
   for (int64_t b = 0; b < B; ++b) {
     const int64_t lo = off[b], hi = off[b + 1];
@@ -112,9 +113,21 @@ static int check(const std::vector<int64_t>& off, int64_t sms) {
     const int64_t c_lo = cta_of_row(off.data(), b, B, N, G, lo);
     const int64_t c_hi = cta_of_row(off.data(), b, B, N, G, hi - 1 < N - 1 ? hi - 1 : N - 1);
     if (c_hi <= c_lo) continue;
-    int64_t ub;
-    const int64_t first = warp_search_replay(off.data(), B, N, c_lo, G, &ub);
-    std::vector<int64_t> slots{2 * c_lo + (lo <= first ? 0 : 1)};
+    bool first;
+    const int64_t prev = b > 0 ? off[b - 1] : -1;
+    if (prev < lo) {  // closed form, as in finalize_kernel
+      const int64_t tau = c_lo > 0 ? range_target(B, N, c_lo, G) : 0;
+      const int64_t cb = lo + kUserStartCost * b;
+      first = c_lo > 0 ? (tau >= cb && tau < cb + kUserStartCost + kTileRows) : lo == 0;
+      // and it agrees with the range start the partial pass uses
+      int64_t ub0;
+      if (first != (lo <= range_begin(off.data(), B, N, c_lo, G, &ub0)))
+        return fail("closed-form first slot", b, c_lo);
+    } else {
+      int64_t ub;
+      first = lo <= warp_search_replay(off.data(), B, N, c_lo, G, &ub);
+    }
+    std::vector<int64_t> slots{2 * c_lo + (first ? 0 : 1)};
     for (int64_t cc = c_lo + 1; cc <= c_hi; ++cc) slots.push_back(2 * cc);
     reduced[b] = slots;
   }
