@@ -60,6 +60,16 @@ def test_one_long_user_split_across_all_ctas():
     _full_parity(make_inputs([200_000], d=128, k=64, dtype="bf16", seed=12))
 
 
+@pytest.mark.parametrize("d,k,dtype", [(128, 128, "bf16"), (64, 64, "fp32"), (256, 256, "bf16")])
+def test_split_users_after_empty_and_full_users(d, k, dtype):
+    # Long users split over many CTA ranges, some right after a run of empty
+    # users and some right after a non-empty user: the finalize pass picks
+    # the first range's partial slot by a range search in the first case and
+    # in closed form in the second; every user against the oracle.
+    lengths = [3000, 0, 0, 0, 40000, 0, 25000, 1, 0, 30000, 17000, 5, 22000, 0]
+    _full_parity(make_inputs(lengths, d=d, k=k, dtype=dtype, seed=d + k + 5))
+
+
 def test_k1_is_column_sum():
     inp = make_inputs([500, 129, 0, 3], d=128, k=1, dtype="bf16", seed=13)
     Xt_g, m_g, _ = run_gpu(inp)
