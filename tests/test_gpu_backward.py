@@ -93,6 +93,16 @@ def test_backward_user_split_across_all_ctas():
     _check(got, want, inp["offsets"])
 
 
+def test_backward_full_size_benchmark_workload():
+    # The benchmark's workload and launch configuration (16 users x 100K
+    # rows, d = k = 128, mixture X, G and g ~ N(0, 1)); every output of every
+    # user against the oracle (about half a second per user on the CPU).
+    from synthetic import generate
+    inp = generate("batch16_n100k_d128_k128_mixture_bf16")
+    got, want = _run(inp, per_user=False, with_g=True, seed=330)
+    _check(got, want, inp["offsets"])
+
+
 def test_backward_bitwise_deterministic():
     inp = make_inputs([40_000, 3, 20_000], d=128, k=128, dtype="bf16", seed=220, x_kind="mixture")
     a, _ = _run(inp, per_user=False, with_g=True, seed=320)

@@ -119,6 +119,40 @@ def test_cached_forward_serves_hits_and_computes_misses(k):
     q.close()
 
 
+def test_cached_forward_full_size():
+    # The benchmark's 16 x 100K workload through the cache: the first call
+    # computes every user; the second keeps ten of the sixteen keys, serves
+    # them from the pool bit for bit and recomputes the other six in place;
+    # sampled users of both calls against the oracle.
+    import torch
+    from gpu_util import assert_total_mass
+    from sketch_attention_compression_b200 import SketchCache, read_device_status
+    from synthetic import generate
+    inp = generate("batch16_n100k_d128_k128_mixture_bf16")
+    q = _query(inp)
+    X = torch.from_numpy(inp["X"]).cuda().to(torch.bfloat16)
+    cache = SketchCache(128, 128, capacity=32, ttl=60.0)
+    keys = [(1000 + b, 1, 7, 0) for b in range(16)]
+    Xt1, m1, hit1, ws = cache.forward(q, keys, 0.0, X, inp["offsets"])
+    assert not hit1.any() and read_device_status(ws) == 0
+    g1x, g1m = Xt1.double().cpu().numpy(), m1.double().cpu().numpy()
+    keys2 = keys[:10] + [(2000 + b, 1, 7, 0) for b in range(10, 16)]
+    Xt2, m2, hit2, _ = cache.forward(q, keys2, 1.0, X, inp["offsets"], workspace=ws)
+    assert list(hit2) == [b < 10 for b in range(16)]
+    assert read_device_status(ws) == 0
+    g2x, g2m = Xt2.double().cpu().numpy(), m2.double().cpu().numpy()
+    assert np.array_equal(g2x[:10], g1x[:10]) and np.array_equal(g2m[:10], g1m[:10])
+    users = [0, 9, 10, 15]
+    Xo, mo = sa_batch(inp["X"], inp["offsets"], inp["P"], inp["W_Q"], inp["W_K"], inp["scale"],
+                      users=users)
+    for b in users:
+        assert_user_close(g1x[b], g1m[b], Xo[b], mo[b], "bf16", f"user {b} (first call)")
+        assert_user_close(g2x[b], g2m[b], Xo[b], mo[b], "bf16", f"user {b} (second call)")
+    assert_total_mass(g2m, inp["offsets"], "bf16")
+    cache.close()
+    q.close()
+
+
 def test_cached_forward_rejects_bad_host_offsets():
     import torch
     from sketch_attention_compression_b200 import SAError, SketchCache

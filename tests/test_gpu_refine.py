@@ -121,6 +121,30 @@ def test_refine_stack_two_layers_k1000():
         o.close()
 
 
+def test_refine_stack_full_size_sampled():
+    # Two layers at k = 1000 on the benchmark's 16 x 100K workload, in the
+    # benchmark's launch configuration; a user's stack depends on its own
+    # rows only, so users 0 and 15 are checked against the oracle's stack
+    # (about four seconds each on the CPU).
+    import torch
+    from sketch_attention_compression_b200 import read_device_status, refine_stack_forward
+    from synthetic import generate
+    inp = generate("batch16_n100k_d128_k1000_mixture_bf16")
+    d, h = 128, 512
+    layers = [refine_params(d, h, seed=321), refine_params(d, h, seed=322)]
+    dev = to_device(inp)
+    qs = [_query(inp["P"], L) for L in layers]
+    rs = [_refine_handle(L) for L in layers]
+    out, ws = refine_stack_forward(qs, rs, torch.from_numpy(inp["P"]).cuda(), dev["X"],
+                                   dev["offsets"])
+    assert read_device_status(ws) == 0
+    users = [0, 15]
+    want = refine_stack(inp["X"], inp["offsets"], inp["P"], layers, users=users)
+    _close_users(out.double().cpu().numpy()[users], want[users], "full-size stack")
+    for o in qs + rs:
+        o.close()
+
+
 def test_refine_stack_reports_bad_offsets():
     import torch
     from sketch_attention_compression_b200 import read_device_status, refine_stack_forward
