@@ -525,8 +525,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         have_s = true;
       }
 
-      // dX_t: TMEM row -> bf16 -> global; each half drains d / 2 columns,
-      // 32 at a time.  With 128 prototypes the warp stages its 32 rows in
+      // dX_t: TMEM row -> bf16 -> global; each half drains d / 2 columns
+      // (all of its 32-column loads in flight before one wait).  With 128 prototypes the warp stages its 32 rows in
       // the part of the [A | dS'] tile that it alone writes (A's box hf,
       // rows 32 q ..), free once MMA3 has read it, then stores whole rows:
       // 128 (d = 64: 64) bytes of a row per 8 (4) lanes, instead of 16
@@ -541,16 +541,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         constexpr int XC = D / 64;  // 32-column chunks per half
         constexpr int U = D / 16;   // 16-byte units per half row
         const uint32_t box = sbase + Pl::kAS + hf * Pl::kXBox;
+        uint32_t xall[XC][32];
+#pragma unroll
+        for (int cc = 0; cc < XC; ++cc)
+          tmem_ld32(lane_addr + Pl::kColDX + hf * (D / 2) + cc * 32, xall[cc]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int cc = 0; cc < XC; ++cc) tmem_pin32(xall[cc]);
+        tc_fence_before();
+        warp_arrive(dx_empty, lane);
 #pragma unroll
         for (int cc = 0; cc < XC; ++cc) {
-          uint32_t xv[32];
-          tmem_ld32(lane_addr + Pl::kColDX + hf * (D / 2) + cc * 32, xv);
-          tmem_wait_ld();
-          tmem_pin32(xv);
-          if (cc == XC - 1) {
-            tc_fence_before();
-            warp_arrive(dx_empty, lane);
-          }
+          const uint32_t (&xv)[32] = xall[cc];
           if constexpr (KM == 64) {
             if (valid) {
               uint4* dst = reinterpret_cast<uint4*>(ba.dX + (r + row) * D + hf * (D / 2) + cc * 32);
