@@ -87,6 +87,8 @@ __global__ void prepare_query_kernel(const void* __restrict__ P, const void* __r
 // when it is 16-byte aligned, else word by word, and finds a unit's user
 // and row with one 32-bit division (rows stay below 2^31).
 constexpr int kUqRows = 32, kUqCols = 64, kUqThreads = 128;
+static_assert(kUqRows == 32, "the Q staging loop takes a unit's row from the low 5 bits");
+static_assert(kUqCols == 64 && kUqThreads == 128, "16 x 8 threads own 4 x 4 outputs each");
 
 size_t user_query_smem(int d) {
   return (static_cast<size_t>(d) * kUqRows + static_cast<size_t>(d) * kUqCols) * sizeof(float);
