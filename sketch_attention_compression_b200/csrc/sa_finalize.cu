@@ -15,16 +15,16 @@
 // chunks, where a chunk is 1024 entries of the user's k*d sketch (one
 // 16-byte piece per thread) and 256 of its k masses, and the runs are long
 // enough that the units of the users that can be split fit in about one
-// wave.  The user's two offsets
-// decide the unit in one round trip: an empty user is zero-filled; for the others
-// cta_of_row gives the CTAs that hold the first and the last row (pure
-// arithmetic on the two offsets), and if they differ the user is split and
-// the unit sums its slots: 2c for each later CTA c (the user starts before
-// their ranges), and for the first CTA slot 2c if that CTA's range starts
-// at the user's first row, else 2c + 1.  That last choice has a closed form
-// when the user before is not empty; otherwise warp 0 searches the range
-// start while every thread's slot loads are in flight.  The validation bits
-// are taken by the first unit of each user.
+// wave.  The user's offsets decide the unit in one round trip: an empty
+// user is zero-filled; for the others cta_of_row gives the CTAs that hold
+// the first and the last row (pure arithmetic on the two offsets), and if
+// they differ the user is split and the unit sums its slots: 2c for each
+// later CTA c (the user starts before their ranges), and for the first CTA
+// slot 2c if that CTA's range starts at the user's first row, else 2c + 1.
+// That last choice has a closed form when the user before is not empty;
+// otherwise warp 0 searches the range start while every thread's slot
+// loads are in flight.  The validation bits are taken by the first unit of
+// each user.
 #include "sa_internal.h"
 #include "sa_ptx.cuh"
 
