@@ -109,6 +109,8 @@ __global__ void __launch_bounds__(kFinThreads, kFinBlocksPerSm)
 #pragma unroll
       for (int t = 0; t < kFinBatch; ++t) {
         const int64_t cc = c_lo + 1 + t;
+        xv[t] = zero;  // threads past the sketch's end add zeros (and store nothing)
+        mv[t] = 0.f;
         if (cc <= c_hi) {
           if (has_x) xv[t] = *reinterpret_cast<const float4*>(a.part_x + (2 * cc) * kd + i);
           if (has_m) mv[t] = a.part_m[(2 * cc) * k + j];
